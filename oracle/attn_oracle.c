@@ -1,0 +1,377 @@
+/*
+ * Exact-attention oracle: plain, slow, fp64 CPU reference.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header or constant with the CUDA path, and the CUDA path never calls it.
+ *
+ * What it computes (the plain definition, written out):
+ *   "Hardware-Aware FP4 FlashAttention-4", section "Planteamiento del
+ *   Problema": attention is the product QK^T, a row softmax of the scores,
+ *   then the product PV.  Section "Causal Backward Cuantizado": the forward
+ *   keeps the per-row log-sum-exp normaliser (LSE) and the backward rebuilds
+ *   the probabilities from it.  "FlashAttention-4发布", section "从V1到V4",
+ *   first bullet: the tiled method is exact -- it reaches this same result
+ *   without writing the N x N matrix -- so the oracle is the untiled
+ *   definition, computed row by row with a two-pass softmax (deliberately not
+ *   the online form).  Masks follow the patterns named in "El FlexAttention
+ *   de PyTorch con FlashAttention-4", intro (sliding window, document
+ *   masking) plus causal; grouped heads follow the FlashAttention-2 bullet of
+ *   "从V1到V4" (GQA/MQA).
+ *
+ * Readings where the pages say nothing (each also listed in the design notes):
+ *   - causal alignment when Sq != Sk is bottom-right: key j allowed for query
+ *     i iff j <= i + (Sk - Sq);
+ *   - window: allowed iff i+(Sk-Sq)-window_left <= j <= i+(Sk-Sq)+window_right,
+ *     a negative bound meaning unbounded on that side;
+ *   - document mask: token t belongs to document d iff
+ *     offsets[d] <= t < offsets[d+1]; query i may see key j only if both lie
+ *     in the same document.  It combines (AND) with causal and window;
+ *   - grouped heads: query head hq reads key/value head hq / (Hq / Hkv);
+ *   - a row with no allowed key has O = 0 and LSE = -inf.
+ *
+ * Parity pins (tests, CPU only): closed forms (equal logits -> mean of V,
+ * one dominant logit -> that V row, constant V -> rows of P sum to one,
+ * causal row 0), library softmax / logsumexp on dense masked scores, mask
+ * and GQA invariants, finite differences for the backward.  Nothing here is
+ * "parity unpinned".
+ *
+ * Layouts (row-major, contiguous):
+ *   q, o, dq, do : [B, Sq, Hq,  D]
+ *   k, v, dk, dv : [B, Sk, Hkv, D]
+ *   lse          : [B, Hq, Sq]
+ * Inputs are either bf16 bit patterns (uint16) converted exactly to double,
+ * or doubles (used by the finite-difference tests).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+typedef struct {
+    int B, Hq, Hkv, Sq, Sk, D;
+    double scale;
+    int causal, window_left, window_right;
+    const int *doc_offsets; /* host int32[num_docs + 1] or NULL */
+    int num_docs;
+} oracle_shape_t;
+
+/* ------------------------------------------------------------------ input */
+
+static double bf16_bits_to_double(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16; /* bf16 is the top half of an fp32 */
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Copy D elements starting at element index `idx` into `out` as doubles. */
+static void load_vec(const void *base, int is_bf16, size_t idx, int D, double *out) {
+    if (is_bf16) {
+        const uint16_t *p = (const uint16_t *)base + idx;
+        for (int d = 0; d < D; ++d) out[d] = bf16_bits_to_double(p[d]);
+    } else {
+        const double *p = (const double *)base + idx;
+        for (int d = 0; d < D; ++d) out[d] = p[d];
+    }
+}
+
+static size_t q_index(const oracle_shape_t *s, int b, int i, int h) {
+    return (((size_t)b * s->Sq + i) * s->Hq + h) * s->D;
+}
+static size_t kv_index(const oracle_shape_t *s, int b, int j, int h) {
+    return (((size_t)b * s->Sk + j) * s->Hkv + h) * s->D;
+}
+
+/* ------------------------------------------------------------------- mask */
+
+/* Document of token t, or -1 when t lies outside every document. */
+static int document_of(const oracle_shape_t *s, long t) {
+    for (int d = 0; d < s->num_docs; ++d)
+        if (s->doc_offsets[d] <= t && t < s->doc_offsets[d + 1]) return d;
+    return -1;
+}
+
+/* The mask predicate, written directly from its definition. */
+static int key_allowed(const oracle_shape_t *s, long i, long j) {
+    long diag = i + (long)(s->Sk - s->Sq);
+    if (s->causal && j > diag) return 0;
+    if (s->window_left >= 0 && j < diag - s->window_left) return 0;
+    if (s->window_right >= 0 && j > diag + s->window_right) return 0;
+    if (s->doc_offsets) {
+        int di = document_of(s, i);
+        if (di < 0 || di != document_of(s, j)) return 0;
+    }
+    return 1;
+}
+
+static int kv_head_of(const oracle_shape_t *s, int hq) {
+    return hq / (s->Hq / s->Hkv);
+}
+
+/* --------------------------------------------------------------- forward */
+
+/*
+ * One query row.  Scores s_j = scale * <q_i, k_j> for allowed j; two passes:
+ * M = max_j s_j, Z = sum_j exp(s_j - M); LSE = M + log Z;
+ * P_j = exp(s_j - LSE); O = sum_j P_j v_j.
+ * Work buffers: s (Sk), qi/kj (D).  kd/vd hold this head's K and V rows
+ * already converted to double ([Sk][D]).
+ */
+static void forward_row(const oracle_shape_t *s, const double *qi,
+                        const double *kd, const double *vd, long i,
+                        double *srow, unsigned char *allow,
+                        double *o_out, double *lse_out) {
+    const int D = s->D, Sk = s->Sk;
+    double M = -INFINITY;
+    long n_allowed = 0;
+    for (long j = 0; j < Sk; ++j) {
+        allow[j] = (unsigned char)key_allowed(s, i, j);
+        if (!allow[j]) continue;
+        const double *kj = kd + (size_t)j * D;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += qi[d] * kj[d];
+        srow[j] = s->scale * dot;
+        if (srow[j] > M) M = srow[j];
+        ++n_allowed;
+    }
+    for (int d = 0; d < D; ++d) o_out[d] = 0.0;
+    if (n_allowed == 0) {
+        *lse_out = -INFINITY;
+        return;
+    }
+    double Z = 0.0;
+    for (long j = 0; j < Sk; ++j)
+        if (allow[j]) Z += exp(srow[j] - M);
+    const double lse = M + log(Z);
+    for (long j = 0; j < Sk; ++j) {
+        if (!allow[j]) continue;
+        const double p = exp(srow[j] - lse);
+        const double *vj = vd + (size_t)j * D;
+        for (int d = 0; d < D; ++d) o_out[d] += p * vj[d];
+    }
+    *lse_out = lse;
+}
+
+/* Convert the K and V rows of one (b, hkv) head to double, [Sk][D]. */
+static void load_head(const oracle_shape_t *s, const void *k, const void *v,
+                      int in_bf16, int b, int hkv, double *kd, double *vd) {
+    for (int j = 0; j < s->Sk; ++j) {
+        load_vec(k, in_bf16, kv_index(s, b, j, hkv), s->D, kd + (size_t)j * s->D);
+        load_vec(v, in_bf16, kv_index(s, b, j, hkv), s->D, vd + (size_t)j * s->D);
+    }
+}
+
+static int shape_ok(const oracle_shape_t *s) {
+    if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->Sq < 1 || s->Sk < 1 || s->D < 1)
+        return 0;
+    if (s->Hq % s->Hkv != 0) return 0;
+    if (s->doc_offsets && s->num_docs < 1) return 0;
+    return 1;
+}
+
+/*
+ * Forward.  rows == NULL: every row; o is [B,Sq,Hq,D], lse is [B,Hq,Sq].
+ * rows != NULL: n_rows triples (b, hq, i); o is [n_rows, D], lse [n_rows].
+ * Returns 0 on success, -1 on a bad shape, -2 on allocation failure.
+ */
+static int attn_fwd_core(const oracle_shape_t *s, const void *q, const void *k,
+                         const void *v, int in_bf16, double *o, double *lse,
+                         const int64_t *rows, int64_t n_rows) {
+    if (!shape_ok(s)) return -1;
+    const int D = s->D;
+    const size_t head_elems = (size_t)s->Sk * D;
+    double *kd = (double *)malloc(head_elems * sizeof(double));
+    double *vd = (double *)malloc(head_elems * sizeof(double));
+    if (!kd || !vd) { free(kd); free(vd); return -2; }
+    int status = 0;
+
+    for (int b = 0; b < s->B && status == 0; ++b) {
+        for (int hkv = 0; hkv < s->Hkv && status == 0; ++hkv) {
+            /* Skip heads no requested row touches. */
+            if (rows) {
+                int used = 0;
+                for (int64_t r = 0; r < n_rows && !used; ++r)
+                    used = rows[3 * r] == b && kv_head_of(s, (int)rows[3 * r + 1]) == hkv;
+                if (!used) continue;
+            }
+            load_head(s, k, v, in_bf16, b, hkv, kd, vd);
+            const int group = s->Hq / s->Hkv;
+            const int64_t n_items = rows ? n_rows : (int64_t)group * s->Sq;
+#pragma omp parallel
+            {
+                double *srow = (double *)malloc((size_t)s->Sk * sizeof(double));
+                unsigned char *allow = (unsigned char *)malloc((size_t)s->Sk);
+                double *qi = (double *)malloc((size_t)D * sizeof(double));
+                if (!srow || !allow || !qi) {
+#pragma omp atomic write
+                    status = -2;
+                } else {
+#pragma omp for schedule(dynamic, 16)
+                    for (int64_t it = 0; it < n_items; ++it) {
+                        int hq, i;
+                        double *o_dst, *lse_dst;
+                        if (rows) {
+                            if (rows[3 * it] != b || kv_head_of(s, (int)rows[3 * it + 1]) != hkv)
+                                continue;
+                            hq = (int)rows[3 * it + 1];
+                            i = (int)rows[3 * it + 2];
+                            o_dst = o + (size_t)it * D;
+                            lse_dst = lse + it;
+                        } else {
+                            hq = hkv * group + (int)(it / s->Sq);
+                            i = (int)(it % s->Sq);
+                            o_dst = o + q_index(s, b, i, hq);
+                            lse_dst = lse + ((size_t)b * s->Hq + hq) * s->Sq + i;
+                        }
+                        load_vec(q, in_bf16, q_index(s, b, i, hq), D, qi);
+                        forward_row(s, qi, kd, vd, i, srow, allow, o_dst, lse_dst);
+                    }
+                }
+                free(srow);
+                free(allow);
+                free(qi);
+            }
+        }
+    }
+    free(kd);
+    free(vd);
+    return status;
+}
+
+/* -------------------------------------------------------------- backward */
+
+/*
+ * Backward of L = sum(O * dO) for one (b, hkv) group, from the definition:
+ *   P_ij  = exp(s_ij - LSE_i)                (rebuilt from the forward's LSE)
+ *   D_i   = sum_d dO_id * O_id               (O from this oracle's forward)
+ *   dV_j += sum_i P_ij dO_i
+ *   dP_ij = <dO_i, v_j>
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j += scale * sum_i dS_ij q_i
+ * dK and dV sum over the Hq/Hkv query heads of the group.  ("Hardware-Aware
+ * FP4 FlashAttention-4", section "Causal Backward Cuantizado": the backward
+ * reconstructs the probabilities from the saved LSE.)
+ */
+static int attn_bwd_core(const oracle_shape_t *s, const void *q, const void *k,
+                         const void *v, const void *dout, int in_bf16,
+                         double *dq, double *dk, double *dv,
+                         double *o_opt, double *lse_opt) {
+    if (!shape_ok(s)) return -1;
+    const int D = s->D, Sq = s->Sq, Sk = s->Sk;
+    const int group = s->Hq / s->Hkv;
+    int status = 0;
+
+    memset(dq, 0, (size_t)s->B * Sq * s->Hq * D * sizeof(double));
+    memset(dk, 0, (size_t)s->B * Sk * s->Hkv * D * sizeof(double));
+    memset(dv, 0, (size_t)s->B * Sk * s->Hkv * D * sizeof(double));
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < s->B; ++b) {
+        for (int hkv = 0; hkv < s->Hkv; ++hkv) {
+            const size_t head_elems = (size_t)Sk * D;
+            double *kd = (double *)malloc(head_elems * sizeof(double));
+            double *vd = (double *)malloc(head_elems * sizeof(double));
+            double *srow = (double *)malloc((size_t)Sk * sizeof(double));
+            unsigned char *allow = (unsigned char *)malloc((size_t)Sk);
+            double *qi = (double *)malloc((size_t)D * sizeof(double));
+            double *doi = (double *)malloc((size_t)D * sizeof(double));
+            double *oi = (double *)malloc((size_t)D * sizeof(double));
+            if (!kd || !vd || !srow || !allow || !qi || !doi || !oi) {
+#pragma omp atomic write
+                status = -2;
+            } else {
+                load_head(s, k, v, in_bf16, b, hkv, kd, vd);
+                for (int g = 0; g < group; ++g) {
+                    const int hq = hkv * group + g;
+                    for (int i = 0; i < Sq; ++i) {
+                        double lse;
+                        load_vec(q, in_bf16, q_index(s, b, i, hq), D, qi);
+                        load_vec(dout, in_bf16, q_index(s, b, i, hq), D, doi);
+                        forward_row(s, qi, kd, vd, i, srow, allow, oi, &lse);
+                        if (o_opt)
+                            memcpy(o_opt + q_index(s, b, i, hq), oi, (size_t)D * sizeof(double));
+                        if (lse_opt) lse_opt[((size_t)b * s->Hq + hq) * Sq + i] = lse;
+                        if (isinf(lse)) continue; /* no allowed key: zero gradient */
+                        double Di = 0.0;
+                        for (int d = 0; d < D; ++d) Di += doi[d] * oi[d];
+                        double *dqi = dq + q_index(s, b, i, hq);
+                        for (int j = 0; j < Sk; ++j) {
+                            if (!allow[j]) continue;
+                            const double *kj = kd + (size_t)j * D;
+                            const double *vj = vd + (size_t)j * D;
+                            const double p = exp(srow[j] - lse);
+                            double dp = 0.0;
+                            for (int d = 0; d < D; ++d) dp += doi[d] * vj[d];
+                            const double ds = p * (dp - Di);
+                            double *dkj = dk + kv_index(s, b, j, hkv);
+                            double *dvj = dv + kv_index(s, b, j, hkv);
+                            for (int d = 0; d < D; ++d) {
+                                dvj[d] += p * doi[d];
+                                dqi[d] += s->scale * ds * kj[d];
+                                dkj[d] += s->scale * ds * qi[d];
+                            }
+                        }
+                    }
+                }
+            }
+            free(kd); free(vd); free(srow); free(allow); free(qi); free(doi); free(oi);
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------ public API */
+
+#define ORACLE_SHAPE                                                        \
+    oracle_shape_t s = {B, Hq, Hkv, Sq, Sk, D, scale, causal, window_left,  \
+                        window_right, doc_offsets, num_docs}
+
+int oracle_attn_fwd_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         double *o, double *lse, int B, int Hq, int Hkv, int Sq,
+                         int Sk, int D, double scale, int causal, int window_left,
+                         int window_right, const int *doc_offsets, int num_docs,
+                         const int64_t *rows, int64_t n_rows) {
+    ORACLE_SHAPE;
+    return attn_fwd_core(&s, q, k, v, 1, o, lse, rows, n_rows);
+}
+
+int oracle_attn_fwd_f64(const double *q, const double *k, const double *v,
+                        double *o, double *lse, int B, int Hq, int Hkv, int Sq,
+                        int Sk, int D, double scale, int causal, int window_left,
+                        int window_right, const int *doc_offsets, int num_docs,
+                        const int64_t *rows, int64_t n_rows) {
+    ORACLE_SHAPE;
+    return attn_fwd_core(&s, q, k, v, 0, o, lse, rows, n_rows);
+}
+
+int oracle_attn_bwd_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         const uint16_t *dout, double *dq, double *dk, double *dv,
+                         double *o, double *lse, int B, int Hq, int Hkv, int Sq,
+                         int Sk, int D, double scale, int causal, int window_left,
+                         int window_right, const int *doc_offsets, int num_docs) {
+    ORACLE_SHAPE;
+    return attn_bwd_core(&s, q, k, v, dout, 1, dq, dk, dv, o, lse);
+}
+
+int oracle_attn_bwd_f64(const double *q, const double *k, const double *v,
+                        const double *dout, double *dq, double *dk, double *dv,
+                        double *o, double *lse, int B, int Hq, int Hkv, int Sq,
+                        int Sk, int D, double scale, int causal, int window_left,
+                        int window_right, const int *doc_offsets, int num_docs) {
+    ORACLE_SHAPE;
+    return attn_bwd_core(&s, q, k, v, dout, 0, dq, dk, dv, o, lse);
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
