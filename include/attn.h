@@ -1,0 +1,131 @@
+/*
+ * tiled_attention_blackwell_b200 -- C ABI of a fused, IO-aware exact
+ * attention library for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Hardware-Aware FP4 FlashAttention-4", section
+ * "Planteamiento del Problema": the product QK^T, a row softmax, the product
+ * PV; section "Causal Backward Cuantizado": the forward keeps the per-row
+ * log-sum-exp; "FlashAttention-4发布", section "从V1到V4", first bullet: the
+ * result is computed tile by tile so the N x N score matrix never reaches
+ * HBM):
+ *
+ *   for every batch b, query head hq, query row i:
+ *     hkv      = hq / (Hq / Hkv)                       (grouped heads, GQA/MQA)
+ *     s_ij     = scale * <q[b,i,hq,:], k[b,j,hkv,:]>   for allowed keys j
+ *     LSE[b,hq,i] = log sum_j exp(s_ij)                (natural log, fp32)
+ *     O[b,i,hq,:] = sum_j exp(s_ij - LSE) * v[b,j,hkv,:]   (bf16, RN)
+ *
+ *   Key j is allowed for query i (shift = Sk - Sq, bottom-right alignment):
+ *     causal != 0        :  j <= i + shift
+ *     window_left  >= 0  :  j >= i + shift - window_left
+ *     window_right >= 0  :  j <= i + shift + window_right
+ *     doc_offsets != NULL:  i and j lie in the same document, where token t
+ *                           belongs to document d iff
+ *                           doc_offsets[d] <= t < doc_offsets[d+1]
+ *   (the sliding-window and document masks are two of the patterns named in
+ *   "El FlexAttention de PyTorch con FlashAttention-4", intro).  A row with
+ *   no allowed key gets O = 0 and LSE = -inf.
+ *
+ * Memory layout (all contiguous, row-major, device memory owned by the
+ * caller; the library allocates nothing per call):
+ *   q, o : bf16 [B, Sq, Hq,  D]
+ *   k, v : bf16 [B, Sk, Hkv, D]
+ *   lse  : fp32 [B, Hq, Sq]
+ *   doc_offsets : int32 [num_docs + 1] in device memory, shared by all
+ *                 batches; must be non-decreasing with doc_offsets[0] = 0 and
+ *                 doc_offsets[num_docs] = Sq.  Malformed offsets give
+ *                 unspecified output values but never out-of-bounds access.
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t, NULL = the legacy
+ * default stream).  Argument errors are reported before anything is
+ * launched.  A kernel that gives up waiting (every device-side wait is
+ * bounded) records ATTN_ERR_DEVICE_TIMEOUT in a per-device status word,
+ * read back with attn_get_device_status().
+ */
+#ifndef TILED_ATTENTION_B200_ATTN_H
+#define TILED_ATTENTION_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ATTN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,    /* bad shape, null pointer, bad mask argument */
+    ATTN_ERR_UNSUPPORTED = 2,    /* valid request outside what is built (e.g. D) */
+    ATTN_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned */
+    ATTN_ERR_LAUNCH = 4,         /* the CUDA launch itself failed */
+    ATTN_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait expired */
+    ATTN_ERR_CUDA = 6            /* another CUDA runtime error (see detail) */
+} attn_status_t;
+
+/* Tuning knobs of the forward.  Pass NULL for the defaults.  None of them
+ * changes the mathematical result, only rounding. */
+typedef struct {
+    /* Online-softmax rescale threshold in log2 units ("La ventaja técnica" of
+     * the ainvest.com FlashAttention-4 page: rescale only when the running
+     * maximum moves significantly).  The running max of a row, and with it
+     * the output accumulator, is updated only when a new block raises the
+     * row maximum by more than this amount; in between, unnormalised
+     * probabilities may reach 2^threshold.  0 = classic online softmax.
+     * Valid range [0, 16].  Default 8. */
+    float rescale_threshold;
+    /* exp2 evaluation ("La ventaja técnica": part of the exponentials run as
+     * a cubic polynomial on the FMA units instead of the special-function
+     * units).  0 = all on the MUFU ex2 unit; 1 = the tuned split
+     * (default); 2 = every column of unmasked tiles by polynomial. */
+    int exp2_mode;
+    int reserved[6]; /* must be zero */
+} attn_fwd_options_t;
+
+/* Fills *opts with the defaults. */
+ATTN_API void attn_fwd_default_options(attn_fwd_options_t *opts);
+
+/*
+ * Forward: O and LSE.  D must be 64 or 128; Hq % Hkv == 0; Sq, Sk >= 1;
+ * scale > 0 and finite; window bounds -1 (unbounded) or >= 0; a document
+ * mask requires Sq == Sk and num_docs >= 1.  q, k, v, o must be 16-byte
+ * aligned.  Returns ATTN_OK once the kernel is enqueued.
+ */
+ATTN_API attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                       int causal, int window_left, int window_right,
+                       const int *doc_offsets, int num_docs, void *stream);
+
+/* attn_fwd with explicit tuning options (NULL = defaults). */
+ATTN_API attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                          int causal, int window_left, int window_right,
+                          const int *doc_offsets, int num_docs,
+                          const attn_fwd_options_t *opts, void *stream);
+
+/* Synchronises `stream`, then reads and clears the device status word of
+ * the current device.  Returns ATTN_OK or ATTN_ERR_DEVICE_TIMEOUT (or
+ * ATTN_ERR_CUDA if the synchronisation itself failed). */
+ATTN_API attn_status_t attn_get_device_status(void *stream);
+
+/* Static description of a status code. */
+ATTN_API const char *attn_status_string(attn_status_t status);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+ATTN_API const char *attn_last_error_detail(void);
+
+/* ATTN_ABI_VERSION of the built library. */
+ATTN_API int attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TILED_ATTENTION_B200_ATTN_H */

@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library builds with nvcc here, loads without a GPU, exports every entry
+point the header declares, and rejects bad arguments before touching CUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from tiled_attention_blackwell_b200 import attn, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return attn.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]*?\b(attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert "attn_fwd" in names and "attn_get_device_status" in names
+    assert set(attn.EXPORTED) <= set(names)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    out = os.popen(f"nm -D --defined-only {attn.library_path()}").read()
+    exported = set(re.findall(r"\b(attn_\w+)\b", out))
+    assert set(declared_functions()) == exported
+
+
+def test_status_strings_and_version(L):
+    assert L.attn_abi_version() == 1
+    for code in range(7):
+        s = L.attn_status_string(code).decode()
+        assert s and s != "unknown status"
+    assert L.attn_status_string(99).decode() == "unknown status"
+
+
+def test_default_options(L):
+    o = attn.default_options()
+    assert o.rescale_threshold == 8.0 and o.exp2_mode == 1 and list(o.reserved) == [0] * 6
+
+
+# Fake, 16-byte-aligned device addresses: validation must reject the call
+# before any CUDA call, so nothing ever dereferences them.
+P = 0x10000
+
+
+def call(L, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, Hq=2, Hkv=2, Sq=16, Sk=16, D=128, scale=0.1,
+             causal=0, wl=-1, wr=-1, docs=None, nd=0, opts=None)
+    a.update(kw)
+    args = [ctypes.c_void_p(a["q"]), ctypes.c_void_p(a["k"]), ctypes.c_void_p(a["v"]),
+            ctypes.c_void_p(a["o"]), ctypes.c_void_p(a["lse"]), a["B"], a["Hq"], a["Hkv"],
+            a["Sq"], a["Sk"], a["D"], a["scale"], a["causal"], a["wl"], a["wr"],
+            ctypes.c_void_p(a["docs"]) if a["docs"] else None, a["nd"]]
+    if a["opts"] is None:
+        return L.attn_fwd(*args, None)
+    return L.attn_fwd_ex(*args, ctypes.byref(a["opts"]), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(lse=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(B=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Sq=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Sk=-3), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), attn.ATTN_ERR_INVALID_ARG),
+    (dict(D=96), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(D=256), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=0.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(scale=-1.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), attn.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), attn.ATTN_ERR_INVALID_ARG),
+    (dict(wl=-2), attn.ATTN_ERR_INVALID_ARG),
+    (dict(wr=-5), attn.ATTN_ERR_INVALID_ARG),
+    (dict(docs=P, nd=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(docs=None, nd=3), attn.ATTN_ERR_INVALID_ARG),
+    (dict(docs=P, nd=2, Sk=32), attn.ATTN_ERR_INVALID_ARG),
+    (dict(q=P + 8), attn.ATTN_ERR_MISALIGNED),
+    (dict(v=P + 2), attn.ATTN_ERR_MISALIGNED),
+    (dict(o=P + 4), attn.ATTN_ERR_MISALIGNED),
+    (dict(lse=P + 2), attn.ATTN_ERR_MISALIGNED),
+])
+def test_invalid_arguments_rejected_before_launch(L, kw, status):
+    assert call(L, **kw) == status
+    assert L.attn_last_error_detail().decode() != ""
+
+
+@pytest.mark.parametrize("field,value", [("rescale_threshold", -1.0),
+                                         ("rescale_threshold", 17.0),
+                                         ("rescale_threshold", float("nan")),
+                                         ("exp2_mode", 3), ("exp2_mode", -1)])
+def test_invalid_options_rejected(L, field, value):
+    opts = attn.default_options()
+    setattr(opts, field, value)
+    assert call(L, opts=opts) == attn.ATTN_ERR_INVALID_ARG
+
+
+def test_reserved_options_must_be_zero(L):
+    opts = attn.default_options()
+    opts.reserved[2] = 1
+    assert call(L, opts=opts) == attn.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
+def test_valid_call_without_gpu_reports_cuda_error(L):
+    assert call(L) == attn.ATTN_ERR_CUDA
+
+
+def test_binding_refuses_cpu_tensors(L):
+    q = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 1, 4)
+    with pytest.raises(TypeError):
+        attn.attn_fwd(q, q, q, q, lse, scale=0.1)

@@ -1,0 +1,195 @@
+"""GPU parity of the attention forward against the fp64 oracle.
+
+Every case runs the CUDA path through the C ABI and compares, element by
+element, with the oracle on the same seeded bf16 inputs.  Tolerances (fixed
+for this operation): O max-abs error <= 2e-2 and mean-abs error <= 2e-3;
+LSE abs error <= 1e-3; rows with no allowed key must give O = 0 and
+LSE = -inf exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tiled_attention_blackwell_b200 import attn, build
+from tiled_attention_blackwell_b200.workloads import WORKLOADS, make_inputs, make_tensors
+
+pytestmark = pytest.mark.gpu
+
+O_MAX, O_MEAN, LSE_TOL = 2e-2, 2e-3, 1e-3
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    build.build()
+    attn.lib()
+    yield
+    assert attn.device_status() == attn.ATTN_OK
+
+
+def run_gpu(t, *, causal=False, window=None, doc_offsets=None, scale=None, options=None):
+    q, k, v = (t[n].to(DEV) for n in ("q", "k", "v"))
+    docs = None if doc_offsets is None else torch.as_tensor(doc_offsets, dtype=torch.int32,
+                                                             device=DEV)
+    o, lse = attn.attention(q, k, v, scale=scale, causal=causal, window=window,
+                            doc_offsets=docs, options=options)
+    torch.cuda.synchronize()
+    return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def check(o, lse, o_ref, lse_ref, what=""):
+    assert not np.isnan(o).any(), f"{what}: NaN in O"
+    empty = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), empty), f"{what}: -inf rows differ"
+    err = np.abs(o - o_ref)
+    assert err.max() <= O_MAX, f"{what}: O max-abs {err.max():.3e}"
+    assert err.mean() <= O_MEAN, f"{what}: O mean-abs {err.mean():.3e}"
+    lse_err = np.abs(np.where(empty, 0.0, lse - lse_ref))
+    assert lse_err.max() <= LSE_TOL, f"{what}: LSE abs {lse_err.max():.3e}"
+    if empty.any():
+        # rows with no key: O exactly zero (LSE layout [B,H,S] vs O [B,S,H,D])
+        b, h, i = np.nonzero(empty)
+        assert np.all(o[b, i, h] == 0.0), f"{what}: empty rows not zero"
+
+
+def full_case(B, Hq, Hkv, Sq, Sk, D, seed, *, causal=False, window=None, doc_offsets=None,
+              options=None, qk_std=1.0, outliers=0.0):
+    t = make_tensors(B, Hq, Hkv, Sq, Sk, D, seed, qk_std=qk_std, k_outlier_frac=outliers)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = run_gpu(t, causal=causal, window=window, doc_offsets=doc_offsets, scale=scale,
+                     options=options)
+    o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=scale, causal=causal,
+                                     window=window, doc_offsets=doc_offsets)
+    check(o, lse, o_ref, lse_ref, f"B{B} Hq{Hq} Hkv{Hkv} Sq{Sq} Sk{Sk} D{D}")
+
+
+# ------------------------------------------------------------------ configs
+
+def test_tiny_d64_workload_full():
+    w = WORKLOADS["tiny_d64"]
+    t = make_inputs(w)
+    o, lse = run_gpu(t, causal=w.causal, scale=w.scale)
+    o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=w.scale, causal=w.causal)
+    check(o, lse, o_ref, lse_ref, "tiny_d64")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("S", [1, 5, 127, 128, 129, 255, 256, 257, 700])
+@pytest.mark.parametrize("causal", [False, True])
+def test_shapes_and_ragged_tails(D, S, causal):
+    full_case(2, 2, 2, S, S, D, seed=100 + S, causal=causal)
+
+
+@pytest.mark.parametrize("heads", [(4, 1), (4, 2), (6, 3), (8, 8)])
+@pytest.mark.parametrize("D", [64, 128])
+def test_grouped_heads(heads, D):
+    full_case(2, heads[0], heads[1], 520, 520, D, seed=7, causal=True)
+
+
+@pytest.mark.parametrize("window", [(0, 0), (37, 50), (100, 0), (300, -1), (-1, 90), (5, 400)])
+def test_sliding_window(window):
+    full_case(1, 2, 2, 900, 900, 128, seed=11, window=window)
+    full_case(1, 2, 1, 600, 600, 64, seed=12, window=window, causal=True)
+
+
+@pytest.mark.parametrize("docs", [[0, 700], [0, 1, 2, 300, 301, 700], [0, 128, 256, 640, 700],
+                                  [0, 97, 400, 401, 555, 700]])
+@pytest.mark.parametrize("causal", [True, False])
+def test_document_mask(docs, causal):
+    full_case(2, 4, 2, 700, 700, 128, seed=13, doc_offsets=docs, causal=causal)
+
+
+@pytest.mark.parametrize("Sq,Sk", [(300, 1000), (1000, 300), (1, 777), (777, 1), (129, 1025)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_unequal_lengths_bottom_right(Sq, Sk, causal):
+    full_case(1, 2, 2, Sq, Sk, 128, seed=21, causal=causal)
+
+
+@pytest.mark.parametrize("tau", [0.0, 8.0, 16.0])
+@pytest.mark.parametrize("exp2_mode", [0, 1, 2])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rescale_threshold_and_exp2_split(tau, exp2_mode, causal):
+    opts = attn.default_options(rescale_threshold=tau, exp2_mode=exp2_mode)
+    full_case(2, 2, 2, 1000, 1000, 128, seed=31, causal=causal, options=opts, qk_std=1.5,
+              outliers=0.01)
+
+
+def test_large_logits_stay_finite():
+    """Logits far from zero (|s| up to hundreds) must not overflow or underflow."""
+    t = make_tensors(1, 2, 2, 600, 600, 128, seed=41, qk_std=4.0)
+    for exp2_mode in (0, 2):
+        opts = attn.default_options(exp2_mode=exp2_mode)
+        o, lse = run_gpu(t, causal=True, scale=1 / math.sqrt(128), options=opts)
+        o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=1 / math.sqrt(128),
+                                         causal=True)
+        check(o, lse, o_ref, lse_ref, f"large logits exp2_mode={exp2_mode}")
+
+
+# -------------------------------------------------------- memory discipline
+
+def test_writes_stay_in_bounds_and_cover_every_row():
+    B, H, S, D = 2, 3, 333, 128
+    t = make_tensors(B, H, H, S, S, D, seed=51)
+    q, k, v = (t[n].to(DEV) for n in ("q", "k", "v"))
+    n_o, n_l, guard = B * S * H * D, B * H * S, 4096
+    o_buf = torch.full((n_o + guard,), float("nan"), dtype=torch.bfloat16, device=DEV)
+    l_buf = torch.full((n_l + guard,), float("nan"), dtype=torch.float32, device=DEV)
+    o = o_buf[:n_o].view(B, S, H, D)
+    lse = l_buf[:n_l].view(B, H, S)
+    attn.attn_fwd(q, k, v, o, lse, scale=0.1, causal=True)
+    torch.cuda.synchronize()
+    assert not torch.isnan(o).any() and not torch.isnan(lse).any()
+    assert torch.isnan(o_buf[n_o:]).all() and torch.isnan(l_buf[n_l:]).all()
+
+
+def test_deterministic_and_stream_aware():
+    t = make_tensors(1, 4, 2, 1000, 1000, 128, seed=61)
+    q, k, v = (t[n].to(DEV) for n in ("q", "k", "v"))
+    o1, l1 = attn.attention(q, k, v, causal=True)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o2, l2 = attn.attention(q, k, v, causal=True, stream=s)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ------------------------------------------- full-size workloads (sampled)
+
+def sample_rows(B, H, S, n_random, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 2, 127, 128, 129, 255, 256, S // 2, S - 257, S - 129, S - 2, S - 1]
+    rows = []
+    for b in range(B):
+        for h in sorted({0, H - 1, int(rng.integers(H))}):
+            for i in fixed:
+                rows.append((b, h, i))
+    for _ in range(n_random):
+        rows.append((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(S))))
+    return np.array(rows, dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", ["outlier_s4096", "causal_s8192", "gqa_doc_s16384",
+                                  "causal_bwd_s4096"])
+def test_full_size_workload_sampled(name):
+    """The benchmark's workloads at full size, in the benchmark's launch
+    configuration: sampled rows against the oracle, plus properties of every
+    row (finite O, finite LSE: every row here has at least one key)."""
+    w = WORKLOADS[name]
+    t = make_inputs(w)
+    o, lse = run_gpu(t, causal=w.causal, doc_offsets=t["doc_offsets"], scale=w.scale)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    rows = sample_rows(w.B, w.Hq, w.S, 200, seed=w.seed)
+    o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=w.scale, causal=w.causal,
+                                     doc_offsets=t["doc_offsets"], rows=rows)
+    o_s = o[rows[:, 0], rows[:, 2], rows[:, 1]]
+    lse_s = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
+    err = np.abs(o_s - o_ref)
+    assert err.max() <= O_MAX, f"{name}: O max-abs {err.max():.3e}"
+    assert err.mean() <= O_MEAN, f"{name}: O mean-abs {err.mean():.3e}"
+    assert np.abs(lse_s - lse_ref).max() <= LSE_TOL

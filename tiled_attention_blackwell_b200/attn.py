@@ -1,0 +1,157 @@
+"""Python binding of the C ABI in ``include/attn.h`` (ctypes).
+
+Argument marshalling only: every step of the attention forward runs in the
+CUDA kernels of ``libattn.so``.  PyTorch supplies device memory and streams.
+There is no fallback: if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
+_lock = threading.Lock()
+_lib = None
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_MISALIGNED = 3
+ATTN_ERR_LAUNCH = 4
+ATTN_ERR_DEVICE_TIMEOUT = 5
+ATTN_ERR_CUDA = 6
+
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_default_options", "attn_get_device_status",
+            "attn_status_string", "attn_last_error_detail", "attn_abi_version")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class FwdOptions(ctypes.Structure):
+    """Mirror of attn_fwd_options_t."""
+    _fields_ = [("rescale_threshold", ctypes.c_float), ("exp2_mode", ctypes.c_int),
+                ("reserved", ctypes.c_int * 6)]
+
+
+_FWD_ARGS = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [ctypes.c_float] + \
+            [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libattn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is not built; run `python -m tiled_attention_blackwell_b200.build`")
+            L = ctypes.CDLL(_LIB_PATH)
+            L.attn_fwd.restype = ctypes.c_int
+            L.attn_fwd.argtypes = _FWD_ARGS + [ctypes.c_void_p]
+            L.attn_fwd_ex.restype = ctypes.c_int
+            L.attn_fwd_ex.argtypes = _FWD_ARGS + [ctypes.POINTER(FwdOptions), ctypes.c_void_p]
+            L.attn_fwd_default_options.restype = None
+            L.attn_fwd_default_options.argtypes = [ctypes.POINTER(FwdOptions)]
+            L.attn_get_device_status.restype = ctypes.c_int
+            L.attn_get_device_status.argtypes = [ctypes.c_void_p]
+            L.attn_status_string.restype = ctypes.c_char_p
+            L.attn_status_string.argtypes = [ctypes.c_int]
+            L.attn_last_error_detail.restype = ctypes.c_char_p
+            L.attn_last_error_detail.argtypes = []
+            L.attn_abi_version.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != ATTN_OK:
+        L = lib()
+        raise AttnError(status, f"{what}: {L.attn_status_string(status).decode()}"
+                                f" ({L.attn_last_error_detail().decode()})")
+
+
+def default_options(**overrides) -> FwdOptions:
+    opts = FwdOptions()
+    lib().attn_fwd_default_options(ctypes.byref(opts))
+    for k, v in overrides.items():
+        setattr(opts, k, v)
+    return opts
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def attn_fwd(q, k, v, o, lse, *, scale, causal=False, window=None, doc_offsets=None,
+             options=None, stream=None):
+    """Enqueue the forward on `stream` (default: torch's current stream).
+
+    q, o: bf16 CUDA [B,Sq,Hq,D]; k, v: bf16 CUDA [B,Sk,Hkv,D]; lse: fp32 CUDA
+    [B,Hq,Sq]; doc_offsets: int32 CUDA [num_docs+1] or None.  All contiguous.
+    """
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
+                        ("v", v, torch.bfloat16), ("o", o, torch.bfloat16),
+                        ("lse", lse, torch.float32)):
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA {dt} tensor")
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    if doc_offsets is not None:
+        if doc_offsets.dtype != torch.int32 or not doc_offsets.is_cuda:
+            raise TypeError("doc_offsets must be a CUDA int32 tensor")
+        docs_ptr, nd = _ptr(doc_offsets), doc_offsets.numel() - 1
+    else:
+        docs_ptr, nd = None, 0
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
+            float(scale), int(bool(causal)), wl, wr, docs_ptr, nd]
+    L = lib()
+    if options is None:
+        st = L.attn_fwd(*args, _stream_handle(stream))
+    else:
+        st = L.attn_fwd_ex(*args, ctypes.byref(options), _stream_handle(stream))
+    _check(st, "attn_fwd")
+
+
+def attention(q, k, v, *, scale=None, causal=False, window=None, doc_offsets=None,
+              options=None, stream=None):
+    """Allocate O and LSE with torch and run the forward.  Returns (O, LSE)."""
+    B, Sq, Hq, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if doc_offsets is not None and not torch.is_tensor(doc_offsets):
+        doc_offsets = torch.as_tensor(doc_offsets, dtype=torch.int32)
+    if doc_offsets is not None and not doc_offsets.is_cuda:
+        doc_offsets = doc_offsets.to(q.device)
+    attn_fwd(q, k, v, o, lse, scale=scale, causal=causal, window=window,
+             doc_offsets=doc_offsets, options=options, stream=stream)
+    return o, lse
+
+
+def device_status(stream=None) -> int:
+    """Synchronise `stream`, then read and clear the device status word."""
+    return lib().attn_get_device_status(_stream_handle(stream))
+
+
+def check_device_status(stream=None):
+    _check(device_status(stream), "device status")

@@ -1,0 +1,273 @@
+// C ABI of the attention library: argument validation, TMA descriptor
+// encoding, kernel selection and launch.  See include/attn.h for the
+// contract of every entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "fwd_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+thread_local char g_detail[512] = "";
+
+attn_status_t fail(attn_status_t status, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+attn_status_t ok() {
+    g_detail[0] = '\0';
+    return ATTN_OK;
+}
+
+// ------------------------------------------------------- device status word
+
+__device__ int g_status_word;
+
+struct DeviceState {
+    std::once_flag once;
+    cudaError_t init_error = cudaSuccess;
+    int *status = nullptr;  // device address of g_status_word
+    int num_sms = 0;
+};
+DeviceState g_devices[kMaxDevices];
+
+attn_status_t device_state(DeviceState **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(ATTN_ERR_UNSUPPORTED, "device index %d", dev);
+    DeviceState &st = g_devices[dev];
+    std::call_once(st.once, [&]() {
+        st.init_error = cudaGetSymbolAddress(reinterpret_cast<void **>(&st.status), g_status_word);
+        if (st.init_error == cudaSuccess)
+            st.init_error = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    });
+    if (st.init_error != cudaSuccess)
+        return fail(ATTN_ERR_CUDA, "device %d set-up: %s", dev, cudaGetErrorString(st.init_error));
+    *out = &st;
+    return ATTN_OK;
+}
+
+// ----------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, []() {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// bf16 tensor [B][S][H][D] as a 4-D map (D, S, H, B), box (64, 128, 1, 1),
+// 128-byte swizzle, zero fill out of bounds.
+attn_status_t make_map(CUtensorMap *map, const void *base, int B, int S, int H, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)H * D * 2, (cuuint64_t)D * 2,
+                                   (cuuint64_t)S * H * D * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)tab::kBlockM, 1, 1};
+    const cuuint32_t estride[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                    strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return ATTN_OK;
+}
+
+// --------------------------------------------------------------- launching
+
+template <int D, int NS, int EXP>
+attn_status_t launch_fwd(const tab::FwdParams &p, int grid, cudaStream_t stream) {
+    using Smem = tab::FwdSmem<D, NS>;
+    constexpr size_t smem = sizeof(Smem) + 1024;
+    static_assert(smem <= 232448, "shared memory budget");
+    auto kernel = tab::attn_fwd_kernel<D, NS, EXP>;
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t attr_err[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::call_once(once[dev], [&]() {
+        attr_err[dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+    });
+    if (attr_err[dev] != cudaSuccess)
+        return fail(ATTN_ERR_LAUNCH, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err[dev]));
+    kernel<<<grid, tab::kFwdThreads, smem, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ATTN_ERR_LAUNCH, "launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+constexpr int kStagesD128 = 4;
+constexpr int kStagesD64 = 8;
+
+template <int D, int NS>
+attn_status_t dispatch_exp(const tab::FwdParams &p, int grid, int exp_mode, cudaStream_t s) {
+    switch (exp_mode) {
+        case 0: return launch_fwd<D, NS, 0>(p, grid, s);
+        case 1: return launch_fwd<D, NS, 1>(p, grid, s);
+        default: return launch_fwd<D, NS, 2>(p, grid, s);
+    }
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+void attn_fwd_default_options(attn_fwd_options_t *opts) {
+    if (!opts) return;
+    *opts = attn_fwd_options_t{};
+    opts->rescale_threshold = 8.0f;
+    opts->exp2_mode = 1;
+}
+
+attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                          int causal, int window_left, int window_right,
+                          const int *doc_offsets, int num_docs,
+                          const attn_fwd_options_t *opts, void *stream) {
+    attn_fwd_options_t op;
+    attn_fwd_default_options(&op);
+    if (opts) op = *opts;
+
+    // ----- validation (no CUDA call before this block completes)
+    if (!q || !k || !v || !o || !lse)
+        return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1)
+        return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, Sq, Sk must be >= 1");
+    if (Hq % Hkv != 0)
+        return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (D != 64 && D != 128)
+        return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (built: 64, 128)", D);
+    if (!(scale > 0.0f) || !std::isfinite(scale))
+        return fail(ATTN_ERR_INVALID_ARG, "scale must be positive and finite");
+    if (window_left < -1 || window_right < -1)
+        return fail(ATTN_ERR_INVALID_ARG, "window bounds must be -1 or >= 0");
+    if ((doc_offsets == nullptr) != (num_docs == 0) || num_docs < 0)
+        return fail(ATTN_ERR_INVALID_ARG, "doc_offsets and num_docs must be given together");
+    if (doc_offsets && Sq != Sk)
+        return fail(ATTN_ERR_INVALID_ARG, "a document mask requires Sq == Sk");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(ATTN_ERR_MISALIGNED, "q, k, v, o must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+        return fail(ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
+    if (!(op.rescale_threshold >= 0.0f && op.rescale_threshold <= 16.0f))
+        return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must lie in [0, 16]");
+    if (op.exp2_mode < 0 || op.exp2_mode > 2)
+        return fail(ATTN_ERR_INVALID_ARG, "exp2_mode must be 0, 1 or 2");
+    for (int r : op.reserved)
+        if (r != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved option fields must be zero");
+    // TMA limits: every byte stride below 2^40.
+    const double max_stride = (double)std::max(Sq, Sk) * Hq * D * 2.0;
+    if (max_stride >= 1099511627776.0)
+        return fail(ATTN_ERR_UNSUPPORTED, "tensor too large for a TMA descriptor");
+    const long long num_qblocks = (Sq + 2LL * tab::kBlockM - 1) / (2LL * tab::kBlockM);
+    const long long grid = num_qblocks * Hq * B;
+    if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+
+    // ----- set-up
+    DeviceState *st = nullptr;
+    attn_status_t s = device_state(&st);
+    if (s != ATTN_OK) return s;
+
+    tab::FwdParams p;
+    memset(&p, 0, sizeof p);
+    if ((s = make_map(&p.tm_q, q, B, Sq, Hq, D)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_k, k, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_v, v, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.doc_offsets = doc_offsets;
+    p.num_docs = num_docs;
+    p.status = st->status;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.group = Hq / Hkv;
+    p.causal = causal ? 1 : 0;
+    p.window_left = window_left;
+    p.window_right = window_right;
+    p.num_qblocks = (int)num_qblocks;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.rescale_threshold = op.rescale_threshold;
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (D == 128) return dispatch_exp<128, kStagesD128>(p, (int)grid, op.exp2_mode, cs);
+    return dispatch_exp<64, kStagesD64>(p, (int)grid, op.exp2_mode, cs);
+}
+
+attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                       int causal, int window_left, int window_right,
+                       const int *doc_offsets, int num_docs, void *stream) {
+    return attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, window_left,
+                       window_right, doc_offsets, num_docs, nullptr, stream);
+}
+
+attn_status_t attn_get_device_status(void *stream) {
+    DeviceState *st = nullptr;
+    attn_status_t s = device_state(&st);
+    if (s != ATTN_OK) return s;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+    int word = 0;
+    e = cudaMemcpy(&word, st->status, sizeof word, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (word != 0) {
+        const int zero = 0;
+        e = cudaMemcpy(st->status, &zero, sizeof zero, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "status clear: %s", cudaGetErrorString(e));
+        return fail(static_cast<attn_status_t>(word), "device reported status %d", word);
+    }
+    return ok();
+}
+
+const char *attn_status_string(attn_status_t status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ATTN_ERR_MISALIGNED: return "misaligned pointer";
+        case ATTN_ERR_LAUNCH: return "kernel launch failed";
+        case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case ATTN_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+const char *attn_last_error_detail(void) { return g_detail; }
+
+int attn_abi_version(void) { return ATTN_ABI_VERSION; }
+
+}  // extern "C"

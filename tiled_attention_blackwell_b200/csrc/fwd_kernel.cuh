@@ -1,0 +1,541 @@
+// Fused exact-attention forward for B200 (sm_100a).
+//
+// One CTA owns two 128-row query tiles of one (batch, query head) -- the
+// 256 x 128 tile shape the FlexAttention page gives for Blackwell ("El
+// FlexAttention de PyTorch con FlashAttention-4", "Limitaciones actuales")
+// -- and streams the key/value blocks its mask allows through shared memory.
+// The two query tiles ping-pong between the tensor cores and the softmax
+// warps ("Hardware-Aware FP4 FlashAttention-4", "Metodología": the two-query
+// pipeline and its tensor-memory ownership protocol).
+//
+// Warp roles (384 threads):
+//   warps 0-3   softmax + correction + epilogue for query tile 0
+//   warps 4-7   the same for query tile 1
+//   warp  8     tcgen05 MMA issue (one thread) and TMEM allocation
+//   warp  9     TMA producer (one thread)
+//   warps 10-11 idle
+// The pipeline stages load -> MMA -> softmax -> correction -> epilogue of the
+// FA4 design ("La ventaja técnica", ainvest.com page) map onto these roles;
+// the correction (rescaling the output accumulator in TMEM) runs inside the
+// softmax warps because threshold gating makes it rare.
+//
+// Tensor memory (512 columns, fp32 cells, lane = query row):
+//   [  0,128) S0 = Q0 K^T   (P0 in bf16 pairs overwrites its first 64 columns)
+//   [128,256) S1 = Q1 K^T   (P1 likewise)
+//   [256,256+D) O0, then O1 -- the full 512-column budget at D = 128 that
+//   "Contribuciones Clave" / "Puntos Clave" of the FP4 page describe.
+//
+// Shared memory: Q0, Q1 and a ring of NS key/value slots, each a 128 x D
+// bf16 tile stored as D/64 column chunks of [128 rows][128 bytes] with the
+// 128-byte swizzle that both TMA and the tcgen05 descriptors use.
+//
+// Online softmax in log2 units: x = s * scale * log2(e).  Each row keeps a
+// running max m and sum l; a new block changes m (and rescales O and l) only
+// when it raises the row max by more than `rescale_threshold` ("La ventaja
+// técnica": rescale only when the max changes significantly; "为Blackwell
+// 而生的性能猛兽" item 1: most rescales are skipped).  Exponentials run on
+// the MUFU ex2 unit or as a cubic polynomial on the FMA pipe ("La ventaja
+// técnica"; "为Blackwell而生的性能猛兽" item 2).
+//
+// Every wait is bounded: on expiry the kernel records a timeout in the
+// device status word, lets its in-flight copies and MMAs finish, frees TMEM
+// and returns.
+#pragma once
+
+#include "exp2_poly.cuh"
+#include "ptx.cuh"
+
+namespace tab {
+
+constexpr int kBlockM = 128;   // query rows per tile = TMEM lanes
+constexpr int kBlockN = 128;   // keys per key/value block
+constexpr int kFwdThreads = 384;
+constexpr int kTmemCols = 512;
+constexpr int kSoftmaxRegs = 208;
+constexpr int kOtherRegs = 88;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kFwdThreads * 168,
+              "register split exceeds the launch allocation");
+constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
+constexpr int kStatusTimeout = 5;                   // ATTN_ERR_DEVICE_TIMEOUT
+
+struct FwdParams {
+    CUtensorMap tm_q;  // bf16 [B][Sq][Hq][D]: dims (D, Sq, Hq, B), box (64, 128, 1, 1)
+    CUtensorMap tm_k;  // bf16 [B][Sk][Hkv][D]
+    CUtensorMap tm_v;
+    __nv_bfloat16 *o;
+    float *lse;
+    const int *doc_offsets;
+    int *status;
+    int num_docs;
+    int B, Hq, Hkv, Sq, Sk, group;
+    int causal, window_left, window_right;
+    int num_qblocks;
+    float scale_log2;
+    float rescale_threshold;
+};
+
+template <int D, int NS>
+struct FwdSmem {
+    static constexpr int kChunks = D / 64;
+    static constexpr int kChunkElems = kBlockM * 64;  // 16 KB
+    __nv_bfloat16 q[2][kChunks][kChunkElems];
+    __nv_bfloat16 kv[NS][kChunks][kChunkElems];
+    uint64_t q_full;
+    uint64_t kv_full[NS];
+    uint64_t kv_empty[NS];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t o_final[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int range[2][2];  // per query tile: first and last key block (inclusive)
+};
+
+// Keys [lo, hi] (inclusive) that query `row` may attend to; lo > hi = none.
+struct KeyRange {
+    int lo, hi;
+};
+
+__device__ __forceinline__ KeyRange row_key_range(const FwdParams &p, int row) {
+    long long lo = 0, hi = (long long)p.Sk - 1;
+    const long long diag = (long long)row + p.Sk - p.Sq;
+    if (p.causal) hi = min(hi, diag);
+    if (p.window_left >= 0) lo = max(lo, diag - p.window_left);
+    if (p.window_right >= 0) hi = min(hi, diag + p.window_right);
+    if (p.doc_offsets != nullptr) {
+        const int *off = p.doc_offsets;
+        if (row < __ldg(off) || row >= __ldg(off + p.num_docs)) return {1, 0};
+        int a = 0, c = p.num_docs;  // off[a] <= row < off[c]
+        while (c - a > 1) {
+            const int m = (a + c) >> 1;
+            if (__ldg(off + m) <= row) a = m; else c = m;
+        }
+        lo = max(lo, (long long)__ldg(off + a));
+        hi = min(hi, (long long)__ldg(off + a + 1) - 1);
+    }
+    if (lo > hi) return {1, 0};
+    return {(int)lo, (int)hi};
+}
+
+// Bounded wait.  Returns false when the CTA is aborting (own timeout or
+// another role's); `honor_abort` = false keeps waiting until the timeout only.
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
+                                             volatile int *abort_flag, int *status,
+                                             bool honor_abort = true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 15u) == 0u) {
+            if (honor_abort && *abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+                *abort_flag = 1;
+                atomicCAS(status, 0, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ float ex2_poly(float x) {
+    // x = j + f, j = round(x) via the 1.5 * 2^23 trick, f in [-1/2, 1/2];
+    // 2^x = p(f) * 2^j with 2^j applied through the exponent field.
+    x = fmaxf(x, -125.0f);
+    const float magic = 12582912.0f;
+    const float t = x + magic;
+    const float f = x - (t - magic);
+    const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Columns (out of every 32) that use the polynomial in EXP_MODE 1.
+constexpr int kPolyPer32 = 12;
+
+template <int EXP_MODE>
+__device__ __forceinline__ bool use_poly(int col) {
+    if (EXP_MODE == 0) return false;
+    if (EXP_MODE == 2) return true;
+    return (col & 31) < kPolyPer32;
+}
+
+template <int D, int NS, int EXP_MODE>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+    using Smem = FwdSmem<D, NS>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_off = smem_u32(smem_raw);
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (raw_off & 1023u)) & 1023u));
+
+    const int warp = warp_id();
+    const int lane = lane_id();
+
+    // Work item: heaviest query blocks first across all heads (causal load
+    // balance), then (batch, head).
+    const int bh_count = p.Hq * p.B;
+    const int qb = p.num_qblocks - 1 - (int)(blockIdx.x / bh_count);
+    const int bh = (int)(blockIdx.x % bh_count);
+    const int hq = bh % p.Hq;
+    const int b = bh / p.Hq;
+    const int hkv = hq / p.group;
+    const int q0 = qb * 2 * kBlockM;
+
+    // ------------------------------------------------------------ prologue
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.s_full[i], 1);
+            mbar_init(&sm.p_full[i], kBlockM);
+            mbar_init(&sm.o_final[i], 1);
+        }
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        // Key-block range of each query tile: union of its rows' key ranges.
+        for (int i = 0; i < 2; ++i) {
+            int lo = 0x7fffffff, hi = -1;
+            for (int t = lane; t < kBlockM; t += 32) {
+                const int row = q0 + i * kBlockM + t;
+                if (row >= p.Sq) break;
+                const KeyRange r = row_key_range(p, row);
+                if (r.lo <= r.hi) {
+                    lo = min(lo, r.lo);
+                    hi = max(hi, r.hi);
+                }
+            }
+            for (int o = 16; o > 0; o >>= 1) {
+                lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+                hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+            }
+            if (lane == 0) {
+                if (hi < 0) {
+                    sm.range[i][0] = 1;
+                    sm.range[i][1] = 0;
+                } else {
+                    sm.range[i][0] = lo / kBlockN;
+                    sm.range[i][1] = hi / kBlockN;
+                }
+            }
+        }
+    }
+    if (warp == 8) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort_flag;
+    const int lo0 = sm.range[0][0], hi0 = sm.range[0][1];
+    const int lo1 = sm.range[1][0], hi1 = sm.range[1][1];
+    const bool has0 = lo0 <= hi0, has1 = lo1 <= hi1;
+    const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : lo1;
+    const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : hi1;
+    const int n_blocks = (has0 || has1) ? (uhi - ulo + 1) : 0;
+    constexpr uint32_t kTileBytes = kBlockM * D * 2;
+
+    // Registers: the softmax warpgroups hold a 128-column score row per
+    // thread; the MMA / TMA warpgroup needs few.  384 x 168 at launch =
+    // 2 x 128 x kSoftmaxRegs + 128 x kOtherRegs.  All four warps of a
+    // warpgroup execute the same setmaxnreg instruction, and each budget
+    // dominates the code of its roles so the compiler allocates per role.
+    if (warp >= 8) {
+        setmaxnreg_dec<kOtherRegs>();
+        if (warp == 9) {
+            // ------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                prefetch_tensormap(&p.tm_q);
+                prefetch_tensormap(&p.tm_k);
+                prefetch_tensormap(&p.tm_v);
+                mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
+                for (int i = 0; i < 2; ++i)
+                    for (int c = 0; c < Smem::kChunks; ++c)
+                        tma_load_4d(sm.q[i][c], &p.tm_q, &sm.q_full, c * 64, q0 + i * kBlockM, hq, b);
+                uint32_t it = 0;
+                bool ok = true;
+                for (int t = 0; t < n_blocks && ok; ++t) {
+                    const int key0 = (ulo + t) * kBlockN;
+                    for (int which = 0; which < 2 && ok; ++which, ++it) {
+                        const uint32_t slot = it % NS;
+                        ok = wait_bounded(&sm.kv_empty[slot], ((it / NS) & 1u) ^ 1u, abort_flag,
+                                          p.status);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(&sm.kv_full[slot], kTileBytes);
+                        const CUtensorMap *map = which ? &p.tm_v : &p.tm_k;
+                        for (int c = 0; c < Smem::kChunks; ++c)
+                            tma_load_4d(sm.kv[slot][c], map, &sm.kv_full[slot], c * 64, key0, hkv, b);
+                    }
+                }
+                // Every copy still in flight lands before the CTA can exit (only
+                // the last NS loads can be outstanding; on the normal path they
+                // have been consumed already).
+                wait_bounded(&sm.q_full, 0, abort_flag, p.status, false);
+                const uint32_t first = it > NS ? it - NS : 0;
+                for (uint32_t L = first; L < it; ++L)
+                    wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status, false);
+            }
+            __syncwarp();
+        } else if (warp == 8) {
+            // ------------------------------------------------------- MMA issuer
+            if (lane == 0 && n_blocks > 0) {
+                constexpr uint32_t kIdescQK = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+                constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlockM, D, 0, 1);
+                const uint32_t q_addr = smem_u32(&sm.q[0][0][0]);
+                const uint32_t kv_addr = smem_u32(&sm.kv[0][0][0]);
+                constexpr uint32_t kQTileBytes = Smem::kChunks * Smem::kChunkElems * 2;
+                constexpr uint32_t kChunkBytes = Smem::kChunkElems * 2;
+                bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status);
+                tc_fence_after();
+                int k_ready = ulo - 1;  // last key block whose K slot was waited on
+                auto ring_pos = [&](int j, int which) -> uint32_t {
+                    return 2u * (uint32_t)(j - ulo) + (uint32_t)which;
+                };
+                auto wait_k = [&](int j) {
+                    const uint32_t L = ring_pos(j, 0);
+                    ok = ok && wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status);
+                    tc_fence_after();
+                    k_ready = j;
+                };
+                auto issue_s = [&](int i, int j) {
+                    if (k_ready < j) wait_k(j);
+                    if (!ok) return;
+                    const uint32_t slot = ring_pos(j, 0) % NS;
+                    const uint32_t a_base = q_addr + i * kQTileBytes;
+                    const uint32_t b_base = kv_addr + slot * kQTileBytes;
+    #pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
+                        mma_ss(tmem + i * kBlockN, smem_desc_sw128(a_base + off, 16, 1024),
+                               smem_desc_sw128(b_base + off, 16, 1024), kIdescQK, ks > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&sm.s_full[i]);
+                };
+                auto active = [&](int i, int j) -> bool {
+                    return i == 0 ? (has0 && j >= lo0 && j <= hi0) : (has1 && j >= lo1 && j <= hi1);
+                };
+
+                for (int i = 0; i < 2; ++i)
+                    if (active(i, ulo)) issue_s(i, ulo);
+                if (ok && k_ready < ulo) wait_k(ulo);
+                if (ok) tc_commit(&sm.kv_empty[ring_pos(ulo, 0) % NS]);
+
+                for (int j = ulo; j <= uhi && ok; ++j) {
+                    const uint32_t Lv = ring_pos(j, 1);
+                    const uint32_t vslot = Lv % NS;
+                    ok = wait_bounded(&sm.kv_full[vslot], (Lv / NS) & 1u, abort_flag, p.status);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t v_base = kv_addr + vslot * kQTileBytes;
+                    for (int i = 0; i < 2 && ok; ++i) {
+                        if (active(i, j)) {
+                            const int lo_i = i == 0 ? lo0 : lo1;
+                            const int hi_i = i == 0 ? hi0 : hi1;
+                            ok = wait_bounded(&sm.p_full[i], (uint32_t)(j - lo_i) & 1u, abort_flag,
+                                              p.status);
+                            if (!ok) break;
+                            tc_fence_after();
+                            const uint32_t o_tmem = tmem + 2 * kBlockN + i * D;
+                            const uint32_t p_tmem = tmem + i * kBlockN;
+    #pragma unroll
+                            for (int ks = 0; ks < kBlockN / 16; ++ks) {
+                                // V chunk layout: key rows of 128 bytes, 8-row groups 1024 B
+                                // apart (SBO), 64-column chunks kChunkBytes apart (LBO).
+                                mma_ts(o_tmem, p_tmem + ks * 8,
+                                       smem_desc_sw128(v_base + ks * 16 * 128, kChunkBytes, 1024),
+                                       kIdescPV, (j > lo_i || ks > 0) ? 1u : 0u);
+                            }
+                            if (j == hi_i) tc_commit(&sm.o_final[i]);
+                        }
+                        if (j + 1 <= uhi && active(i, j + 1)) issue_s(i, j + 1);
+                    }
+                    if (!ok) break;
+                    if (j + 1 <= uhi && k_ready < j + 1) wait_k(j + 1);
+                    if (!ok) break;
+                    tc_commit(&sm.kv_empty[vslot]);
+                    if (j + 1 <= uhi) tc_commit(&sm.kv_empty[ring_pos(j + 1, 0) % NS]);
+                }
+                if (!ok) {
+                    // Let every MMA already issued finish before TMEM is freed.
+                    tc_commit(&sm.drain);
+                    wait_bounded(&sm.drain, 0, abort_flag, p.status, false);
+                }
+            }
+            __syncwarp();
+        }
+        // warps 10-11: idle
+    } else {
+        // ------------------------------------- softmax / correction / epilogue
+        setmaxnreg_inc<kSoftmaxRegs>();
+        const int i = warp >> 2;
+        const int row_in_tile = threadIdx.x & (kBlockM - 1);
+        const int row = q0 + i * kBlockM + row_in_tile;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t s_tmem = tmem + lane_base + i * kBlockN;
+        const uint32_t o_tmem = tmem + lane_base + 2 * kBlockN + i * D;
+        const KeyRange kr = row_key_range(p, row);
+        const int lo_b = i == 0 ? lo0 : lo1;
+        const int hi_b = i == 0 ? hi0 : hi1;
+        const float c = p.scale_log2;
+        const float tau = p.rescale_threshold;
+        float m_run = -INFINITY;
+        float l_run = 0.0f;
+        bool ok = true;
+
+        for (int j = lo_b; j <= hi_b; ++j) {
+            const int t = j - lo_b;
+            ok = wait_bounded(&sm.s_full[i], (uint32_t)t & 1u, abort_flag, p.status);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+
+            float s[kBlockN];
+#pragma unroll
+            for (int ch = 0; ch < kBlockN / 32; ++ch) {
+                uint32_t r[32];
+                tmem_ld32(s_tmem + ch * 32, r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s[ch * 32 + e] = __uint_as_float(r[e]);
+            }
+            tmem_wait_ld();
+
+            const int key0 = j * kBlockN;
+            const bool need_mask = key0 < kr.lo || key0 + kBlockN - 1 > kr.hi;
+            const bool masked = __any_sync(0xffffffffu, need_mask);
+            if (masked) {
+#pragma unroll
+                for (int e = 0; e < kBlockN; ++e) {
+                    const int key = key0 + e;
+                    if (key < kr.lo || key > kr.hi) s[e] = -INFINITY;
+                }
+            }
+            float mx[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx[e] = s[e];
+#pragma unroll
+            for (int e = 8; e < kBlockN; ++e) mx[e & 7] = fmaxf(mx[e & 7], s[e]);
+            const float row_max =
+                fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m_cand = row_max * c;
+            float alpha = 1.0f;
+            if (m_cand > m_run + tau) {
+                alpha = ex2_mufu(m_run - m_cand);
+                m_run = m_cand;
+            }
+            const float m_use = m_run == -INFINITY ? 0.0f : m_run;
+
+            l_run *= alpha;
+
+            // Probabilities: p = 2^(x - m), row sum, bf16 pairs into TMEM.
+            float sum[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sum[e] = 0.0f;
+            uint32_t pk[kBlockN / 2];
+            if (masked) {
+#pragma unroll
+                for (int e = 0; e < kBlockN; e += 2) {
+                    const float p0 = ex2_mufu(fmaf(s[e], c, -m_use));
+                    const float p1 = ex2_mufu(fmaf(s[e + 1], c, -m_use));
+                    sum[(e >> 1) & 7] += p0 + p1;
+                    pk[e >> 1] = pack_bf16x2(p0, p1);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < kBlockN; e += 2) {
+                    const float x0 = fmaf(s[e], c, -m_use);
+                    const float x1 = fmaf(s[e + 1], c, -m_use);
+                    const float p0 = use_poly<EXP_MODE>(e) ? ex2_poly(x0) : ex2_mufu(x0);
+                    const float p1 = use_poly<EXP_MODE>(e + 1) ? ex2_poly(x1) : ex2_mufu(x1);
+                    sum[(e >> 1) & 7] += p0 + p1;
+                    pk[e >> 1] = pack_bf16x2(p0, p1);
+                }
+            }
+            l_run += ((sum[0] + sum[1]) + (sum[2] + sum[3])) +
+                     ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+#pragma unroll
+            for (int h = 0; h < kBlockN / 64; ++h) {
+                uint32_t r[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = pk[h * 32 + e];
+                tmem_st32(s_tmem + h * 32, r);
+            }
+            // Correction: rescale this row of O in TMEM (rare once the max
+            // settles).  PV of the previous block is complete: the commit that
+            // signalled S of this block covers every earlier MMA.
+            if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t r[32];
+                    tmem_ld32(o_tmem + ch * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                    tmem_st32(o_tmem + ch * 32, r);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.p_full[i]);
+        }
+
+        // ----------------------------------------------------------- epilogue
+        const bool has_blocks = lo_b <= hi_b;
+        if (ok && has_blocks) {
+            ok = wait_bounded(&sm.o_final[i], 0, abort_flag, p.status);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+        }
+        if (ok) {
+            const bool row_ok = row < p.Sq;
+            const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+            __nv_bfloat16 *o_row =
+                p.o + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)D;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t r[32];
+                if (has_blocks) {
+                    tmem_ld32(o_tmem + ch * 32, r);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = 0u;
+                }
+                uint4 out[4];
+                uint32_t *w = reinterpret_cast<uint32_t *>(out);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
+                                       __uint_as_float(r[2 * e + 1]) * inv_l);
+                if (row_ok) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(o_row + ch * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = out[e];
+                }
+            }
+            if (row_ok) {
+                const float lse = l_run > 0.0f ? (m_run + log2f(l_run)) * 0.69314718055994531f
+                                               : -INFINITY;
+                p.lse[((size_t)b * p.Hq + hq) * p.Sq + row] = lse;
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace tab
