@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Attention-forward benchmark on B200: TFLOP/s and % of BF16 tensor peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one forward pass (O and LSE) over one batch of the named workload
+(default: the causal S=8192 one), inputs resident in HBM.  Prints ONE JSON
+line on rank 0.  For N > 1 (launched under torchrun) every rank runs an
+independent replica of the same workload on its own GPU: the path needs no
+exchange between GPUs, so there is no collective on the data path ("replicas
+only"); ranks synchronise only to start and stop the clock, and the time is
+the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle (the only reference this
+method has) on a bounded sample of rows of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from tiled_attention_blackwell_b200.workloads import (HEADLINE, WORKLOADS,  # noqa: E402
+                                                      make_inputs, useful_flops)
+
+METRIC = "attention fwd TFLOP/s and % of B200 BF16 tensor peak (S=8192 causal, D=128)"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["tiled_attention_blackwell_b200/csrc/fwd_kernel.cuh",
+                  "tiled_attention_blackwell_b200/csrc/ptx.cuh",
+                  "tiled_attention_blackwell_b200/csrc/exp2_poly.cuh",
+                  "tiled_attention_blackwell_b200/csrc/attn_api.cu"]
+
+
+# ------------------------------------------------------------------ helpers
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing leg (faster local iteration)")
+    ap.add_argument("--exp2-mode", type=int, default=None)
+    ap.add_argument("--rescale-threshold", type=float, default=None)
+    return ap.parse_args(argv)
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"fwd_{config}_ncu.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_sources_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def allowed_keys_per_row(w, doc_offsets):
+    """Number of keys each query row may see (for FLOP accounting of a row
+    sample): causal -> i + 1, document-causal -> i - doc_start + 1."""
+    i = np.arange(w.S, dtype=np.int64)
+    if doc_offsets is not None:
+        starts = np.repeat(doc_offsets[:-1], np.diff(doc_offsets)).astype(np.int64)
+        return (i - starts + 1) if w.causal else np.repeat(np.diff(doc_offsets), np.diff(doc_offsets))
+    return (i + 1) if w.causal else np.full(w.S, w.S, dtype=np.int64)
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            uuid = str(uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                mask = get(self.h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- distributed
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return rank, world, local
+
+
+def init_process_group(world: int, local: int, backend: str = "nccl"):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120), **kw)
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(w, inputs, n_rows: int, seed: int = 0):
+    """Time the oracle on `n_rows` random rows of the workload.  Returns
+    (seconds, useful FLOPs, threads)."""
+    import oracle  # test infrastructure: only this leg of the benchmark loads it
+    rng = np.random.default_rng(seed)
+    rows = np.stack([rng.integers(0, w.B, n_rows), rng.integers(0, w.Hq, n_rows),
+                     rng.integers(0, w.S, n_rows)], axis=1).astype(np.int64)
+    keys = allowed_keys_per_row(w, inputs["doc_offsets"])
+    flops = float((4.0 * w.D * keys[rows[:, 2]]).sum())
+    t0 = time.perf_counter()
+    oracle.attn_fwd(inputs["q"], inputs["k"], inputs["v"], scale=w.scale, causal=w.causal,
+                    window=None if w.window == (-1, -1) else w.window,
+                    doc_offsets=inputs["doc_offsets"], rows=rows)
+    return time.perf_counter() - t0, flops, oracle.num_threads()
+
+
+def rows_for_seconds(w, inputs, seconds: float) -> int:
+    """Calibrate the row count so the oracle runs for about `seconds`."""
+    n = 500
+    dt, _, _ = oracle_sample(w, inputs, n, seed=123)
+    return max(100, int(n * seconds / max(dt, 1e-3)))
+
+
+def workload_config(w, doc_offsets):
+    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.S, "Sk": w.S,
+           "D": w.D, "mask": ("document-causal" if doc_offsets is not None else
+                              ("causal" if w.causal else "none")),
+           "scale": w.scale}
+    if doc_offsets is not None:
+        cfg["num_docs"] = int(len(doc_offsets) - 1)
+    io_bytes = 2 * (2 * w.B * w.S * w.Hq * w.D + 2 * w.B * w.S * w.Hkv * w.D) + 4 * w.B * w.Hq * w.S
+    cfg["io_bytes"] = io_bytes
+    cfg["l2"] = (f"inputs+outputs {io_bytes / 2**20:.0f} MiB > L2 126 MiB; no flush"
+                 if io_bytes > L2_BYTES else "L2 flushed between steps")
+    return cfg
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    init_process_group(world, local)
+    device = torch.device("cuda", local)
+    from tiled_attention_blackwell_b200 import attn
+
+    w = WORKLOADS[args.config]
+    inp = make_inputs(w)
+    docs_np = inp["doc_offsets"]
+    flops = useful_flops(w.B, w.Hq, w.S, w.S, w.D, causal=w.causal, doc_offsets=docs_np)
+    cfg = workload_config(w, docs_np)
+    cfg["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
+
+    host = {n: inp[n].pin_memory() for n in ("q", "k", "v")}
+    dev = {n: host[n].to(device) for n in host}
+    docs = None if docs_np is None else torch.as_tensor(docs_np, dtype=torch.int32, device=device)
+    o = torch.empty_like(dev["q"])
+    lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=device)
+    flush = None if cfg["io_bytes"] > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8,
+                                                                 device=device)
+    opts = None
+    if args.exp2_mode is not None or args.rescale_threshold is not None:
+        kw = {}
+        if args.exp2_mode is not None:
+            kw["exp2_mode"] = args.exp2_mode
+        if args.rescale_threshold is not None:
+            kw["rescale_threshold"] = args.rescale_threshold
+        opts = attn.default_options(**kw)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        attn.attn_fwd(dev["q"], dev["k"], dev["v"], o, lse, scale=w.scale, causal=w.causal,
+                      window=None if w.window == (-1, -1) else w.window, doc_offsets=docs,
+                      options=opts, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    attn.check_device_status(stream)
+
+    # ---- device-resident timing: K steps, per-launch events on the launch stream
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    with sampler:
+        t_begin.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(world)
+    attn.check_device_status(stream)
+    total_ms = t_begin.elapsed_time(t_end)
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms_max = max_over_ranks(total_ms, world, device)
+    ms_per_step = total_ms_max / args.steps
+    value = flops * args.steps * world / (total_ms_max / 1e3) / 1e12
+    launch_avg_ms = float(np.mean(launch_ms))
+
+    # ---- end to end through the C ABI: pinned host inputs in, O and LSE out
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+
+    def e2e_step():
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    for _ in range(min(args.warmup, 3)):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    e2e_value = flops * args.steps * world / (e2e_ms / 1e3) / 1e12
+
+    peaks, peak_kind = read_peaks()
+    achieved = flops / (launch_avg_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": cfg,
+        "pct_of_peak": round(100.0 * value / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(w.name),
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else "fallback 1590 TFLOP/s",
+                     "frac_of_sustained": round(achieved / float(
+                         peaks.get("bf16_tflops_sustained", peak)), 4),
+                     "flops_per_launch": flops, "launch_ms": round(launch_avg_ms, 4)},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_rows = rows_for_seconds(w, inp, 15.0)
+        dt, fl, cores = oracle_sample(w, inp, n_rows)
+        result["cpu_baseline"] = {
+            "value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n_rows} random (b, head, row) rows of {w.name}, fp64, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.config]
+    inp = make_inputs(w)
+    cfg = workload_config(w, inp["doc_offsets"])
+    cfg["parallelism"] = "CPU oracle, rank 0 only"
+    # each step: ~2 s of oracle work, so steps + warmup end within minutes
+    n_rows = rows_for_seconds(w, inp, 2.0)
+    for i in range(args.warmup):
+        oracle_sample(w, inp, n_rows, seed=1000 + i)
+    times, fl_total, cores = [], 0.0, 1
+    for i in range(args.steps):
+        dt, fl, cores = oracle_sample(w, inp, n_rows, seed=i)
+        times.append(dt)
+        fl_total += fl
+    total = sum(times)
+    value = fl_total / total / 1e12
+    result = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": cfg,
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{n_rows} random (b, head, row) rows of {w.name} per step, fp64"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -139,6 +139,11 @@ attn_status_t dispatch_exp(const tab::FwdParams &p, int grid, int exp_mode, cuda
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+#ifdef ATTN_TRACE
+long long *g_trace = nullptr;
+int g_trace_ctas = 0;
+#endif
+
 }  // namespace
 
 extern "C" {
@@ -221,6 +226,10 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
     p.num_qblocks = (int)num_qblocks;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.rescale_threshold = op.rescale_threshold;
+#ifdef ATTN_TRACE
+    p.trace = g_trace;
+    p.trace_ctas = g_trace_ctas;
+#endif
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (D == 128) return dispatch_exp<128, kStagesD128>(p, (int)grid, op.exp2_mode, cs);
@@ -269,5 +278,14 @@ const char *attn_status_string(attn_status_t status) {
 const char *attn_last_error_detail(void) { return g_detail; }
 
 int attn_abi_version(void) { return ATTN_ABI_VERSION; }
+
+#ifdef ATTN_TRACE
+// Trace builds only: device buffer of trace_ctas * 3 * 96 * 8 int64 for the
+// clock64 event log of the first trace_ctas CTAs (NULL disables).
+ATTN_API void attn_trace_set_buffer(long long *device_buffer, int trace_ctas) {
+    g_trace = device_buffer;
+    g_trace_ctas = device_buffer ? trace_ctas : 0;
+}
+#endif
 
 }  // extern "C"

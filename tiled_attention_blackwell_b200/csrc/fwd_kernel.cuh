@@ -72,7 +72,27 @@ struct FwdParams {
     int num_qblocks;
     float scale_log2;
     float rescale_threshold;
+    long long *trace;  // clock64 event log (trace builds only), else null
+    int trace_ctas;
 };
+
+// Opt-in event trace (compile with -DATTN_TRACE): lane 0 of warps 0 and 4
+// (the two softmax warpgroups) and of the MMA warp record clock64() at the
+// hand-off points of each key block, for the first `trace_ctas` CTAs.
+constexpr int kTraceIters = 96;
+constexpr int kTraceEvents = 8;
+#ifdef ATTN_TRACE
+#define ATTN_TRACE_EVENT(role, iter, ev)                                                    \
+    do {                                                                                  \
+        if (p.trace && (int)blockIdx.x < p.trace_ctas && (iter) < kTraceIters && lane == 0) \
+            p.trace[(((size_t)blockIdx.x * 3 + (role)) * kTraceIters + (iter)) *            \
+                        kTraceEvents + (ev)] = clock64();                                 \
+    } while (0)
+#else
+#define ATTN_TRACE_EVENT(role, iter, ev) \
+    do {                                 \
+    } while (0)
+#endif
 
 template <int D, int NS>
 struct FwdSmem {
@@ -284,15 +304,24 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             }
             __syncwarp();
         } else if (warp == 8) {
-            // ------------------------------------------------------- MMA issuer
-            if (lane == 0 && n_blocks > 0) {
+            // --------------------------------------------------- MMA issuer
+            // The whole warp runs the schedule, so control flow and descriptor
+            // arithmetic stay warp-uniform; one elected lane issues the
+            // tcgen05 instructions (and the commits that track them).
+            if (n_blocks > 0) {
+                const bool leader = elect_one();
                 constexpr uint32_t kIdescQK = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
                 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlockM, D, 0, 1);
-                const uint32_t q_addr = smem_u32(&sm.q[0][0][0]);
-                const uint32_t kv_addr = smem_u32(&sm.kv[0][0][0]);
                 constexpr uint32_t kQTileBytes = Smem::kChunks * Smem::kChunkElems * 2;
                 constexpr uint32_t kChunkBytes = Smem::kChunkElems * 2;
-                bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status);
+                // Base descriptors; a K-step or a ring slot only moves the start
+                // address (bits 0-13, in 16-byte units), a constant add.
+                const uint64_t q_desc = smem_desc_sw128(smem_u32(&sm.q[0][0][0]), 16, 1024);
+                const uint64_t k_desc = smem_desc_sw128(smem_u32(&sm.kv[0][0][0]), 16, 1024);
+                const uint64_t v_desc =
+                    smem_desc_sw128(smem_u32(&sm.kv[0][0][0]), kChunkBytes, 1024);
+                bool ok = __all_sync(0xffffffffu,
+                                     wait_bounded(&sm.q_full, 0, abort_flag, p.status));
                 tc_fence_after();
                 int k_ready = ulo - 1;  // last key block whose K slot was waited on
                 auto ring_pos = [&](int j, int which) -> uint32_t {
@@ -300,71 +329,92 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 };
                 auto wait_k = [&](int j) {
                     const uint32_t L = ring_pos(j, 0);
-                    ok = ok && wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status);
+                    if (ok)
+                        ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[L % NS],
+                                                                  (L / NS) & 1u, abort_flag,
+                                                                  p.status));
                     tc_fence_after();
                     k_ready = j;
                 };
                 auto issue_s = [&](int i, int j) {
                     if (k_ready < j) wait_k(j);
                     if (!ok) return;
-                    const uint32_t slot = ring_pos(j, 0) % NS;
-                    const uint32_t a_base = q_addr + i * kQTileBytes;
-                    const uint32_t b_base = kv_addr + slot * kQTileBytes;
-    #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * kChunkBytes + (ks & 3) * 32;
-                        mma_ss(tmem + i * kBlockN, smem_desc_sw128(a_base + off, 16, 1024),
-                               smem_desc_sw128(b_base + off, 16, 1024), kIdescQK, ks > 0 ? 1u : 0u);
+                    const uint64_t a0 = q_desc + ((i * kQTileBytes) >> 4);
+                    const uint64_t b0 = k_desc + (((ring_pos(j, 0) % NS) * kQTileBytes) >> 4);
+                    if (leader) {
+#pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint32_t off = ((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4;
+                            mma_ss(tmem + i * kBlockN, a0 + off, b0 + off, kIdescQK,
+                                   ks > 0 ? 1u : 0u);
+                        }
+                        tc_commit(&sm.s_full[i]);
                     }
-                    tc_commit(&sm.s_full[i]);
+                    __syncwarp();
                 };
                 auto active = [&](int i, int j) -> bool {
-                    return i == 0 ? (has0 && j >= lo0 && j <= hi0) : (has1 && j >= lo1 && j <= hi1);
+                    return i == 0 ? (has0 && j >= lo0 && j <= hi0)
+                                  : (has1 && j >= lo1 && j <= hi1);
                 };
 
                 for (int i = 0; i < 2; ++i)
                     if (active(i, ulo)) issue_s(i, ulo);
                 if (ok && k_ready < ulo) wait_k(ulo);
-                if (ok) tc_commit(&sm.kv_empty[ring_pos(ulo, 0) % NS]);
+                if (ok && leader) tc_commit(&sm.kv_empty[ring_pos(ulo, 0) % NS]);
+                __syncwarp();
 
                 for (int j = ulo; j <= uhi && ok; ++j) {
                     const uint32_t Lv = ring_pos(j, 1);
                     const uint32_t vslot = Lv % NS;
-                    ok = wait_bounded(&sm.kv_full[vslot], (Lv / NS) & 1u, abort_flag, p.status);
+                    ATTN_TRACE_EVENT(2, j - ulo, 0);
+                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[vslot], (Lv / NS) & 1u,
+                                                              abort_flag, p.status));
+                    ATTN_TRACE_EVENT(2, j - ulo, 1);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t v_base = kv_addr + vslot * kQTileBytes;
+                    const uint64_t vb = v_desc + ((vslot * kQTileBytes) >> 4);
                     for (int i = 0; i < 2 && ok; ++i) {
                         if (active(i, j)) {
                             const int lo_i = i == 0 ? lo0 : lo1;
                             const int hi_i = i == 0 ? hi0 : hi1;
-                            ok = wait_bounded(&sm.p_full[i], (uint32_t)(j - lo_i) & 1u, abort_flag,
-                                              p.status);
+                            ATTN_TRACE_EVENT(2, j - ulo, 2 + 3 * i);
+                            ok = __all_sync(0xffffffffu,
+                                            wait_bounded(&sm.p_full[i], (uint32_t)(j - lo_i) & 1u,
+                                                         abort_flag, p.status));
+                            ATTN_TRACE_EVENT(2, j - ulo, 3 + 3 * i);
                             if (!ok) break;
                             tc_fence_after();
                             const uint32_t o_tmem = tmem + 2 * kBlockN + i * D;
                             const uint32_t p_tmem = tmem + i * kBlockN;
-    #pragma unroll
-                            for (int ks = 0; ks < kBlockN / 16; ++ks) {
-                                // V chunk layout: key rows of 128 bytes, 8-row groups 1024 B
-                                // apart (SBO), 64-column chunks kChunkBytes apart (LBO).
-                                mma_ts(o_tmem, p_tmem + ks * 8,
-                                       smem_desc_sw128(v_base + ks * 16 * 128, kChunkBytes, 1024),
-                                       kIdescPV, (j > lo_i || ks > 0) ? 1u : 0u);
+                            const uint32_t first = j > lo_i ? 1u : 0u;
+                            if (leader) {
+#pragma unroll
+                                for (int ks = 0; ks < kBlockN / 16; ++ks) {
+                                    // V chunk: key rows of 128 bytes, 8-row groups 1024 B
+                                    // apart (SBO), 64-column chunks kChunkBytes apart (LBO).
+                                    mma_ts(o_tmem, p_tmem + ks * 8, vb + ((ks * 16 * 128) >> 4),
+                                           kIdescPV, ks > 0 ? 1u : first);
+                                }
+                                if (j == hi_i) tc_commit(&sm.o_final[i]);
                             }
-                            if (j == hi_i) tc_commit(&sm.o_final[i]);
+                            __syncwarp();
                         }
                         if (j + 1 <= uhi && active(i, j + 1)) issue_s(i, j + 1);
+                        ATTN_TRACE_EVENT(2, j - ulo, 4 + 3 * i);
                     }
                     if (!ok) break;
                     if (j + 1 <= uhi && k_ready < j + 1) wait_k(j + 1);
                     if (!ok) break;
-                    tc_commit(&sm.kv_empty[vslot]);
-                    if (j + 1 <= uhi) tc_commit(&sm.kv_empty[ring_pos(j + 1, 0) % NS]);
+                    if (leader) {
+                        tc_commit(&sm.kv_empty[vslot]);
+                        if (j + 1 <= uhi) tc_commit(&sm.kv_empty[ring_pos(j + 1, 0) % NS]);
+                    }
+                    __syncwarp();
                 }
                 if (!ok) {
                     // Let every MMA already issued finish before TMEM is freed.
-                    tc_commit(&sm.drain);
+                    if (leader) tc_commit(&sm.drain);
+                    __syncwarp();
                     wait_bounded(&sm.drain, 0, abort_flag, p.status, false);
                 }
             }
@@ -391,10 +441,12 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
 
         for (int j = lo_b; j <= hi_b; ++j) {
             const int t = j - lo_b;
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 0);
             ok = wait_bounded(&sm.s_full[i], (uint32_t)t & 1u, abort_flag, p.status);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 1);
 
             float s[kBlockN];
 #pragma unroll
@@ -405,6 +457,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 for (int e = 0; e < 32; ++e) s[ch * 32 + e] = __uint_as_float(r[e]);
             }
             tmem_wait_ld();
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 2);
 
             const int key0 = j * kBlockN;
             const bool need_mask = key0 < kr.lo || key0 + kBlockN - 1 > kr.hi;
@@ -431,6 +484,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 m_run = m_cand;
             }
             const float m_use = m_run == -INFINITY ? 0.0f : m_run;
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 3);
 
             l_run *= alpha;
 
@@ -460,6 +514,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             }
             l_run += ((sum[0] + sum[1]) + (sum[2] + sum[3])) +
                      ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
 #pragma unroll
             for (int h = 0; h < kBlockN / 64; ++h) {
                 uint32_t r[32];
@@ -483,6 +538,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 }
             }
             tmem_wait_st();
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 5);
             tc_fence_before();
             mbar_arrive(&sm.p_full[i]);
         }

@@ -21,6 +21,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+
+// True in exactly one lane of a fully active warp (elect.sync).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
+}
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 // ------------------------------------------------------------------ mbarrier
