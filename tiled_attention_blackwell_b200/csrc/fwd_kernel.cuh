@@ -51,8 +51,8 @@ constexpr int kBlockM = 128;   // query rows per tile = TMEM lanes
 constexpr int kBlockN = 128;   // keys per key/value block
 constexpr int kFwdThreads = 384;
 constexpr int kTmemCols = 512;
-constexpr int kSoftmaxRegs = 208;
-constexpr int kOtherRegs = 88;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kOtherRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kFwdThreads * 168,
               "register split exceeds the launch allocation");
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
@@ -104,7 +104,8 @@ struct FwdSmem {
     uint64_t kv_full[NS];
     uint64_t kv_empty[NS];
     uint64_t s_full[2];
-    uint64_t p_full[2];
+    uint64_t p_half[2];  // P of keys [0, 64) of the block is in TMEM
+    uint64_t p_full[2];  // all of P (and any O correction) is in TMEM
     uint64_t o_final[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -169,7 +170,24 @@ __device__ __forceinline__ float ex2_poly(float x) {
     return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
-// Columns (out of every 32) that use the polynomial in EXP_MODE 1.
+// Two lanes at once with packed f32x2 arithmetic; same steps as ex2_poly.
+__device__ __forceinline__ void ex2_poly2(float &y0, float &y1, float x0, float x1) {
+    x0 = fmaxf(x0, -125.0f);
+    x1 = fmaxf(x1, -125.0f);
+    const float magic = 12582912.0f;
+    float t0, t1, j0, j1, f0, f1, p0, p1;
+    add2(t0, t1, x0, x1, magic, magic);
+    add2(j0, j1, t0, t1, -magic, -magic);
+    add2(f0, f1, x0, x1, -j0, -j1);
+    fma2(p0, p1, kExp2C3, kExp2C3, f0, f1, kExp2C2, kExp2C2);
+    fma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
+    fma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// Columns (out of every 32) that use the polynomial in EXP_MODE 1 (taken in
+// pairs: both columns of a pair use the same unit).
 constexpr int kPolyPer32 = 12;
 
 template <int EXP_MODE>
@@ -177,6 +195,30 @@ __device__ __forceinline__ bool use_poly(int col) {
     if (EXP_MODE == 0) return false;
     if (EXP_MODE == 2) return true;
     return (col & 31) < kPolyPer32;
+}
+
+// Half a row of a block: p = 2^(s*c - m) for 64 scores (packed pairs), the
+// exponentials split between MUFU and the polynomial per EXP_MODE; returns
+// the row sum and writes the bf16 pairs to pk.
+template <int EXP_MODE>
+__device__ __forceinline__ float exp_pack_half(const float *s, float c, float neg_m,
+                                               uint32_t *pk) {
+    float sum0 = 0.0f, sum1 = 0.0f, sum2 = 0.0f, sum3 = 0.0f;
+#pragma unroll
+    for (int e = 0; e < kBlockN / 2; e += 2) {
+        float x0, x1, p0, p1;
+        fma2(x0, x1, s[e], s[e + 1], c, c, neg_m, neg_m);
+        if (use_poly<EXP_MODE>(e)) {
+            ex2_poly2(p0, p1, x0, x1);
+        } else {
+            p0 = ex2_mufu(x0);
+            p1 = ex2_mufu(x1);
+        }
+        if ((e & 2) == 0) add2(sum0, sum1, sum0, sum1, p0, p1);
+        else add2(sum2, sum3, sum2, sum3, p0, p1);
+        pk[e >> 1] = pack_bf16x2(p0, p1);
+    }
+    return (sum0 + sum1) + (sum2 + sum3);
 }
 
 template <int D, int NS, int EXP_MODE>
@@ -209,6 +251,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.s_full[i], 1);
+            mbar_init(&sm.p_half[i], kBlockM);
             mbar_init(&sm.p_full[i], kBlockM);
             mbar_init(&sm.o_final[i], 1);
         }
@@ -377,24 +420,35 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                         if (active(i, j)) {
                             const int lo_i = i == 0 ? lo0 : lo1;
                             const int hi_i = i == 0 ? hi0 : hi1;
-                            ATTN_TRACE_EVENT(2, j - ulo, 2 + 3 * i);
-                            ok = __all_sync(0xffffffffu,
-                                            wait_bounded(&sm.p_full[i], (uint32_t)(j - lo_i) & 1u,
-                                                         abort_flag, p.status));
-                            ATTN_TRACE_EVENT(2, j - ulo, 3 + 3 * i);
-                            if (!ok) break;
-                            tc_fence_after();
+                            const uint32_t par = (uint32_t)(j - lo_i) & 1u;
                             const uint32_t o_tmem = tmem + 2 * kBlockN + i * D;
                             const uint32_t p_tmem = tmem + i * kBlockN;
                             const uint32_t first = j > lo_i ? 1u : 0u;
+                            // PV in two halves of 64 keys, each as soon as its P is in TMEM.
+                            // V chunk: key rows of 128 bytes, 8-row groups 1024 B apart
+                            // (SBO), 64-column chunks kChunkBytes apart (LBO).
+                            ATTN_TRACE_EVENT(2, j - ulo, 2 + 3 * i);
+                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_half[i], par,
+                                                                      abort_flag, p.status));
+                            if (!ok) break;
+                            tc_fence_after();
                             if (leader) {
 #pragma unroll
-                                for (int ks = 0; ks < kBlockN / 16; ++ks) {
-                                    // V chunk: key rows of 128 bytes, 8-row groups 1024 B
-                                    // apart (SBO), 64-column chunks kChunkBytes apart (LBO).
+                                for (int ks = 0; ks < kBlockN / 32; ++ks)
                                     mma_ts(o_tmem, p_tmem + ks * 8, vb + ((ks * 16 * 128) >> 4),
                                            kIdescPV, ks > 0 ? 1u : first);
-                                }
+                            }
+                            __syncwarp();
+                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_full[i], par,
+                                                                      abort_flag, p.status));
+                            ATTN_TRACE_EVENT(2, j - ulo, 3 + 3 * i);
+                            if (!ok) break;
+                            tc_fence_after();
+                            if (leader) {
+#pragma unroll
+                                for (int ks = kBlockN / 32; ks < kBlockN / 16; ++ks)
+                                    mma_ts(o_tmem, p_tmem + ks * 8, vb + ((ks * 16 * 128) >> 4),
+                                           kIdescPV, 1u);
                                 if (j == hi_i) tc_commit(&sm.o_final[i]);
                             }
                             __syncwarp();
@@ -448,95 +502,102 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             tc_fence_after();
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 1);
 
-            float s[kBlockN];
-#pragma unroll
-            for (int ch = 0; ch < kBlockN / 32; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(s_tmem + ch * 32, r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[ch * 32 + e] = __uint_as_float(r[e]);
-            }
+            // Scores of this row: two halves, the max of the first half overlaps
+            // the load of the second.
+            uint32_t sr[kBlockN];
+            tmem_ld32(s_tmem + 0, sr + 0);
+            tmem_ld32(s_tmem + 32, sr + 32);
             tmem_wait_ld();
-            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 2);
+            reg_fence32(sr + 0);
+            reg_fence32(sr + 32);
+            tmem_ld32(s_tmem + 64, sr + 64);
+            tmem_ld32(s_tmem + 96, sr + 96);
+            float *s = reinterpret_cast<float *>(sr);
 
             const int key0 = j * kBlockN;
             const bool need_mask = key0 < kr.lo || key0 + kBlockN - 1 > kr.hi;
             const bool masked = __any_sync(0xffffffffu, need_mask);
             if (masked) {
 #pragma unroll
-                for (int e = 0; e < kBlockN; ++e) {
+                for (int e = 0; e < kBlockN / 2; ++e) {
                     const int key = key0 + e;
                     if (key < kr.lo || key > kr.hi) s[e] = -INFINITY;
                 }
             }
-            float mx[8];
+            float mx[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx[e] = s[e];
+            for (int u = 0; u < 4; ++u) mx[u] = fmax3(s[u], s[u + 4], s[u + 8]);
 #pragma unroll
-            for (int e = 8; e < kBlockN; ++e) mx[e & 7] = fmaxf(mx[e & 7], s[e]);
-            const float row_max =
-                fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            for (int e = 12; e < kBlockN / 2 - 4; e += 8)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], s[e + u], s[e + 4 + u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) mx[u] = fmaxf(mx[u], s[kBlockN / 2 - 4 + u]);
+            tmem_wait_ld();
+            reg_fence32(sr + 64);
+            reg_fence32(sr + 96);
+            if (masked) {
+#pragma unroll
+                for (int e = kBlockN / 2; e < kBlockN; ++e) {
+                    const int key = key0 + e;
+                    if (key < kr.lo || key > kr.hi) s[e] = -INFINITY;
+                }
+            }
+#pragma unroll
+            for (int e = kBlockN / 2; e < kBlockN; e += 8)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], s[e + u], s[e + 4 + u]);
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 2);
+            const float row_max = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
             const float m_cand = row_max * c;
             float alpha = 1.0f;
             if (m_cand > m_run + tau) {
                 alpha = ex2_mufu(m_run - m_cand);
                 m_run = m_cand;
             }
-            const float m_use = m_run == -INFINITY ? 0.0f : m_run;
+            const float neg_m = m_run == -INFINITY ? 0.0f : -m_run;
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 3);
 
             l_run *= alpha;
 
-            // Probabilities: p = 2^(x - m), row sum, bf16 pairs into TMEM.
-            float sum[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sum[e] = 0.0f;
-            uint32_t pk[kBlockN / 2];
-            if (masked) {
-#pragma unroll
-                for (int e = 0; e < kBlockN; e += 2) {
-                    const float p0 = ex2_mufu(fmaf(s[e], c, -m_use));
-                    const float p1 = ex2_mufu(fmaf(s[e + 1], c, -m_use));
-                    sum[(e >> 1) & 7] += p0 + p1;
-                    pk[e >> 1] = pack_bf16x2(p0, p1);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < kBlockN; e += 2) {
-                    const float x0 = fmaf(s[e], c, -m_use);
-                    const float x1 = fmaf(s[e + 1], c, -m_use);
-                    const float p0 = use_poly<EXP_MODE>(e) ? ex2_poly(x0) : ex2_mufu(x0);
-                    const float p1 = use_poly<EXP_MODE>(e + 1) ? ex2_poly(x1) : ex2_mufu(x1);
-                    sum[(e >> 1) & 7] += p0 + p1;
-                    pk[e >> 1] = pack_bf16x2(p0, p1);
-                }
-            }
-            l_run += ((sum[0] + sum[1]) + (sum[2] + sum[3])) +
-                     ((sum[4] + sum[5]) + (sum[6] + sum[7]));
-            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
-#pragma unroll
-            for (int h = 0; h < kBlockN / 64; ++h) {
-                uint32_t r[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = pk[h * 32 + e];
-                tmem_st32(s_tmem + h * 32, r);
-            }
-            // Correction: rescale this row of O in TMEM (rare once the max
-            // settles).  PV of the previous block is complete: the commit that
-            // signalled S of this block covers every earlier MMA.
+            // Correction first: rescale this row of O in TMEM (rare once the
+            // max settles) before any P of this block is handed over.  PV of
+            // the previous block is complete: the commit that signalled S of
+            // this block covers every earlier MMA.
             if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
                 for (int ch = 0; ch < D / 32; ++ch) {
                     uint32_t r[32];
                     tmem_ld32(o_tmem + ch * 32, r);
                     tmem_wait_ld();
+                    reg_fence32(r);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                    for (int e = 0; e < 32; e += 2) {
+                        float a0, a1;
+                        mul2(a0, a1, __uint_as_float(r[e]), __uint_as_float(r[e + 1]), alpha,
+                             alpha);
+                        r[e] = __float_as_uint(a0);
+                        r[e + 1] = __float_as_uint(a1);
+                    }
                     tmem_st32(o_tmem + ch * 32, r);
                 }
             }
+
+            // Probabilities p = 2^(s*c - m) in pairs, row sum, bf16 pairs to
+            // TMEM, in two halves: the MMA warp starts PV on keys [0, 64) while
+            // this warp computes keys [64, 128).  Masked blocks (-inf scores)
+            // use MUFU only: ex2(-inf) = 0 exactly.
+            uint32_t pk[kBlockN / 2];
+            l_run += masked ? exp_pack_half<0>(s, c, neg_m, pk)
+                            : exp_pack_half<EXP_MODE>(s, c, neg_m, pk);
+            tmem_st32(s_tmem + 0, pk + 0);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.p_half[i]);
+            l_run += masked ? exp_pack_half<0>(s + 64, c, neg_m, pk + 32)
+                            : exp_pack_half<EXP_MODE>(s + 64, c, neg_m, pk + 32);
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
+            tmem_st32(s_tmem + 32, pk + 32);
             tmem_wait_st();
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 5);
             tc_fence_before();
@@ -561,6 +622,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 if (has_blocks) {
                     tmem_ld32(o_tmem + ch * 32, r);
                     tmem_wait_ld();
+                    reg_fence32(r);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) r[e] = 0u;
