@@ -119,6 +119,18 @@ attn_status_t launch_fwd(const tab::FwdParams &p, int grid, cudaStream_t stream)
     });
     if (attr_err[dev] != cudaSuccess)
         return fail(ATTN_ERR_LAUNCH, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err[dev]));
+    // The kernel moves registers between warpgroups with setmaxnreg; if the
+    // compiled per-thread count does not cover the split, the increase would
+    // wait forever, so never launch such a build.
+    static cudaFuncAttributes attrs[kMaxDevices];
+    static cudaError_t attrs_err[kMaxDevices];
+    static std::once_flag attrs_once[kMaxDevices];
+    std::call_once(attrs_once[dev], [&]() { attrs_err[dev] = cudaFuncGetAttributes(&attrs[dev], kernel); });
+    if (attrs_err[dev] != cudaSuccess)
+        return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes: %s", cudaGetErrorString(attrs_err[dev]));
+    if (attrs[dev].numRegs < tab::kLaunchRegs)
+        return fail(ATTN_ERR_LAUNCH, "kernel compiled with %d registers per thread, %d needed",
+                    attrs[dev].numRegs, tab::kLaunchRegs);
     kernel<<<grid, tab::kFwdThreads, smem, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ATTN_ERR_LAUNCH, "launch: %s", cudaGetErrorString(e));

@@ -51,9 +51,14 @@ constexpr int kBlockM = 128;   // query rows per tile = TMEM lanes
 constexpr int kBlockN = 128;   // keys per key/value block
 constexpr int kFwdThreads = 384;
 constexpr int kTmemCols = 512;
+// Registers: 384 threads launch with 168 each (65536 / 384, in steps of 8).
+// setmaxnreg moves them from the MMA / TMA warpgroup to the two softmax
+// warpgroups; the split must not exceed the launch allocation (a larger
+// request would wait forever), and the host checks the compiled count.
+constexpr int kLaunchRegs = 168;
 constexpr int kSoftmaxRegs = 216;
 constexpr int kOtherRegs = 72;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kFwdThreads * 168,
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kFwdThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int kStatusTimeout = 5;                   // ATTN_ERR_DEVICE_TIMEOUT
@@ -186,15 +191,17 @@ __device__ __forceinline__ void ex2_poly2(float &y0, float &y1, float x0, float 
     y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
-// Columns (out of every 32) that use the polynomial in EXP_MODE 1 (taken in
-// pairs: both columns of a pair use the same unit).
-constexpr int kPolyPer32 = 12;
-
+// Column pairs that use the polynomial in EXP_MODE 1: one pair in eight,
+// spread through the row so MUFU and FMA work interleave.  (Measured on
+// B200 for the causal S=8192 forward: 1/8 of pairs is the fastest split; a
+// quarter, two fifths, a half and a clustered 12-of-32 split are slower, and
+// all-polynomial is slowest: the cubic costs more FMA-pipe cycles per element
+// than one MUFU ex2, so it only pays where it fills MUFU stalls.)
 template <int EXP_MODE>
 __device__ __forceinline__ bool use_poly(int col) {
     if (EXP_MODE == 0) return false;
     if (EXP_MODE == 2) return true;
-    return (col & 31) < kPolyPer32;
+    return ((col >> 1) & 7) == 3;
 }
 
 // Half a row of a block: p = 2^(s*c - m) for 64 scores (packed pairs), the
