@@ -1,0 +1,102 @@
+"""Host-side logic of bench.py on the CPU: FLOP accounting, the reduction
+of timings over ranks (world size 2 on gloo), and the reference arm's
+rank handling.  The path needs no data exchange between GPUs (replicas
+only); ranks meet only to start and stop the clock."""
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+from tiled_attention_blackwell_b200.workloads import WORKLOADS, Workload, useful_flops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        dev = torch.device("cpu")
+        ms = [12.5, 17.0][rank]
+        out[rank] = (bench.max_over_ranks(ms, world, dev), bench.sum_over_ranks(ms, world, dev))
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_and_sum_over_two_gloo_ranks():
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert res[0] == res[1] == (17.0, 29.5)
+
+
+def test_single_rank_reductions_are_identity():
+    dev = torch.device("cpu")
+    assert bench.max_over_ranks(3.0, 1, dev) == 3.0
+    assert bench.sum_over_ranks(3.0, 1, dev) == 3.0
+
+
+@pytest.mark.parametrize("name", ["causal_s8192", "gqa_doc_s16384", "outlier_s4096",
+                                  "tiny_d64"])
+def test_row_key_counts_match_dense_mask(name):
+    """The per-row key counts used for the CPU sample's FLOPs equal the
+    allowed-set sizes of the mask, on a shrunken copy of the workload."""
+    w0 = WORKLOADS[name]
+    S = 1000
+    w = Workload(name, 1, 1, 1, S, w0.D, w0.causal, w0.seed, doc_lengths=w0.doc_lengths)
+    docs = None
+    if w.doc_lengths:
+        docs = np.array([0, 130, 131, 600, 1000], dtype=np.int32)
+    keys = bench.allowed_keys_per_row(w, docs)
+    i = np.arange(S)[:, None]
+    j = np.arange(S)[None, :]
+    allowed = np.ones((S, S), dtype=bool)
+    if w.causal:
+        allowed &= j <= i
+    if docs is not None:
+        ids = np.repeat(np.arange(len(docs) - 1), np.diff(docs))
+        allowed &= ids[:, None] == ids[None, :]
+    np.testing.assert_array_equal(keys, allowed.sum(axis=1))
+    # and the whole-workload convention: causal = half of the square
+    if docs is None:
+        full = useful_flops(1, 1, S, S, w.D, causal=w.causal)
+        expect = 4.0 * w.D * (S * S / 2 if w.causal else S * S)
+        assert full == expect
+
+
+def test_reference_arm_other_ranks_exit_silently():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", "--config", "tiny_d64"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_prints_one_json_line():
+    import json
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", "--config", "tiny_d64"], cwd=ROOT,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [x for x in r.stdout.splitlines() if x.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["higher_is_better"] is True
