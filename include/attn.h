@@ -110,6 +110,35 @@ ATTN_API attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, 
                           const int *doc_offsets, int num_docs,
                           const attn_fwd_options_t *opts, void *stream);
 
+/*
+ * Backward ("Hardware-Aware FP4 FlashAttention-4", "Causal Backward
+ * Cuantizado": gradients from the saved LSE, probabilities rebuilt rather
+ * than stored).  For L with dO = dL/dO:
+ *   D_i   = sum_d dO[b,i,hq,d] * O[b,i,hq,d]
+ *   P_ij  = exp(s_ij - LSE[b,hq,i])           (allowed keys, else 0)
+ *   dS_ij = P_ij * (<dO_i, v_j> - D_i)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j  = scale * sum_i dS_ij q_i            (summed over the query heads
+ *   dV_j  =         sum_i P_ij dO_i             of a GQA group)
+ * Inputs: q, k, v as for attn_fwd; o (bf16 [B,Sq,Hq,D]) and lse (fp32
+ * [B,Hq,Sq]) from attn_fwd on the same inputs and mask; dout bf16
+ * [B,Sq,Hq,D].  Outputs: dq fp32 [B,Sq,Hq,D]; dk, dv bf16 [B,Sk,Hkv,D].
+ * Every output element is written.  workspace: device memory of at least
+ * attn_bwd_workspace_size() bytes, 16-byte aligned, owned by the caller
+ * (holds D_i between the kernels of one call; contents on entry ignored).
+ * Same shape, mask and alignment rules as attn_fwd (dq, dk, dv, o, dout
+ * 16-byte aligned).  The result is deterministic (no atomics).  Calls are
+ * asynchronous on `stream`.
+ */
+ATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D);
+
+ATTN_API attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                                const float *lse, const void *dout, float *dq, void *dk,
+                                void *dv, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                                float scale, int causal, int window_left, int window_right,
+                                const int *doc_offsets, int num_docs, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
 /* Synchronises `stream`, then reads and clears the device status word of
  * the current device.  Returns ATTN_OK or ATTN_ERR_DEVICE_TIMEOUT (or
  * ATTN_ERR_CUDA if the synchronisation itself failed). */

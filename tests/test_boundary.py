@@ -121,6 +121,40 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
     assert call(L) == attn.ATTN_ERR_CUDA
 
 
+def call_bwd(L, **kw):
+    a = dict(ptr=P, lse=P, ws=P, B=1, Hq=2, Hkv=2, Sq=16, Sk=16, D=128, scale=0.1, causal=1,
+             wl=-1, wr=-1, docs=None, nd=0, wsb=1 << 20)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    ptrs = [vp(a.get(n, a["ptr"])) for n in ("q", "k", "v", "o")]
+    ptrs += [vp(a["lse"])]
+    ptrs += [vp(a.get(n, a["ptr"])) for n in ("dout", "dq", "dk", "dv")]
+    return L.attn_bwd(*ptrs, a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Sk"], a["D"], a["scale"],
+                      a["causal"], a["wl"], a["wr"], vp(a["docs"]) if a["docs"] else None, a["nd"],
+                      vp(a["ws"]), a["wsb"], None)
+
+
+def test_bwd_workspace_size(L):
+    assert L.attn_bwd_workspace_size(2, 16, 16, 4096, 4096, 128) >= 2 * 16 * 4096 * 4
+    assert L.attn_bwd_workspace_size(2, 16, 16, 4096, 4096, 128) % 256 == 0
+    assert L.attn_bwd_workspace_size(0, 16, 16, 4096, 4096, 128) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dq=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(ws=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), attn.ATTN_ERR_INVALID_ARG),
+    (dict(D=80), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=0.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(wsb=64), attn.ATTN_ERR_INVALID_ARG),
+    (dict(dk=P + 8), attn.ATTN_ERR_MISALIGNED),
+    (dict(ws=P + 4), attn.ATTN_ERR_MISALIGNED),
+    (dict(docs=P, nd=1, Sk=20), attn.ATTN_ERR_INVALID_ARG),
+])
+def test_bwd_invalid_arguments_rejected_before_launch(L, kw, status):
+    assert call_bwd(L, **kw) == status
+
+
 def test_binding_refuses_cpu_tensors(L):
     q = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
     lse = torch.zeros(1, 1, 4)

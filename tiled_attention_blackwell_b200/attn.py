@@ -25,8 +25,9 @@ ATTN_ERR_LAUNCH = 4
 ATTN_ERR_DEVICE_TIMEOUT = 5
 ATTN_ERR_CUDA = 6
 
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_default_options", "attn_get_device_status",
-            "attn_status_string", "attn_last_error_detail", "attn_abi_version")
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_default_options", "attn_bwd",
+            "attn_bwd_workspace_size", "attn_get_device_status", "attn_status_string",
+            "attn_last_error_detail", "attn_abi_version")
 
 
 class AttnError(RuntimeError):
@@ -71,6 +72,13 @@ def lib():
             L.attn_last_error_detail.restype = ctypes.c_char_p
             L.attn_last_error_detail.argtypes = []
             L.attn_abi_version.restype = ctypes.c_int
+            L.attn_bwd_workspace_size.restype = ctypes.c_size_t
+            L.attn_bwd_workspace_size.argtypes = [ctypes.c_int] * 6
+            L.attn_bwd.restype = ctypes.c_int
+            L.attn_bwd.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 6 + \
+                [ctypes.c_float] + [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int,
+                                                         ctypes.c_void_p, ctypes.c_size_t,
+                                                         ctypes.c_void_p]
             _lib = L
     return _lib
 
@@ -146,6 +154,63 @@ def attention(q, k, v, *, scale=None, causal=False, window=None, doc_offsets=Non
     attn_fwd(q, k, v, o, lse, scale=scale, causal=causal, window=window,
              doc_offsets=doc_offsets, options=options, stream=stream)
     return o, lse
+
+
+def bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D) -> int:
+    """Bytes of device workspace attn_bwd needs."""
+    return int(lib().attn_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D))
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, *, scale, causal=False, window=None,
+             doc_offsets=None, stream=None):
+    """Enqueue the backward on `stream`.  dq fp32 [B,Sq,Hq,D]; dk, dv bf16
+    [B,Sk,Hkv,D]; workspace a CUDA uint8 tensor of at least
+    bwd_workspace_size() bytes."""
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
+                        ("v", v, torch.bfloat16), ("o", o, torch.bfloat16),
+                        ("lse", lse, torch.float32), ("dout", dout, torch.bfloat16),
+                        ("dq", dq, torch.float32), ("dk", dk, torch.bfloat16),
+                        ("dv", dv, torch.bfloat16)):
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA {dt} tensor")
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise TypeError("workspace must be a contiguous CUDA tensor")
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    if doc_offsets is not None:
+        if doc_offsets.dtype != torch.int32 or not doc_offsets.is_cuda:
+            raise TypeError("doc_offsets must be a CUDA int32 tensor")
+        docs_ptr, nd = _ptr(doc_offsets), doc_offsets.numel() - 1
+    else:
+        docs_ptr, nd = None, 0
+    st = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                        _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, D, float(scale),
+                        int(bool(causal)), wl, wr, docs_ptr, nd, _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(st, "attn_bwd")
+
+
+def attention_backward(q, k, v, o, lse, dout, *, scale=None, causal=False, window=None,
+                       doc_offsets=None, stream=None):
+    """Allocate dQ (fp32), dK, dV (bf16) and the workspace with torch and run
+    the backward.  Returns (dQ, dK, dV)."""
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    ws = torch.empty(bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D), dtype=torch.uint8,
+                     device=q.device)
+    if doc_offsets is not None and not torch.is_tensor(doc_offsets):
+        doc_offsets = torch.as_tensor(doc_offsets, dtype=torch.int32)
+    if doc_offsets is not None and not doc_offsets.is_cuda:
+        doc_offsets = doc_offsets.to(q.device)
+    attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, ws, scale=scale, causal=causal, window=window,
+             doc_offsets=doc_offsets, stream=stream)
+    return dq, dk, dv
 
 
 def device_status(stream=None) -> int:

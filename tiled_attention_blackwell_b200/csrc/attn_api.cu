@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
 
 namespace {
@@ -151,6 +152,79 @@ attn_status_t dispatch_exp(const tab::FwdParams &p, int grid, int exp_mode, cuda
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Shape and mask checks shared by the forward and the backward.
+attn_status_t check_common(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                           int window_left, int window_right, const int *doc_offsets,
+                           int num_docs) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1)
+        return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, Sq, Sk must be >= 1");
+    if (Hq % Hkv != 0)
+        return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (D != 64 && D != 128)
+        return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (built: 64, 128)", D);
+    if (!(scale > 0.0f) || !std::isfinite(scale))
+        return fail(ATTN_ERR_INVALID_ARG, "scale must be positive and finite");
+    if (window_left < -1 || window_right < -1)
+        return fail(ATTN_ERR_INVALID_ARG, "window bounds must be -1 or >= 0");
+    if ((doc_offsets == nullptr) != (num_docs == 0) || num_docs < 0)
+        return fail(ATTN_ERR_INVALID_ARG, "doc_offsets and num_docs must be given together");
+    if (doc_offsets && Sq != Sk)
+        return fail(ATTN_ERR_INVALID_ARG, "a document mask requires Sq == Sk");
+    const double max_stride = (double)std::max(Sq, Sk) * Hq * D * 4.0;
+    if (max_stride >= 1099511627776.0)
+        return fail(ATTN_ERR_UNSUPPORTED, "tensor too large for a TMA descriptor");
+    return ATTN_OK;
+}
+
+template <class Kernel>
+attn_status_t prepare_kernel(Kernel kernel, size_t smem, int threads, int min_regs) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess)
+        return fail(ATTN_ERR_LAUNCH, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    cudaFuncAttributes attrs;
+    e = cudaFuncGetAttributes(&attrs, kernel);
+    if (e != cudaSuccess)
+        return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes: %s", cudaGetErrorString(e));
+    if (attrs.numRegs < min_regs || attrs.maxThreadsPerBlock < threads)
+        return fail(ATTN_ERR_LAUNCH, "kernel build cannot be launched (%d regs, %d threads)",
+                    attrs.numRegs, attrs.maxThreadsPerBlock);
+    return ATTN_OK;
+}
+
+constexpr int kBwdStagesQ = 2;
+constexpr int kBwdStagesKV = 4;
+
+template <int D>
+attn_status_t launch_bwd(const tab::BwdParams &p, cudaStream_t stream) {
+    using DkdvS = tab::DkdvSmem<D, kBwdStagesQ>;
+    using DqS = tab::DqSmem<D, kBwdStagesKV>;
+    constexpr size_t smem_dkdv = sizeof(DkdvS) + 1024;
+    constexpr size_t smem_dq = sizeof(DqS) + 1024;
+    static_assert(smem_dkdv <= 232448 && smem_dq <= 232448, "shared memory budget");
+    auto k_pre = tab::attn_bwd_preprocess_kernel<D>;
+    auto k_dkdv = tab::attn_bwd_dkdv_kernel<D, kBwdStagesQ>;
+    auto k_dq = tab::attn_bwd_dq_kernel<D, kBwdStagesKV>;
+    static std::once_flag once[kMaxDevices];
+    static attn_status_t prep[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::call_once(once[dev], [&]() {
+        prep[dev] = prepare_kernel(k_dkdv, smem_dkdv, tab::kBwdThreads, 0);
+        if (prep[dev] == ATTN_OK) prep[dev] = prepare_kernel(k_dq, smem_dq, tab::kBwdThreads, 0);
+    });
+    if (prep[dev] != ATTN_OK) return fail(prep[dev], "backward kernels could not be prepared");
+    const long long rows = (long long)p.B * p.Sq * p.Hq;
+    k_pre<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);
+    k_dkdv<<<p.num_kb * p.Hkv * p.B, tab::kBwdThreads, smem_dkdv, stream>>>(p);
+    k_dq<<<p.num_qb * p.Hq * p.B, tab::kBwdThreads, smem_dq, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ATTN_ERR_LAUNCH, "launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 #ifdef ATTN_TRACE
 long long *g_trace = nullptr;
 int g_trace_ctas = 0;
@@ -179,20 +253,11 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
     // ----- validation (no CUDA call before this block completes)
     if (!q || !k || !v || !o || !lse)
         return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
-    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1)
-        return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, Sq, Sk must be >= 1");
-    if (Hq % Hkv != 0)
-        return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
-    if (D != 64 && D != 128)
-        return fail(ATTN_ERR_UNSUPPORTED, "head dim %d (built: 64, 128)", D);
-    if (!(scale > 0.0f) || !std::isfinite(scale))
-        return fail(ATTN_ERR_INVALID_ARG, "scale must be positive and finite");
-    if (window_left < -1 || window_right < -1)
-        return fail(ATTN_ERR_INVALID_ARG, "window bounds must be -1 or >= 0");
-    if ((doc_offsets == nullptr) != (num_docs == 0) || num_docs < 0)
-        return fail(ATTN_ERR_INVALID_ARG, "doc_offsets and num_docs must be given together");
-    if (doc_offsets && Sq != Sk)
-        return fail(ATTN_ERR_INVALID_ARG, "a document mask requires Sq == Sk");
+    {
+        attn_status_t c = check_common(B, Hq, Hkv, Sq, Sk, D, scale, window_left, window_right,
+                                       doc_offsets, num_docs);
+        if (c != ATTN_OK) return c;
+    }
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
         return fail(ATTN_ERR_MISALIGNED, "q, k, v, o must be 16-byte aligned");
     if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
@@ -203,10 +268,6 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
         return fail(ATTN_ERR_INVALID_ARG, "exp2_mode must be 0, 1 or 2");
     for (int r : op.reserved)
         if (r != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved option fields must be zero");
-    // TMA limits: every byte stride below 2^40.
-    const double max_stride = (double)std::max(Sq, Sk) * Hq * D * 2.0;
-    if (max_stride >= 1099511627776.0)
-        return fail(ATTN_ERR_UNSUPPORTED, "tensor too large for a TMA descriptor");
     const long long num_qblocks = (Sq + 2LL * tab::kBlockM - 1) / (2LL * tab::kBlockM);
     const long long grid = num_qblocks * Hq * B;
     if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
@@ -254,6 +315,72 @@ attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, flo
                        const int *doc_offsets, int num_docs, void *stream) {
     return attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, window_left,
                        window_right, doc_offsets, num_docs, nullptr, stream);
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
+    (void)Hkv;
+    (void)Sk;
+    (void)D;
+    if (B < 1 || Hq < 1 || Sq < 1) return 0;
+    const size_t n = (size_t)B * Hq * Sq * sizeof(float);
+    return (n + 255) & ~(size_t)255;
+}
+
+attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *o,
+                       const float *lse, const void *dout, float *dq, void *dk, void *dv,
+                       int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                       int window_left, int window_right, const int *doc_offsets, int num_docs,
+                       void *workspace, size_t workspace_bytes, void *stream) {
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+        return fail(ATTN_ERR_INVALID_ARG, "null pointer");
+    attn_status_t s = check_common(B, Hq, Hkv, Sq, Sk, D, scale, window_left, window_right,
+                                   doc_offsets, num_docs);
+    if (s != ATTN_OK) return s;
+    for (const void *ptr : {q, k, v, o, dout, (const void *)dq, (const void *)dk, (const void *)dv,
+                            (const void *)workspace})
+        if (!aligned16(ptr)) return fail(ATTN_ERR_MISALIGNED, "tensors and workspace must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+        return fail(ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
+    const size_t need = attn_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D);
+    if (workspace_bytes < need)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+    const long long num_qb = (Sq + 127LL) / 128, num_kb = (Sk + 127LL) / 128;
+    if (num_qb * Hq * B > 0x7fffffffLL || num_kb * Hkv * B > 0x7fffffffLL)
+        return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+
+    DeviceState *st = nullptr;
+    if ((s = device_state(&st)) != ATTN_OK) return s;
+    tab::BwdParams p;
+    memset(&p, 0, sizeof p);
+    if ((s = make_map(&p.tm_q, q, B, Sq, Hq, D)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_do, dout, B, Sq, Hq, D)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_k, k, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_v, v, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    p.o = static_cast<const __nv_bfloat16 *>(o);
+    p.dout = static_cast<const __nv_bfloat16 *>(dout);
+    p.lse = lse;
+    p.dval = static_cast<float *>(workspace);
+    p.dq = dq;
+    p.dk = static_cast<__nv_bfloat16 *>(dk);
+    p.dv = static_cast<__nv_bfloat16 *>(dv);
+    p.doc_offsets = doc_offsets;
+    p.num_docs = num_docs;
+    p.status = st->status;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.group = Hq / Hkv;
+    p.causal = causal ? 1 : 0;
+    p.window_left = window_left;
+    p.window_right = window_right;
+    p.num_qb = (int)num_qb;
+    p.num_kb = (int)num_kb;
+    p.scale = scale;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    return D == 128 ? launch_bwd<128>(p, cs) : launch_bwd<64>(p, cs);
 }
 
 attn_status_t attn_get_device_status(void *stream) {

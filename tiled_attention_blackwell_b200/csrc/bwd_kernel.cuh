@@ -1,0 +1,755 @@
+// Fused exact-attention backward for B200 (sm_100a).
+//
+// Gradients of O = softmax(scale * Q K^T + mask) V given dO, rebuilding the
+// probabilities from the forward's LSE instead of storing them
+// ("Hardware-Aware FP4 FlashAttention-4", "Causal Backward Cuantizado": the
+// backward reconstructs the probabilities from the saved normaliser;
+// "FlashAttention-4发布", "从V1到V4", first bullet: recomputation).  With
+// D_i = sum_d dO_id O_id, P = exp(s - LSE), dP = dO V^T, dS = P (dP - D):
+//   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+//
+// Three kernels, no atomics (deterministic):
+//   attn_bwd_preprocess_kernel  D_i into the caller's workspace
+//   attn_bwd_dkdv_kernel        one CTA per (batch, kv head, 128-key block):
+//                               keys in TMEM lanes, S^T = K Q^T and
+//                               dP^T = V dO^T per query block, P^T and dS^T
+//                               written back into TMEM as bf16, then
+//                               dV += P^T dO and dK += dS^T Q (A from TMEM);
+//                               the query heads of a GQA group accumulate
+//                               into the same TMEM.
+//   attn_bwd_dq_kernel          one CTA per (batch, query head, 128-row
+//                               block): S = Q K^T, dP = dO V^T, dS into
+//                               TMEM, dQ += dS K.
+// Warp roles in both main kernels (192 threads): warps 0-3 elementwise
+// (one TMEM lane each), warp 4 MMA issue (warp-uniform, one elected lane),
+// warp 5 TMA producer.  Every wait is bounded as in the forward.
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace tab {
+
+constexpr int kBwdThreads = 192;
+constexpr int kBwdMmaWarp = 4;
+constexpr int kBwdLoadWarp = 5;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdParams {
+    CUtensorMap tm_q;   // bf16 [B][Sq][Hq][D], box (64, 128, 1, 1)
+    CUtensorMap tm_do;  // bf16 [B][Sq][Hq][D]
+    CUtensorMap tm_k;   // bf16 [B][Sk][Hkv][D]
+    CUtensorMap tm_v;
+    const __nv_bfloat16 *o;
+    const __nv_bfloat16 *dout;
+    const float *lse;   // [B][Hq][Sq], natural log
+    float *dval;        // workspace: D_i, [B][Hq][Sq]
+    float *dq;          // fp32 [B][Sq][Hq][D]
+    __nv_bfloat16 *dk;  // bf16 [B][Sk][Hkv][D]
+    __nv_bfloat16 *dv;
+    const int *doc_offsets;
+    int *status;
+    int num_docs;
+    int B, Hq, Hkv, Sq, Sk, group;
+    int causal, window_left, window_right;
+    int num_qb, num_kb;  // 128-row query blocks, 128-key blocks
+    float scale;
+    float scale_log2;
+};
+
+// --------------------------------------------------------------- preprocess
+
+// One warp per (b, i, hq) row: D_i = sum_d dO_id * O_id in fp32.
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const BwdParams p) {
+    const long long rows = (long long)p.B * p.Sq * p.Hq;
+    const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (w >= rows) return;
+    const int lane = threadIdx.x & 31;
+    float acc = 0.0f;
+    for (int d = lane * 4; d < D; d += 128) {
+        const uint2 ov = *reinterpret_cast<const uint2 *>(p.o + w * D + d);
+        const uint2 gv = *reinterpret_cast<const uint2 *>(p.dout + w * D + d);
+        const __nv_bfloat162 *o2 = reinterpret_cast<const __nv_bfloat162 *>(&ov);
+        const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&gv);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const float2 of = __bfloat1622float2(o2[e]);
+            const float2 gf = __bfloat1622float2(g2[e]);
+            acc = fmaf(of.x, gf.x, acc);
+            acc = fmaf(of.y, gf.y, acc);
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+        const int hq = (int)(w % p.Hq);
+        const int i = (int)((w / p.Hq) % p.Sq);
+        const int b = (int)(w / ((long long)p.Hq * p.Sq));
+        p.dval[((size_t)b * p.Hq + hq) * p.Sq + i] = acc;
+    }
+}
+
+// --------------------------------------------------------------- dK and dV
+
+template <int D, int NSQ>
+struct DkdvSmem {
+    static constexpr int kChunks = D / 64;
+    static constexpr int kChunkElems = 128 * 64;  // 16 KB
+    __nv_bfloat16 k[kChunks][kChunkElems];
+    __nv_bfloat16 v[kChunks][kChunkElems];
+    __nv_bfloat16 q[NSQ][kChunks][kChunkElems];
+    __nv_bfloat16 dout[NSQ][kChunks][kChunkElems];
+    float lse2[NSQ][128];  // LSE * log2(e) of the block's rows (+inf past Sq)
+    float dval[NSQ][128];  // D_i of the block's rows (0 past Sq)
+    int rlo[NSQ][128];     // key interval of each row (lo > hi: none)
+    int rhi[NSQ][128];
+    int full[NSQ];         // every (row, key) pair of the item is allowed
+    uint64_t kv_full;
+    uint64_t st_full[NSQ];
+    uint64_t st_empty[NSQ];
+    uint64_t s_full, dp_full, p_ready, ds_ready, final_bar, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int qb_lo, qb_hi;
+};
+
+template <int D, int NSQ>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+    using Smem = DkdvSmem<D, NSQ>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_off = smem_u32(smem_raw);
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (raw_off & 1023u)) & 1023u));
+    const int warp = warp_id();
+    const int lane = lane_id();
+
+    // Work item: lowest key blocks first (under a causal mask they see the
+    // most query blocks), then (batch, kv head).
+    const int bh_count = p.Hkv * p.B;
+    const int kb = (int)(blockIdx.x / bh_count);
+    const int bh = (int)(blockIdx.x % bh_count);
+    const int hkv = bh % p.Hkv;
+    const int b = bh / p.Hkv;
+    const int k0 = kb * 128;
+    const int k1 = min(k0 + 127, p.Sk - 1);
+    constexpr uint32_t kTileBytes = 128 * D * 2;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.kv_full, 1);
+        for (int s = 0; s < NSQ; ++s) {
+            mbar_init(&sm.st_full[s], 32);
+            mbar_init(&sm.st_empty[s], 1);
+        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.dp_full, 1);
+        mbar_init(&sm.p_ready, 128);
+        mbar_init(&sm.ds_ready, 128);
+        mbar_init(&sm.final_bar, 1);
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kBwdLoadWarp) {
+        // Query blocks whose rows can see this key block: the first and last
+        // rows of a block bound its rows' key intervals (the intervals'
+        // ends never decrease with the row), so a block is kept when its
+        // first row's lower end is <= k1 and its last row's upper end is
+        // >= k0.  Rows without keys count as (-1, -1).
+        int lo = 0x7fffffff, hi = -1;
+        for (int qb = lane; qb < p.num_qb; qb += 32) {
+            const int r0 = qb * 128;
+            const int r1 = min(r0 + 127, p.Sq - 1);
+            KeyRange a = row_key_range(p, r0);
+            KeyRange z = row_key_range(p, r1);
+            const int a_lo = a.lo <= a.hi ? a.lo : -1;
+            const int z_hi = z.lo <= z.hi ? z.hi : -1;
+            if (a_lo <= k1 && z_hi >= k0) {
+                lo = min(lo, qb);
+                hi = max(hi, qb);
+            }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        if (lane == 0) {
+            sm.qb_lo = lo;
+            sm.qb_hi = hi;
+        }
+    }
+    if (warp == kBwdMmaWarp) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort_flag;
+    const int qb_lo = sm.qb_lo, qb_hi = sm.qb_hi;
+    const int n_qb = qb_hi >= qb_lo ? qb_hi - qb_lo + 1 : 0;
+    const int n_items = n_qb * p.group;  // (query head in group, query block)
+    // TMEM columns: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D)
+    constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+
+    if (warp == kBwdLoadWarp) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&p.tm_q);
+            prefetch_tensormap(&p.tm_do);
+            prefetch_tensormap(&p.tm_k);
+            prefetch_tensormap(&p.tm_v);
+            mbar_arrive_expect_tx(&sm.kv_full, 2 * kTileBytes);
+            for (int c = 0; c < Smem::kChunks; ++c) {
+                tma_load_4d(sm.k[c], &p.tm_k, &sm.kv_full, c * 64, k0, hkv, b);
+                tma_load_4d(sm.v[c], &p.tm_v, &sm.kv_full, c * 64, k0, hkv, b);
+            }
+        }
+        __syncwarp();
+        bool ok = true;
+        int issued = 0;
+        for (int it = 0; it < n_items && ok; ++it) {
+            const int s = it % NSQ;
+            const int g = it / n_qb;
+            const int qb = qb_lo + it % n_qb;
+            const int hq = hkv * p.group + g;
+            ok = __all_sync(0xffffffffu, wait_bounded(&sm.st_empty[s], ((it / NSQ) & 1) ^ 1,
+                                                      abort_flag, p.status));
+            if (!ok) break;
+            // Per-row data of this query block.
+            bool full = true;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int idx = lane + 32 * m;
+                const int r = qb * 128 + idx;
+                float l2 = INFINITY, dv = 0.0f;
+                KeyRange kr = {1, 0};
+                if (r < p.Sq) {
+                    const size_t ri = ((size_t)b * p.Hq + hq) * p.Sq + r;
+                    l2 = __ldg(p.lse + ri) * kLog2e;
+                    dv = p.dval[ri];
+                    kr = row_key_range(p, r);
+                }
+                sm.lse2[s][idx] = l2;
+                sm.dval[s][idx] = dv;
+                sm.rlo[s][idx] = kr.lo;
+                sm.rhi[s][idx] = kr.hi;
+                full = full && r < p.Sq && kr.lo <= k0 && kr.hi >= k1;
+            }
+            full = __all_sync(0xffffffffu, full);
+            if (lane == 0) {
+                sm.full[s] = full ? 1 : 0;
+                mbar_arrive_expect_tx(&sm.st_full[s], 2 * kTileBytes);
+                for (int c = 0; c < Smem::kChunks; ++c) {
+                    tma_load_4d(sm.q[s][c], &p.tm_q, &sm.st_full[s], c * 64, qb * 128, hq, b);
+                    tma_load_4d(sm.dout[s][c], &p.tm_do, &sm.st_full[s], c * 64, qb * 128, hq, b);
+                }
+            } else {
+                mbar_arrive(&sm.st_full[s]);
+            }
+            ++issued;
+        }
+        // Copies still in flight land before the CTA can exit.
+        wait_bounded(&sm.kv_full, 0, abort_flag, p.status, false);
+        for (int it = issued > NSQ ? issued - NSQ : 0; it < issued; ++it)
+            wait_bounded(&sm.st_full[it % NSQ], (it / NSQ) & 1, abort_flag, p.status, false);
+        __syncwarp();
+    } else if (warp == kBwdMmaWarp) {
+        // --------------------------------------------------------- MMA issue
+        if (n_items > 0) {
+            const bool leader = elect_one();
+            constexpr uint32_t kIdescT = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+            constexpr uint32_t kIdescG = idesc_bf16_f32(128, D, 0, 1);    // dV, dK
+            constexpr uint32_t kTile = Smem::kChunks * Smem::kChunkElems * 2;
+            constexpr uint32_t kChunkBytes = Smem::kChunkElems * 2;
+            const uint64_t k_desc = smem_desc_sw128(smem_u32(&sm.k[0][0]), 16, 1024);
+            const uint64_t v_desc = smem_desc_sw128(smem_u32(&sm.v[0][0]), 16, 1024);
+            const uint64_t q_kdesc = smem_desc_sw128(smem_u32(&sm.q[0][0][0]), 16, 1024);
+            const uint64_t do_kdesc = smem_desc_sw128(smem_u32(&sm.dout[0][0][0]), 16, 1024);
+            const uint64_t q_mdesc = smem_desc_sw128(smem_u32(&sm.q[0][0][0]), kChunkBytes, 1024);
+            const uint64_t do_mdesc =
+                smem_desc_sw128(smem_u32(&sm.dout[0][0][0]), kChunkBytes, 1024);
+            bool ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full, 0, abort_flag, p.status));
+            auto wait_stage = [&](int it) {
+                if (ok)
+                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.st_full[it % NSQ],
+                                                              (it / NSQ) & 1, abort_flag,
+                                                              p.status));
+                tc_fence_after();
+            };
+            // X^T = A X^T for A in {K, V} (keys in lanes), X in {Q, dO} of stage s.
+            auto issue_t = [&](uint64_t a_desc, uint64_t x_desc, int s, uint32_t col,
+                               uint64_t *bar) {
+                const uint64_t xb = x_desc + ((s * kTile) >> 4);
+                if (leader) {
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = ((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4;
+                        mma_ss(tmem + col, a_desc + off, xb + off, kIdescT, ks > 0 ? 1u : 0u);
+                    }
+                    tc_commit(bar);
+                }
+                __syncwarp();
+            };
+            // G += A_tmem Y, A = P^T or dS^T (bf16 in TMEM, keys in lanes, 128
+            // rows along K), Y = dO or Q of stage s read MN-major.
+            auto issue_g = [&](uint32_t a_col, uint64_t y_desc, int s, uint32_t col, bool first) {
+                const uint64_t yb = y_desc + ((s * kTile) >> 4);
+                if (leader) {
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ts(tmem + col, tmem + a_col + ks * 8, yb + ((ks * 16 * 128) >> 4),
+                               kIdescG, (!first || ks > 0) ? 1u : 0u);
+                }
+                __syncwarp();
+            };
+            wait_stage(0);
+            if (ok) {
+                issue_t(k_desc, q_kdesc, 0, kColS, &sm.s_full);
+                issue_t(v_desc, do_kdesc, 0, kColDP, &sm.dp_full);
+            }
+            for (int it = 0; it < n_items && ok; ++it) {
+                const int s = it % NSQ;
+                ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_ready, it & 1, abort_flag,
+                                                          p.status));
+                if (!ok) break;
+                tc_fence_after();
+                issue_g(kColS, do_mdesc, s, kColDV, it == 0);
+                if (it + 1 < n_items) {
+                    wait_stage(it + 1);
+                    if (!ok) break;
+                    issue_t(k_desc, q_kdesc, (it + 1) % NSQ, kColS, &sm.s_full);
+                }
+                ok = __all_sync(0xffffffffu, wait_bounded(&sm.ds_ready, it & 1, abort_flag,
+                                                          p.status));
+                if (!ok) break;
+                tc_fence_after();
+                issue_g(kColDP, q_mdesc, s, kColDK, it == 0);
+                if (leader) tc_commit(&sm.st_empty[s]);
+                __syncwarp();
+                if (it + 1 < n_items) issue_t(v_desc, do_kdesc, (it + 1) % NSQ, kColDP, &sm.dp_full);
+            }
+            if (ok) {
+                if (leader) tc_commit(&sm.final_bar);
+                __syncwarp();
+            } else {
+                if (leader) tc_commit(&sm.drain);
+                __syncwarp();
+                wait_bounded(&sm.drain, 0, abort_flag, p.status, false);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- elementwise
+        const int key = k0 + (warp & 3) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const float c = p.scale_log2;
+        bool ok = true;
+        for (int it = 0; it < n_items; ++it) {
+            const int s = it % NSQ;
+            ok = __all_sync(0xffffffffu, wait_bounded(&sm.s_full, it & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[128];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) tmem_ld32(tmem + lane_base + kColS + ch * 32, sr + ch * 32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) reg_fence32(sr + ch * 32);
+            float *pv = reinterpret_cast<float *>(sr);  // S^T row, then P^T row
+            const bool full = sm.full[s] != 0;
+            const float4 *l4 = reinterpret_cast<const float4 *>(sm.lse2[s]);
+            uint32_t pk[64];
+            if (full) {
+#pragma unroll
+                for (int e = 0; e < 128; e += 4) {
+                    const float4 l = l4[e >> 2];
+                    pv[e + 0] = ex2_mufu(fmaf(pv[e + 0], c, -l.x));
+                    pv[e + 1] = ex2_mufu(fmaf(pv[e + 1], c, -l.y));
+                    pv[e + 2] = ex2_mufu(fmaf(pv[e + 2], c, -l.z));
+                    pv[e + 3] = ex2_mufu(fmaf(pv[e + 3], c, -l.w));
+                    pk[(e >> 1) + 0] = pack_bf16x2(pv[e + 0], pv[e + 1]);
+                    pk[(e >> 1) + 1] = pack_bf16x2(pv[e + 2], pv[e + 3]);
+                }
+            } else {
+                const int4 *lo4 = reinterpret_cast<const int4 *>(sm.rlo[s]);
+                const int4 *hi4 = reinterpret_cast<const int4 *>(sm.rhi[s]);
+#pragma unroll
+                for (int e = 0; e < 128; e += 4) {
+                    const float4 l = l4[e >> 2];
+                    const int4 lo = lo4[e >> 2];
+                    const int4 hi = hi4[e >> 2];
+                    pv[e + 0] = (lo.x <= key && key <= hi.x) ? ex2_mufu(fmaf(pv[e + 0], c, -l.x)) : 0.0f;
+                    pv[e + 1] = (lo.y <= key && key <= hi.y) ? ex2_mufu(fmaf(pv[e + 1], c, -l.y)) : 0.0f;
+                    pv[e + 2] = (lo.z <= key && key <= hi.z) ? ex2_mufu(fmaf(pv[e + 2], c, -l.z)) : 0.0f;
+                    pv[e + 3] = (lo.w <= key && key <= hi.w) ? ex2_mufu(fmaf(pv[e + 3], c, -l.w)) : 0.0f;
+                    pk[(e >> 1) + 0] = pack_bf16x2(pv[e + 0], pv[e + 1]);
+                    pk[(e >> 1) + 1] = pack_bf16x2(pv[e + 2], pv[e + 3]);
+                }
+            }
+            tmem_st32(tmem + lane_base + kColS, pk);
+            tmem_st32(tmem + lane_base + kColS + 32, pk + 32);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.p_ready);
+
+            // dS^T = P^T (dP^T - D) for this key against the block's rows.
+            ok = __all_sync(0xffffffffu, wait_bounded(&sm.dp_full, it & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            const float4 *d4 = reinterpret_cast<const float4 *>(sm.dval[s]);
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + kColDP + ch * 32, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) {
+                    const float4 dd = d4[(ch * 32 + e) >> 2];
+                    const float* pp = pv + ch * 32 + e;
+                    const float g0 = pp[0] * (__uint_as_float(r[e + 0]) - dd.x);
+                    const float g1 = pp[1] * (__uint_as_float(r[e + 1]) - dd.y);
+                    const float g2 = pp[2] * (__uint_as_float(r[e + 2]) - dd.z);
+                    const float g3 = pp[3] * (__uint_as_float(r[e + 3]) - dd.w);
+                    pk[(ch * 32 + e) / 2 + 0] = pack_bf16x2(g0, g1);
+                    pk[(ch * 32 + e) / 2 + 1] = pack_bf16x2(g2, g3);
+                }
+            }
+            tmem_st32(tmem + lane_base + kColDP, pk);
+            tmem_st32(tmem + lane_base + kColDP + 32, pk + 32);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.ds_ready);
+        }
+        // ------------------------------------------------------- epilogue
+        if (ok && n_items > 0) {
+            ok = __all_sync(0xffffffffu, wait_bounded(&sm.final_bar, 0, abort_flag, p.status));
+            tc_fence_after();
+        }
+        if (ok) {
+            const bool key_ok = key < p.Sk;
+            const size_t base = (((size_t)b * p.Sk + key) * p.Hkv + hkv) * (size_t)D;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = which == 0 ? kColDK : kColDV;
+                const float mul = which == 0 ? p.scale : 1.0f;
+                __nv_bfloat16 *dst_row = (which == 0 ? p.dk : p.dv) + base;
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t r[32];
+                    if (n_items > 0) {
+                        tmem_ld32(tmem + lane_base + col + ch * 32, r);
+                        tmem_wait_ld();
+                        reg_fence32(r);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) r[e] = 0u;
+                    }
+                    uint4 out[4];
+                    uint32_t *w = reinterpret_cast<uint32_t *>(out);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul,
+                                           __uint_as_float(r[2 * e + 1]) * mul);
+                    if (key_ok) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(dst_row + ch * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) dst[e] = out[e];
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kBwdMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// --------------------------------------------------------------------- dQ
+
+template <int D, int NS>
+struct DqSmem {
+    static constexpr int kChunks = D / 64;
+    static constexpr int kChunkElems = 128 * 64;
+    __nv_bfloat16 q[kChunks][kChunkElems];
+    __nv_bfloat16 dout[kChunks][kChunkElems];
+    __nv_bfloat16 kv[NS][kChunks][kChunkElems];
+    uint64_t q_full;
+    uint64_t kv_full[NS];
+    uint64_t kv_empty[NS];
+    uint64_t s_full, ds_ready, final_bar, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int range[2];
+};
+
+template <int D, int NS>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+    using Smem = DqSmem<D, NS>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_off = smem_u32(smem_raw);
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (raw_off & 1023u)) & 1023u));
+    const int warp = warp_id();
+    const int lane = lane_id();
+
+    // Heaviest query blocks first (causal load balance), then (batch, head).
+    const int bh_count = p.Hq * p.B;
+    const int qb = p.num_qb - 1 - (int)(blockIdx.x / bh_count);
+    const int bh = (int)(blockIdx.x % bh_count);
+    const int hq = bh % p.Hq;
+    const int b = bh / p.Hq;
+    const int hkv = hq / p.group;
+    const int q0 = qb * 128;
+    constexpr uint32_t kTileBytes = 128 * D * 2;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.ds_ready, 128);
+        mbar_init(&sm.final_bar, 1);
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kBwdLoadWarp) {
+        int lo = 0x7fffffff, hi = -1;
+        for (int t = lane; t < 128; t += 32) {
+            const int row = q0 + t;
+            if (row >= p.Sq) break;
+            const KeyRange r = row_key_range(p, row);
+            if (r.lo <= r.hi) {
+                lo = min(lo, r.lo);
+                hi = max(hi, r.hi);
+            }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        if (lane == 0) {
+            sm.range[0] = hi < 0 ? 1 : lo / 128;
+            sm.range[1] = hi < 0 ? 0 : hi / 128;
+        }
+    }
+    if (warp == kBwdMmaWarp) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort_flag;
+    const int lo_b = sm.range[0], hi_b = sm.range[1];
+    const int n_blocks = hi_b >= lo_b ? hi_b - lo_b + 1 : 0;
+    // TMEM columns: S [0,128) (dS as bf16 pairs over its first 64), dP [128,256), dQ [256,256+D)
+    constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+
+    if (warp == kBwdLoadWarp) {
+        if (lane == 0) {
+            prefetch_tensormap(&p.tm_q);
+            prefetch_tensormap(&p.tm_do);
+            prefetch_tensormap(&p.tm_k);
+            prefetch_tensormap(&p.tm_v);
+            mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
+            for (int c = 0; c < Smem::kChunks; ++c) {
+                tma_load_4d(sm.q[c], &p.tm_q, &sm.q_full, c * 64, q0, hq, b);
+                tma_load_4d(sm.dout[c], &p.tm_do, &sm.q_full, c * 64, q0, hq, b);
+            }
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = 0; t < n_blocks && ok; ++t) {
+                const int key0 = (lo_b + t) * 128;
+                for (int which = 0; which < 2 && ok; ++which, ++it) {
+                    const uint32_t slot = it % NS;
+                    ok = wait_bounded(&sm.kv_empty[slot], ((it / NS) & 1u) ^ 1u, abort_flag,
+                                      p.status);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&sm.kv_full[slot], kTileBytes);
+                    const CUtensorMap *map = which ? &p.tm_v : &p.tm_k;
+                    for (int c = 0; c < Smem::kChunks; ++c)
+                        tma_load_4d(sm.kv[slot][c], map, &sm.kv_full[slot], c * 64, key0, hkv, b);
+                }
+            }
+            wait_bounded(&sm.q_full, 0, abort_flag, p.status, false);
+            const uint32_t first = it > NS ? it - NS : 0;
+            for (uint32_t L = first; L < it; ++L)
+                wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status, false);
+        }
+        __syncwarp();
+    } else if (warp == kBwdMmaWarp) {
+        if (n_blocks > 0) {
+            const bool leader = elect_one();
+            constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t kIdescQ = idesc_bf16_f32(128, D, 0, 1);
+            constexpr uint32_t kTile = Smem::kChunks * Smem::kChunkElems * 2;
+            constexpr uint32_t kChunkBytes = Smem::kChunkElems * 2;
+            const uint64_t q_desc = smem_desc_sw128(smem_u32(&sm.q[0][0]), 16, 1024);
+            const uint64_t do_desc = smem_desc_sw128(smem_u32(&sm.dout[0][0]), 16, 1024);
+            const uint64_t kv_kdesc = smem_desc_sw128(smem_u32(&sm.kv[0][0][0]), 16, 1024);
+            const uint64_t kv_mdesc =
+                smem_desc_sw128(smem_u32(&sm.kv[0][0][0]), kChunkBytes, 1024);
+            bool ok = __all_sync(0xffffffffu, wait_bounded(&sm.q_full, 0, abort_flag, p.status));
+            tc_fence_after();
+            for (int t = 0; t < n_blocks && ok; ++t) {
+                const uint32_t Lk = 2u * t, Lv = 2u * t + 1;
+                ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[Lk % NS], (Lk / NS) & 1u,
+                                                          abort_flag, p.status));
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t kb_k = kv_kdesc + (((Lk % NS) * kTile) >> 4);
+                if (leader) {
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = ((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4;
+                        mma_ss(tmem + kColS, q_desc + off, kb_k + off, kIdescS, ks > 0 ? 1u : 0u);
+                    }
+                }
+                __syncwarp();
+                ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[Lv % NS], (Lv / NS) & 1u,
+                                                          abort_flag, p.status));
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t vb_k = kv_kdesc + (((Lv % NS) * kTile) >> 4);
+                if (leader) {
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = ((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4;
+                        mma_ss(tmem + kColDP, do_desc + off, vb_k + off, kIdescS,
+                               ks > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&sm.s_full);
+                    tc_commit(&sm.kv_empty[Lv % NS]);  // V of this block is consumed
+                }
+                __syncwarp();
+                ok = __all_sync(0xffffffffu, wait_bounded(&sm.ds_ready, (uint32_t)t & 1u,
+                                                          abort_flag, p.status));
+                if (!ok) break;
+                tc_fence_after();
+                const uint64_t kb_m = kv_mdesc + (((Lk % NS) * kTile) >> 4);
+                if (leader) {
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ts(tmem + kColDQ, tmem + kColS + ks * 8, kb_m + ((ks * 16 * 128) >> 4),
+                               kIdescQ, (t > 0 || ks > 0) ? 1u : 0u);
+                    tc_commit(&sm.kv_empty[Lk % NS]);  // K of this block is consumed
+                }
+                __syncwarp();
+            }
+            if (ok) {
+                if (leader) tc_commit(&sm.final_bar);
+                __syncwarp();
+            } else {
+                if (leader) tc_commit(&sm.drain);
+                __syncwarp();
+                wait_bounded(&sm.drain, 0, abort_flag, p.status, false);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- elementwise
+        const int row_in = (warp & 3) * 32 + lane;
+        const int row = q0 + row_in;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const bool row_ok = row < p.Sq;
+        const KeyRange kr = row_ok ? row_key_range(p, row) : KeyRange{1, 0};
+        const size_t ri = ((size_t)b * p.Hq + hq) * p.Sq + (row_ok ? row : 0);
+        const float l2 = row_ok ? __ldg(p.lse + ri) * kLog2e : INFINITY;
+        const float dval = row_ok ? p.dval[ri] : 0.0f;
+        const float c = p.scale_log2;
+        bool ok = true;
+        for (int t = 0; t < n_blocks; ++t) {
+            const int j = lo_b + t;
+            ok = __all_sync(0xffffffffu, wait_bounded(&sm.s_full, (uint32_t)t & 1u, abort_flag,
+                                                      p.status));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[128];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) tmem_ld32(tmem + lane_base + kColS + ch * 32, sr + ch * 32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) reg_fence32(sr + ch * 32);
+            float *pv = reinterpret_cast<float *>(sr);
+            const int key0 = j * 128;
+            const bool masked =
+                __any_sync(0xffffffffu, key0 < kr.lo || key0 + 127 > kr.hi);
+            if (masked) {
+#pragma unroll
+                for (int e = 0; e < 128; ++e) {
+                    const int key = key0 + e;
+                    pv[e] = (key >= kr.lo && key <= kr.hi) ? ex2_mufu(fmaf(pv[e], c, -l2)) : 0.0f;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 128; ++e) pv[e] = ex2_mufu(fmaf(pv[e], c, -l2));
+            }
+            uint32_t pk[64];
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + kColDP + ch * 32, r);
+                tmem_wait_ld();
+                reg_fence32(r);
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float g0 = pv[ch * 32 + e] * (__uint_as_float(r[e]) - dval);
+                    const float g1 = pv[ch * 32 + e + 1] * (__uint_as_float(r[e + 1]) - dval);
+                    pk[(ch * 32 + e) / 2] = pack_bf16x2(g0, g1);
+                }
+            }
+            tmem_st32(tmem + lane_base + kColS, pk);
+            tmem_st32(tmem + lane_base + kColS + 32, pk + 32);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.ds_ready);
+        }
+        if (ok && n_blocks > 0) {
+            ok = __all_sync(0xffffffffu, wait_bounded(&sm.final_bar, 0, abort_flag, p.status));
+            tc_fence_after();
+        }
+        if (ok) {
+            float *dst_row = p.dq + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)D;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t r[32];
+                if (n_blocks > 0) {
+                    tmem_ld32(tmem + lane_base + kColDQ + ch * 32, r);
+                    tmem_wait_ld();
+                    reg_fence32(r);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) r[e] = 0u;
+                }
+                if (row_ok) {
+                    float4 *dst = reinterpret_cast<float4 *>(dst_row + ch * 32);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(r[4 * e]) * p.scale,
+                                             __uint_as_float(r[4 * e + 1]) * p.scale,
+                                             __uint_as_float(r[4 * e + 2]) * p.scale,
+                                             __uint_as_float(r[4 * e + 3]) * p.scale);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kBwdMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace tab

@@ -42,6 +42,7 @@
 // and returns.
 #pragma once
 
+#include "common.cuh"
 #include "exp2_poly.cuh"
 #include "ptx.cuh"
 
@@ -60,8 +61,6 @@ constexpr int kSoftmaxRegs = 216;
 constexpr int kOtherRegs = 72;
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kFwdThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
-constexpr int kStatusTimeout = 5;                   // ATTN_ERR_DEVICE_TIMEOUT
 
 struct FwdParams {
     CUtensorMap tm_q;  // bf16 [B][Sq][Hq][D]: dims (D, Sq, Hq, B), box (64, 128, 1, 1)
@@ -117,52 +116,6 @@ struct FwdSmem {
     int abort_flag;
     int range[2][2];  // per query tile: first and last key block (inclusive)
 };
-
-// Keys [lo, hi] (inclusive) that query `row` may attend to; lo > hi = none.
-struct KeyRange {
-    int lo, hi;
-};
-
-__device__ __forceinline__ KeyRange row_key_range(const FwdParams &p, int row) {
-    long long lo = 0, hi = (long long)p.Sk - 1;
-    const long long diag = (long long)row + p.Sk - p.Sq;
-    if (p.causal) hi = min(hi, diag);
-    if (p.window_left >= 0) lo = max(lo, diag - p.window_left);
-    if (p.window_right >= 0) hi = min(hi, diag + p.window_right);
-    if (p.doc_offsets != nullptr) {
-        const int *off = p.doc_offsets;
-        if (row < __ldg(off) || row >= __ldg(off + p.num_docs)) return {1, 0};
-        int a = 0, c = p.num_docs;  // off[a] <= row < off[c]
-        while (c - a > 1) {
-            const int m = (a + c) >> 1;
-            if (__ldg(off + m) <= row) a = m; else c = m;
-        }
-        lo = max(lo, (long long)__ldg(off + a));
-        hi = min(hi, (long long)__ldg(off + a + 1) - 1);
-    }
-    if (lo > hi) return {1, 0};
-    return {(int)lo, (int)hi};
-}
-
-// Bounded wait.  Returns false when the CTA is aborting (own timeout or
-// another role's); `honor_abort` = false keeps waiting until the timeout only.
-__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
-                                             volatile int *abort_flag, int *status,
-                                             bool honor_abort = true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 15u) == 0u) {
-            if (honor_abort && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-                *abort_flag = 1;
-                atomicCAS(status, 0, kStatusTimeout);
-                return false;
-            }
-        }
-    }
-}
 
 __device__ __forceinline__ float ex2_poly(float x) {
     // x = j + f, j = round(x) via the 1.5 * 2^23 trick, f in [-1/2, 1/2];
