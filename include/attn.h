@@ -139,6 +139,37 @@ ATTN_API attn_status_t attn_bwd(const void *q, const void *k, const void *v, con
                                 const int *doc_offsets, int num_docs, void *workspace,
                                 size_t workspace_bytes, void *stream);
 
+/*
+ * attn_bwd without a workspace argument, for callers that cannot allocate
+ * device memory at the point where they run the backward: a framework
+ * plugin or kernel hook that is handed only its input and output pointers
+ * and has no allocator of its own, or a serving/training loop that must not
+ * call cudaMalloc on its hot path (an allocation can synchronise the device
+ * and stall every stream, and can fail with out-of-memory mid-step).  (The
+ * attention pages have no counterpart of this entry point; it exists for
+ * such callers.)
+ *
+ * Same arguments, contract and results as attn_bwd, minus the workspace.
+ * The D_i scratch lives in one fixed device array inside the library (4 MiB,
+ * held on every GPU that loads the library until the process exits), so:
+ *   - B * Hq * Sq must not exceed 1048576 rows; larger calls return
+ *     ATTN_ERR_UNSUPPORTED before anything is launched;
+ *   - the first call on a device looks up that array's device address (and
+ *     prepares the kernels); make that first call before any stream
+ *     capture on that device;
+ *   - every call on a device shares the array: calls that can run on the GPU
+ *     at the same time (different streams, different host threads) race on
+ *     it and must be ordered by the caller (same stream, or events).  Nothing
+ *     in it needs to start at zero: each call writes every entry it reads.
+ * Nothing is allocated: no cudaMalloc / cudaFree, no library allocator.
+ */
+ATTN_API attn_status_t attn_bwd_noalloc(const void *q, const void *k, const void *v,
+                                        const void *o, const float *lse, const void *dout,
+                                        float *dq, void *dk, void *dv, int B, int Hq, int Hkv,
+                                        int Sq, int Sk, int D, float scale, int causal,
+                                        int window_left, int window_right,
+                                        const int *doc_offsets, int num_docs, void *stream);
+
 /* Synchronises `stream`, then reads and clears the device status word of
  * the current device.  Returns ATTN_OK or ATTN_ERR_DEVICE_TIMEOUT (or
  * ATTN_ERR_CUDA if the synchronisation itself failed). */

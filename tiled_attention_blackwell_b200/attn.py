@@ -26,8 +26,8 @@ ATTN_ERR_DEVICE_TIMEOUT = 5
 ATTN_ERR_CUDA = 6
 
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_default_options", "attn_bwd",
-            "attn_bwd_workspace_size", "attn_get_device_status", "attn_status_string",
-            "attn_last_error_detail", "attn_abi_version")
+            "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_status",
+            "attn_status_string", "attn_last_error_detail", "attn_abi_version")
 
 
 class AttnError(RuntimeError):
@@ -78,6 +78,10 @@ def lib():
             L.attn_bwd.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 6 + \
                 [ctypes.c_float] + [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int,
                                                          ctypes.c_void_p, ctypes.c_size_t,
+                                                         ctypes.c_void_p]
+            L.attn_bwd_noalloc.restype = ctypes.c_int
+            L.attn_bwd_noalloc.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 6 + \
+                [ctypes.c_float] + [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int,
                                                          ctypes.c_void_p]
             _lib = L
     return _lib
@@ -211,6 +215,24 @@ def attention_backward(q, k, v, o, lse, dout, *, scale=None, causal=False, windo
     attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, ws, scale=scale, causal=causal, window=window,
              doc_offsets=doc_offsets, stream=stream)
     return dq, dk, dv
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, *, scale, causal=False, window=None,
+                     doc_offsets=None, stream=None):
+    """attn_bwd for callers that cannot allocate device memory: the library
+    uses its own fixed scratch (B*Hq*Sq <= 1048576 rows) instead of a
+    workspace.  Calls that may run on the GPU at the same time must be
+    ordered by the caller (they share that scratch)."""
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    docs_ptr, nd = (None, 0) if doc_offsets is None else (_ptr(doc_offsets),
+                                                           doc_offsets.numel() - 1)
+    st = lib().attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, D,
+                                float(scale), int(bool(causal)), wl, wr, docs_ptr, nd,
+                                _stream_handle(stream))
+    _check(st, "attn_bwd_noalloc")
 
 
 def device_status(stream=None) -> int:

@@ -230,6 +230,19 @@ long long *g_trace = nullptr;
 int g_trace_ctas = 0;
 #endif
 
+// ------------------------------------------ scratch of attn_bwd_noalloc
+// D_i of up to kNoAllocRows rows for callers that cannot allocate a
+// workspace.  The array exists on every device that loads the library.
+constexpr size_t kNoAllocRows = size_t(1) << 20;  // 4 MiB of fp32
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocRows];
+
+struct NoAllocScratch {
+    std::once_flag once;
+    cudaError_t err = cudaSuccess;
+    void *ptr = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
 }  // namespace
 
 extern "C" {
@@ -381,6 +394,34 @@ attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     return D == 128 ? launch_bwd<128>(p, cs) : launch_bwd<64>(p, cs);
+}
+
+attn_status_t attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,
+                               const float *lse, const void *dout, float *dq, void *dk,
+                               void *dv, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                               float scale, int causal, int window_left, int window_right,
+                               const int *doc_offsets, int num_docs, void *stream) {
+    if (B < 1 || Hq < 1 || Sq < 1)
+        return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Sq must be >= 1");
+    const long long rows = (long long)B * Hq * Sq;
+    if (rows > (long long)kNoAllocRows)
+        return fail(ATTN_ERR_UNSUPPORTED,
+                    "attn_bwd_noalloc: B*Hq*Sq = %lld rows exceeds the built-in scratch of "
+                    "%zu rows; use attn_bwd with a workspace",
+                    rows, kNoAllocRows);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(ATTN_ERR_UNSUPPORTED, "device index %d", dev);
+    // Once per device, with that device current: the host-side name of the
+    // array is not a device address; look the address up.
+    NoAllocScratch &sc = g_noalloc[dev];
+    std::call_once(sc.once, [&]() { sc.err = cudaGetSymbolAddress(&sc.ptr, g_noalloc_scratch); });
+    if (sc.err != cudaSuccess || sc.ptr == nullptr)
+        return fail(ATTN_ERR_CUDA, "scratch address lookup: %s", cudaGetErrorString(sc.err));
+    return attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D, scale, causal,
+                    window_left, window_right, doc_offsets, num_docs, sc.ptr,
+                    kNoAllocRows * sizeof(float), stream);
 }
 
 attn_status_t attn_get_device_status(void *stream) {
