@@ -41,6 +41,7 @@ UNIT = "TFLOP/s"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["tiled_attention_blackwell_b200/csrc/fwd_kernel.cuh",
+                  "tiled_attention_blackwell_b200/csrc/common.cuh",
                   "tiled_attention_blackwell_b200/csrc/ptx.cuh",
                   "tiled_attention_blackwell_b200/csrc/exp2_poly.cuh",
                   "tiled_attention_blackwell_b200/csrc/attn_api.cu"]
@@ -276,6 +277,24 @@ def run_ours(args):
     docs = None if docs_np is None else torch.as_tensor(docs_np, dtype=torch.int32, device=device)
     o = torch.empty_like(dev["q"])
     lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=device)
+    window = None if w.window == (-1, -1) else w.window
+    if w.backward:
+        # Backward workload: O and LSE come from one forward before timing;
+        # a step is one attn_bwd (preprocess, dK/dV and dQ kernels).
+        flops *= 2.5
+        attn.attn_fwd(dev["q"], dev["k"], dev["v"], o, lse, scale=w.scale, causal=w.causal,
+                      window=window, doc_offsets=docs)
+        host.update(o=o.cpu().pin_memory(), lse=lse.cpu().pin_memory(),
+                    dout=inp["dout"].pin_memory())
+        dev.update(o=o, lse=lse, dout=host["dout"].to(device))
+        g_dq = torch.empty(dev["q"].shape, dtype=torch.float32, device=device)
+        g_dk = torch.empty_like(dev["k"])
+        g_dv = torch.empty_like(dev["v"])
+        ws = torch.empty(attn.bwd_workspace_size(w.B, w.Hq, w.Hkv, w.S, w.S, w.D),
+                         dtype=torch.uint8, device=device)
+        outputs = [g_dq, g_dk, g_dv]
+    else:
+        outputs = [o, lse]
     flush = None if cfg["io_bytes"] > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8,
                                                                  device=device)
     opts = None
@@ -289,9 +308,13 @@ def run_ours(args):
     stream = torch.cuda.current_stream(device)
 
     def step():
-        attn.attn_fwd(dev["q"], dev["k"], dev["v"], o, lse, scale=w.scale, causal=w.causal,
-                      window=None if w.window == (-1, -1) else w.window, doc_offsets=docs,
-                      options=opts, stream=stream)
+        if w.backward:
+            attn.attn_bwd(dev["q"], dev["k"], dev["v"], dev["o"], dev["lse"], dev["dout"], g_dq,
+                          g_dk, g_dv, ws, scale=w.scale, causal=w.causal, window=window,
+                          doc_offsets=docs, stream=stream)
+        else:
+            attn.attn_fwd(dev["q"], dev["k"], dev["v"], o, lse, scale=w.scale, causal=w.causal,
+                          window=window, doc_offsets=docs, options=opts, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -324,18 +347,17 @@ def run_ours(args):
     value = flops * args.steps * world / (total_ms_max / 1e3) / 1e12
     launch_avg_ms = float(np.mean(launch_ms))
 
-    # ---- end to end through the C ABI: pinned host inputs in, O and LSE out
-    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    # ---- end to end through the C ABI: pinned host inputs in, results out
+    out_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outputs]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in outputs)
 
     def e2e_step():
         for n in host:
             dev[n].copy_(host[n], non_blocking=True)
         step()
-        o_host.copy_(o, non_blocking=True)
-        lse_host.copy_(lse, non_blocking=True)
+        for hst, dvc in zip(out_host, outputs):
+            hst.copy_(dvc, non_blocking=True)
 
     for _ in range(min(args.warmup, 3)):
         e2e_step()
@@ -354,8 +376,10 @@ def run_ours(args):
     peaks, peak_kind = read_peaks()
     achieved = flops / (launch_avg_ms / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
+    metric = METRIC if not w.backward else \
+        f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()})"
     result = {
-        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "metric": metric, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": cfg,
@@ -367,13 +391,15 @@ def run_ours(args):
                      if peak_kind == "measured" else "fallback 1590 TFLOP/s",
                      "frac_of_sustained": round(achieved / float(
                          peaks.get("bf16_tflops_sustained", peak)), 4),
-                     "flops_per_launch": flops, "launch_ms": round(launch_avg_ms, 4)},
+                     "flops_per_launch": flops, "launch_ms": round(launch_avg_ms, 4),
+                     "kernel": "attn_bwd (preprocess, dK/dV, dQ kernels per step)"
+                     if w.backward else "attn_fwd_kernel"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (3 if w.backward else 1),
         "clocks": sampler.summary(),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not w.backward:
         n_rows = rows_for_seconds(w, inp, 15.0)
         dt, fl, cores = oracle_sample(w, inp, n_rows)
         result["cpu_baseline"] = {

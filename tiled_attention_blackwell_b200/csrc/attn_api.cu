@@ -392,6 +392,10 @@ attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *
     p.num_kb = (int)num_kb;
     p.scale = scale;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+#ifdef ATTN_TRACE
+    p.trace = g_trace;
+    p.trace_ctas = g_trace_ctas;
+#endif
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     return D == 128 ? launch_bwd<128>(p, cs) : launch_bwd<64>(p, cs);
 }

@@ -20,9 +20,11 @@
 //   attn_bwd_dq_kernel          one CTA per (batch, query head, 128-row
 //                               block): S = Q K^T, dP = dO V^T, dS into
 //                               TMEM, dQ += dS K.
-// Warp roles in both main kernels (192 threads): warps 0-3 elementwise
-// (one TMEM lane each), warp 4 MMA issue (warp-uniform, one elected lane),
-// warp 5 TMA producer.  Every wait is bounded as in the forward.
+// Warp roles in both main kernels (320 threads): warps 0-7 elementwise
+// (warps 0-3 take columns [0, 64) of each 128-wide tile, warps 4-7 columns
+// [64, 128); one TMEM lane per thread; the work is purely elementwise, so the
+// halves need no exchange), warp 8 MMA issue (warp-uniform, one elected
+// lane), warp 9 TMA producer.  Every wait is bounded as in the forward.
 #pragma once
 
 #include "common.cuh"
@@ -30,10 +32,26 @@
 
 namespace tab {
 
-constexpr int kBwdThreads = 192;
-constexpr int kBwdMmaWarp = 4;
-constexpr int kBwdLoadWarp = 5;
+constexpr int kBwdThreads = 320;
+constexpr int kBwdMmaWarp = 8;
+constexpr int kBwdLoadWarp = 9;
+
+// TMEM column of the bf16 operand (P, P^T, dS or dS^T) for K-step ks of a
+// 128-wide contraction: each elementwise warpgroup writes its 64 columns'
+// pairs into the first 32 columns of its own half of the score tile, so the
+// two halves never touch each other's cells.
+__device__ __forceinline__ uint32_t half_operand_col(uint32_t base, int ks) {
+    return base + (ks < 4 ? ks * 8 : 64 + (ks - 4) * 8);
+}
 constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x for element e of a 64-wide row half: two pairs in five on the FMA pipe
+// (our cubic, clamped at -125), the rest on MUFU, spread so the two units
+// work side by side.  Used only where no element is masked.
+__device__ __forceinline__ float bwd_ex2(float x, int e) {
+    const int pair = (e >> 1) % 5;
+    return (pair == 1 || pair == 3) ? ex2_poly(x) : ex2_mufu(x);
+}
 
 struct BwdParams {
     CUtensorMap tm_q;   // bf16 [B][Sq][Hq][D], box (64, 128, 1, 1)
@@ -55,7 +73,24 @@ struct BwdParams {
     int num_qb, num_kb;  // 128-row query blocks, 128-key blocks
     float scale;
     float scale_log2;
+    long long *trace;  // clock64 event log (trace builds only), else null
+    int trace_ctas;
 };
+
+// Opt-in event trace of the dK/dV kernel (compile with -DATTN_TRACE), same
+// layout as the forward's: [cta][role][item][event], roles 0 = elementwise
+// warp 0, 1 = TMA producer, 2 = MMA warp.
+#ifdef ATTN_TRACE
+#define BWD_TRACE(role, iter, ev)                                                            \
+    do {                                                                                   \
+        if (p.trace && (int)blockIdx.x < p.trace_ctas && (iter) < 96 && lane == 0)            \
+            p.trace[(((size_t)blockIdx.x * 3 + (role)) * 96 + (iter)) * 8 + (ev)] = clock64(); \
+    } while (0)
+#else
+#define BWD_TRACE(role, iter, ev) \
+    do {                          \
+    } while (0)
+#endif
 
 // --------------------------------------------------------------- preprocess
 
@@ -142,8 +177,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.dp_full, 1);
-        mbar_init(&sm.p_ready, 128);
-        mbar_init(&sm.ds_ready, 128);
+        mbar_init(&sm.p_ready, 256);
+        mbar_init(&sm.ds_ready, 256);
         mbar_init(&sm.final_bar, 1);
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
@@ -209,45 +244,82 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
         __syncwarp();
         bool ok = true;
         int issued = 0;
+        // The per-row data of the next item (LSE, D_i, key interval, whether
+        // the whole item is unmasked) is computed one item ahead, while this
+        // warp would otherwise wait for a free stage; after the wait only the
+        // tile copies and the shared-memory stores remain.
+        float nl[4], nd[4];
+        int nlo[4], nhi[4];
+        bool nfull = true;
+        auto prefetch = [&](int it) {
+            const int g = it / n_qb;
+            const int qb = qb_lo + it % n_qb;
+            const size_t rb = ((size_t)b * p.Hq + hkv * p.group + g) * p.Sq;
+            nfull = true;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int r = qb * 128 + lane + 32 * m;
+                const size_t ri = rb + (r < p.Sq ? r : 0);  // in bounds either way
+                nl[m] = ld_nc_f32(p.lse + ri);
+                nd[m] = ld_nc_f32(p.dval + ri);
+                const KeyRange kr = r < p.Sq ? row_key_range(p, r) : KeyRange{1, 0};
+                nlo[m] = kr.lo;
+                nhi[m] = kr.hi;
+                nfull = nfull && r < p.Sq && kr.lo <= k0 && kr.hi >= k1;
+            }
+            nfull = __all_sync(0xffffffffu, nfull);
+        };
+        if (n_items > 0) prefetch(0);
         for (int it = 0; it < n_items && ok; ++it) {
             const int s = it % NSQ;
             const int g = it / n_qb;
             const int qb = qb_lo + it % n_qb;
             const int hq = hkv * p.group + g;
+            float cl[4], cd[4];
+            int clo[4], chi[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                cl[m] = nl[m];
+                cd[m] = nd[m];
+                clo[m] = nlo[m];
+                chi[m] = nhi[m];
+                if (qb * 128 + lane + 32 * m >= p.Sq) {
+                    cl[m] = INFINITY;
+                    cd[m] = 0.0f;
+                }
+            }
+            const bool full = nfull;
+            if (it + 1 < n_items) prefetch(it + 1);
+            BWD_TRACE(1, it, 0);
             ok = __all_sync(0xffffffffu, wait_bounded(&sm.st_empty[s], ((it / NSQ) & 1) ^ 1,
                                                       abort_flag, p.status));
+            BWD_TRACE(1, it, 1);
             if (!ok) break;
-            // Per-row data of this query block.
-            bool full = true;
+            // The tiles go first: the copy is the long pole.
+            if (lane < 2) {
+                // lane 0 copies the Q tile, lane 1 the dO tile, side by side
+                mbar_expect_tx(&sm.st_full[s], kTileBytes);
+                for (int c = 0; c < Smem::kChunks; ++c) {
+                    if (lane == 0)
+                        tma_load_4d(sm.q[s][c], &p.tm_q, &sm.st_full[s], c * 64, qb * 128, hq, b);
+                    else
+                        tma_load_4d(sm.dout[s][c], &p.tm_do, &sm.st_full[s], c * 64, qb * 128,
+                                    hq, b);
+                }
+            }
+            BWD_TRACE(1, it, 3);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const int idx = lane + 32 * m;
-                const int r = qb * 128 + idx;
-                float l2 = INFINITY, dv = 0.0f;
-                KeyRange kr = {1, 0};
-                if (r < p.Sq) {
-                    const size_t ri = ((size_t)b * p.Hq + hq) * p.Sq + r;
-                    l2 = __ldg(p.lse + ri) * kLog2e;
-                    dv = p.dval[ri];
-                    kr = row_key_range(p, r);
-                }
-                sm.lse2[s][idx] = l2;
-                sm.dval[s][idx] = dv;
-                sm.rlo[s][idx] = kr.lo;
-                sm.rhi[s][idx] = kr.hi;
-                full = full && r < p.Sq && kr.lo <= k0 && kr.hi >= k1;
+                sm.lse2[s][idx] = cl[m] * kLog2e;
+                sm.dval[s][idx] = cd[m];
+                sm.rlo[s][idx] = clo[m];
+                sm.rhi[s][idx] = chi[m];
             }
-            full = __all_sync(0xffffffffu, full);
-            if (lane == 0) {
-                sm.full[s] = full ? 1 : 0;
-                mbar_arrive_expect_tx(&sm.st_full[s], 2 * kTileBytes);
-                for (int c = 0; c < Smem::kChunks; ++c) {
-                    tma_load_4d(sm.q[s][c], &p.tm_q, &sm.st_full[s], c * 64, qb * 128, hq, b);
-                    tma_load_4d(sm.dout[s][c], &p.tm_do, &sm.st_full[s], c * 64, qb * 128, hq, b);
-                }
-            } else {
-                mbar_arrive(&sm.st_full[s]);
-            }
+            if (lane == 0) sm.full[s] = full ? 1 : 0;
+            BWD_TRACE(1, it, 4);
+            mbar_arrive(&sm.st_full[s]);  // each lane publishes its own rows
+            BWD_TRACE(1, it, 2);
             ++issued;
         }
         // Copies still in flight land before the CTA can exit.
@@ -299,8 +371,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
                 if (leader) {
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_ts(tmem + col, tmem + a_col + ks * 8, yb + ((ks * 16 * 128) >> 4),
-                               kIdescG, (!first || ks > 0) ? 1u : 0u);
+                        mma_ts(tmem + col, tmem + half_operand_col(a_col, ks),
+                               yb + ((ks * 16 * 128) >> 4), kIdescG,
+                               (!first || ks > 0) ? 1u : 0u);
                 }
                 __syncwarp();
             };
@@ -311,21 +384,28 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
             }
             for (int it = 0; it < n_items && ok; ++it) {
                 const int s = it % NSQ;
+                BWD_TRACE(2, it, 0);
                 ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_ready, it & 1, abort_flag,
                                                           p.status));
+                BWD_TRACE(2, it, 1);
                 if (!ok) break;
                 tc_fence_after();
                 issue_g(kColS, do_mdesc, s, kColDV, it == 0);
+                BWD_TRACE(2, it, 2);
                 if (it + 1 < n_items) {
                     wait_stage(it + 1);
+                    BWD_TRACE(2, it, 3);
                     if (!ok) break;
                     issue_t(k_desc, q_kdesc, (it + 1) % NSQ, kColS, &sm.s_full);
                 }
+                BWD_TRACE(2, it, 4);
                 ok = __all_sync(0xffffffffu, wait_bounded(&sm.ds_ready, it & 1, abort_flag,
                                                           p.status));
+                BWD_TRACE(2, it, 5);
                 if (!ok) break;
                 tc_fence_after();
                 issue_g(kColDP, q_mdesc, s, kColDK, it == 0);
+                BWD_TRACE(2, it, 6);
                 if (leader) tc_commit(&sm.st_empty[s]);
                 __syncwarp();
                 if (it + 1 < n_items) issue_t(v_desc, do_kdesc, (it + 1) % NSQ, kColDP, &sm.dp_full);
@@ -342,40 +422,45 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
     } else {
         // ---------------------------------------------------- elementwise
         const int key = k0 + (warp & 3) * 32 + lane;
+        const int h = warp >> 2;  // this warpgroup's half of the columns
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t s_col = tmem + lane_base + kColS + h * 64;
+        const uint32_t dp_col = tmem + lane_base + kColDP + h * 64;
         const float c = p.scale_log2;
         bool ok = true;
         for (int it = 0; it < n_items; ++it) {
             const int s = it % NSQ;
+            if (warp == 0) BWD_TRACE(0, it, 0);
             ok = __all_sync(0xffffffffu, wait_bounded(&sm.s_full, it & 1, abort_flag, p.status));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[128];
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) tmem_ld32(tmem + lane_base + kColS + ch * 32, sr + ch * 32);
+            if (warp == 0) BWD_TRACE(0, it, 1);
+            uint32_t sr[64];
+            tmem_ld32(s_col, sr);
+            tmem_ld32(s_col + 32, sr + 32);
             tmem_wait_ld();
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) reg_fence32(sr + ch * 32);
-            float *pv = reinterpret_cast<float *>(sr);  // S^T row, then P^T row
+            reg_fence32(sr);
+            reg_fence32(sr + 32);
+            float *pv = reinterpret_cast<float *>(sr);  // S^T half row, then P^T
             const bool full = sm.full[s] != 0;
-            const float4 *l4 = reinterpret_cast<const float4 *>(sm.lse2[s]);
-            uint32_t pk[64];
+            const float4 *l4 = reinterpret_cast<const float4 *>(sm.lse2[s] + h * 64);
+            uint32_t pk[32];
             if (full) {
 #pragma unroll
-                for (int e = 0; e < 128; e += 4) {
+                for (int e = 0; e < 64; e += 4) {
                     const float4 l = l4[e >> 2];
-                    pv[e + 0] = ex2_mufu(fmaf(pv[e + 0], c, -l.x));
-                    pv[e + 1] = ex2_mufu(fmaf(pv[e + 1], c, -l.y));
-                    pv[e + 2] = ex2_mufu(fmaf(pv[e + 2], c, -l.z));
-                    pv[e + 3] = ex2_mufu(fmaf(pv[e + 3], c, -l.w));
+                    pv[e + 0] = bwd_ex2(fmaf(pv[e + 0], c, -l.x), e + 0);
+                    pv[e + 1] = bwd_ex2(fmaf(pv[e + 1], c, -l.y), e + 1);
+                    pv[e + 2] = bwd_ex2(fmaf(pv[e + 2], c, -l.z), e + 2);
+                    pv[e + 3] = bwd_ex2(fmaf(pv[e + 3], c, -l.w), e + 3);
                     pk[(e >> 1) + 0] = pack_bf16x2(pv[e + 0], pv[e + 1]);
                     pk[(e >> 1) + 1] = pack_bf16x2(pv[e + 2], pv[e + 3]);
                 }
             } else {
-                const int4 *lo4 = reinterpret_cast<const int4 *>(sm.rlo[s]);
-                const int4 *hi4 = reinterpret_cast<const int4 *>(sm.rhi[s]);
+                const int4 *lo4 = reinterpret_cast<const int4 *>(sm.rlo[s] + h * 64);
+                const int4 *hi4 = reinterpret_cast<const int4 *>(sm.rhi[s] + h * 64);
 #pragma unroll
-                for (int e = 0; e < 128; e += 4) {
+                for (int e = 0; e < 64; e += 4) {
                     const float4 l = l4[e >> 2];
                     const int4 lo = lo4[e >> 2];
                     const int4 hi = hi4[e >> 2];
@@ -387,40 +472,39 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
                     pk[(e >> 1) + 1] = pack_bf16x2(pv[e + 2], pv[e + 3]);
                 }
             }
-            tmem_st32(tmem + lane_base + kColS, pk);
-            tmem_st32(tmem + lane_base + kColS + 32, pk + 32);
+            tmem_st32(s_col, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_ready);
+            if (warp == 0) BWD_TRACE(0, it, 2);
 
-            // dS^T = P^T (dP^T - D) for this key against the block's rows.
+            // dS^T = P^T (dP^T - D) for this key against this half's rows.
             ok = __all_sync(0xffffffffu, wait_bounded(&sm.dp_full, it & 1, abort_flag, p.status));
             if (!ok) break;
             tc_fence_after();
-            const float4 *d4 = reinterpret_cast<const float4 *>(sm.dval[s]);
+            if (warp == 0) BWD_TRACE(0, it, 3);
+            uint32_t dr[64];
+            tmem_ld32(dp_col, dr);
+            tmem_ld32(dp_col + 32, dr + 32);
+            tmem_wait_ld();
+            reg_fence32(dr);
+            reg_fence32(dr + 32);
+            const float4 *d4 = reinterpret_cast<const float4 *>(sm.dval[s] + h * 64);
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + kColDP + ch * 32, r);
-                tmem_wait_ld();
-                reg_fence32(r);
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                    const float4 dd = d4[(ch * 32 + e) >> 2];
-                    const float* pp = pv + ch * 32 + e;
-                    const float g0 = pp[0] * (__uint_as_float(r[e + 0]) - dd.x);
-                    const float g1 = pp[1] * (__uint_as_float(r[e + 1]) - dd.y);
-                    const float g2 = pp[2] * (__uint_as_float(r[e + 2]) - dd.z);
-                    const float g3 = pp[3] * (__uint_as_float(r[e + 3]) - dd.w);
-                    pk[(ch * 32 + e) / 2 + 0] = pack_bf16x2(g0, g1);
-                    pk[(ch * 32 + e) / 2 + 1] = pack_bf16x2(g2, g3);
-                }
+            for (int e = 0; e < 64; e += 4) {
+                const float4 dd = d4[e >> 2];
+                const float g0 = pv[e + 0] * (__uint_as_float(dr[e + 0]) - dd.x);
+                const float g1 = pv[e + 1] * (__uint_as_float(dr[e + 1]) - dd.y);
+                const float g2 = pv[e + 2] * (__uint_as_float(dr[e + 2]) - dd.z);
+                const float g3 = pv[e + 3] * (__uint_as_float(dr[e + 3]) - dd.w);
+                pk[(e >> 1) + 0] = pack_bf16x2(g0, g1);
+                pk[(e >> 1) + 1] = pack_bf16x2(g2, g3);
             }
-            tmem_st32(tmem + lane_base + kColDP, pk);
-            tmem_st32(tmem + lane_base + kColDP + 32, pk + 32);
+            tmem_st32(dp_col, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.ds_ready);
+            if (warp == 0) BWD_TRACE(0, it, 4);
         }
         // ------------------------------------------------------- epilogue
         if (ok && n_items > 0) {
@@ -429,14 +513,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
         }
         if (ok) {
             const bool key_ok = key < p.Sk;
-            const size_t base = (((size_t)b * p.Sk + key) * p.Hkv + hkv) * (size_t)D;
+            const size_t base = (((size_t)b * p.Sk + key) * p.Hkv + hkv) * (size_t)D + h * (D / 2);
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                const uint32_t col = which == 0 ? kColDK : kColDV;
+                const uint32_t col = (which == 0 ? kColDK : kColDV) + h * (D / 2);
                 const float mul = which == 0 ? p.scale : 1.0f;
                 __nv_bfloat16 *dst_row = (which == 0 ? p.dk : p.dv) + base;
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < D / 64; ++ch) {
                     uint32_t r[32];
                     if (n_items > 0) {
                         tmem_ld32(tmem + lane_base + col + ch * 32, r);
@@ -482,7 +566,7 @@ struct DqSmem {
     uint64_t q_full;
     uint64_t kv_full[NS];
     uint64_t kv_empty[NS];
-    uint64_t s_full, ds_ready, final_bar, drain;
+    uint64_t s_full, dp_free, ds_ready, final_bar, drain;
     uint32_t tmem_base;
     int abort_flag;
     int range[2];
@@ -515,7 +599,8 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
             mbar_init(&sm.kv_empty[s], 1);
         }
         mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.ds_ready, 128);
+        mbar_init(&sm.dp_free, 256);
+        mbar_init(&sm.ds_ready, 256);
         mbar_init(&sm.final_bar, 1);
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
@@ -553,8 +638,11 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
     volatile int *abort_flag = &sm.abort_flag;
     const int lo_b = sm.range[0], hi_b = sm.range[1];
     const int n_blocks = hi_b >= lo_b ? hi_b - lo_b + 1 : 0;
-    // TMEM columns: S [0,128) (dS as bf16 pairs over its first 64), dP [128,256), dQ [256,256+D)
-    constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+    // TMEM columns: S of even blocks [0,128), dP [128,256), dQ [256,256+D), S of
+    // odd blocks [384,512).  dS (bf16 pairs) goes over its block's S.  The
+    // second S buffer lets S and dP of the next block run on the tensor
+    // cores while this block's dS is computed.
+    constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColS1 = 384;
 
     if (warp == kBwdLoadWarp) {
         if (lane == 0) {
@@ -602,25 +690,33 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                 smem_desc_sw128(smem_u32(&sm.kv[0][0][0]), kChunkBytes, 1024);
             bool ok = __all_sync(0xffffffffu, wait_bounded(&sm.q_full, 0, abort_flag, p.status));
             tc_fence_after();
-            for (int t = 0; t < n_blocks && ok; ++t) {
-                const uint32_t Lk = 2u * t, Lv = 2u * t + 1;
-                ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[Lk % NS], (Lk / NS) & 1u,
-                                                          abort_flag, p.status));
-                if (!ok) break;
+            auto wait_slot = [&](uint32_t L) {
+                if (ok)
+                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u,
+                                                              abort_flag, p.status));
                 tc_fence_after();
+            };
+            // S of block t into its buffer (needs K), then dP (needs V); one
+            // commit signals both.
+            auto issue_s = [&](int t) {
+                const uint32_t Lk = 2u * t;
+                wait_slot(Lk);
+                if (!ok) return;
                 const uint64_t kb_k = kv_kdesc + (((Lk % NS) * kTile) >> 4);
+                const uint32_t col = (t & 1) ? kColS1 : kColS;
                 if (leader) {
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t off = ((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4;
-                        mma_ss(tmem + kColS, q_desc + off, kb_k + off, kIdescS, ks > 0 ? 1u : 0u);
+                        mma_ss(tmem + col, q_desc + off, kb_k + off, kIdescS, ks > 0 ? 1u : 0u);
                     }
                 }
                 __syncwarp();
-                ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[Lv % NS], (Lv / NS) & 1u,
-                                                          abort_flag, p.status));
-                if (!ok) break;
-                tc_fence_after();
+            };
+            auto issue_dp = [&](int t) {
+                const uint32_t Lv = 2u * t + 1;
+                wait_slot(Lv);
+                if (!ok) return;
                 const uint64_t vb_k = kv_kdesc + (((Lv % NS) * kTile) >> 4);
                 if (leader) {
 #pragma unroll
@@ -633,16 +729,33 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                     tc_commit(&sm.kv_empty[Lv % NS]);  // V of this block is consumed
                 }
                 __syncwarp();
+            };
+            issue_s(0);
+            issue_dp(0);
+            for (int t = 0; t < n_blocks && ok; ++t) {
+                if (t + 1 < n_blocks) {
+                    issue_s(t + 1);  // other S buffer: its last reader (dQ of t-1) is queued
+                    if (!ok) break;
+                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.dp_free, (uint32_t)t & 1u,
+                                                              abort_flag, p.status));
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_dp(t + 1);
+                    if (!ok) break;
+                }
                 ok = __all_sync(0xffffffffu, wait_bounded(&sm.ds_ready, (uint32_t)t & 1u,
                                                           abort_flag, p.status));
                 if (!ok) break;
                 tc_fence_after();
+                const uint32_t Lk = 2u * t;
                 const uint64_t kb_m = kv_mdesc + (((Lk % NS) * kTile) >> 4);
+                const uint32_t col = (t & 1) ? kColS1 : kColS;
                 if (leader) {
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_ts(tmem + kColDQ, tmem + kColS + ks * 8, kb_m + ((ks * 16 * 128) >> 4),
-                               kIdescQ, (t > 0 || ks > 0) ? 1u : 0u);
+                        mma_ts(tmem + kColDQ, tmem + half_operand_col(col, ks),
+                               kb_m + ((ks * 16 * 128) >> 4), kIdescQ,
+                               (t > 0 || ks > 0) ? 1u : 0u);
                     tc_commit(&sm.kv_empty[Lk % NS]);  // K of this block is consumed
                 }
                 __syncwarp();
@@ -660,7 +773,9 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
         // ---------------------------------------------------- elementwise
         const int row_in = (warp & 3) * 32 + lane;
         const int row = q0 + row_in;
+        const int h = warp >> 2;  // this warpgroup's half of the columns
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t dp_col = tmem + lane_base + kColDP + h * 64;
         const bool row_ok = row < p.Sq;
         const KeyRange kr = row_ok ? row_key_range(p, row) : KeyRange{1, 0};
         const size_t ri = ((size_t)b * p.Hq + hq) * p.Sq + (row_ok ? row : 0);
@@ -674,42 +789,40 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                                                       p.status));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sr[128];
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) tmem_ld32(tmem + lane_base + kColS + ch * 32, sr + ch * 32);
+            const uint32_t s_col = tmem + lane_base + ((t & 1) ? kColS1 : kColS) + h * 64;
+            uint32_t sr[64], dr[64];
+            tmem_ld32(s_col, sr);
+            tmem_ld32(s_col + 32, sr + 32);
+            tmem_ld32(dp_col, dr);
+            tmem_ld32(dp_col + 32, dr + 32);
             tmem_wait_ld();
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) reg_fence32(sr + ch * 32);
+            reg_fence32(sr);
+            reg_fence32(sr + 32);
+            reg_fence32(dr);
+            reg_fence32(dr + 32);
+            tc_fence_before();
+            mbar_arrive(&sm.dp_free);  // dP of the next block may overwrite it now
             float *pv = reinterpret_cast<float *>(sr);
-            const int key0 = j * 128;
-            const bool masked =
-                __any_sync(0xffffffffu, key0 < kr.lo || key0 + 127 > kr.hi);
+            const int key0 = j * 128 + h * 64;
+            const bool masked = __any_sync(0xffffffffu, key0 < kr.lo || key0 + 63 > kr.hi);
             if (masked) {
 #pragma unroll
-                for (int e = 0; e < 128; ++e) {
+                for (int e = 0; e < 64; ++e) {
                     const int key = key0 + e;
                     pv[e] = (key >= kr.lo && key <= kr.hi) ? ex2_mufu(fmaf(pv[e], c, -l2)) : 0.0f;
                 }
             } else {
 #pragma unroll
-                for (int e = 0; e < 128; ++e) pv[e] = ex2_mufu(fmaf(pv[e], c, -l2));
+                for (int e = 0; e < 64; ++e) pv[e] = bwd_ex2(fmaf(pv[e], c, -l2), e);
             }
-            uint32_t pk[64];
+            uint32_t pk[32];
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t r[32];
-                tmem_ld32(tmem + lane_base + kColDP + ch * 32, r);
-                tmem_wait_ld();
-                reg_fence32(r);
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float g0 = pv[ch * 32 + e] * (__uint_as_float(r[e]) - dval);
-                    const float g1 = pv[ch * 32 + e + 1] * (__uint_as_float(r[e + 1]) - dval);
-                    pk[(ch * 32 + e) / 2] = pack_bf16x2(g0, g1);
-                }
+            for (int e = 0; e < 64; e += 2) {
+                const float g0 = pv[e] * (__uint_as_float(dr[e]) - dval);
+                const float g1 = pv[e + 1] * (__uint_as_float(dr[e + 1]) - dval);
+                pk[e / 2] = pack_bf16x2(g0, g1);
             }
-            tmem_st32(tmem + lane_base + kColS, pk);
-            tmem_st32(tmem + lane_base + kColS + 32, pk + 32);
+            tmem_st32(s_col, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.ds_ready);
@@ -719,12 +832,12 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
             tc_fence_after();
         }
         if (ok) {
-            float *dst_row = p.dq + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)D;
+            float *dst_row = p.dq + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)D + h * (D / 2);
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
+            for (int ch = 0; ch < D / 64; ++ch) {
                 uint32_t r[32];
                 if (n_blocks > 0) {
-                    tmem_ld32(tmem + lane_base + kColDQ + ch * 32, r);
+                    tmem_ld32(tmem + lane_base + kColDQ + h * (D / 2) + ch * 32, r);
                     tmem_wait_ld();
                     reg_fence32(r);
                 } else {

@@ -2,6 +2,7 @@
 // interval every supported mask reduces to, and bounded mbarrier waits.
 #pragma once
 
+#include "exp2_poly.cuh"
 #include "ptx.cuh"
 
 namespace tab {
@@ -58,6 +59,37 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
             }
         }
     }
+}
+
+// Software 2^x for the FMA pipe ("La ventaja técnica", ainvest.com page:
+// part of the exponentials as a cubic on the CUDA cores): our minimax cubic
+// (exp2_poly.cuh, fitted by fit_exp2.py) with 2^round(x) applied through the
+// exponent field.
+__device__ __forceinline__ float ex2_poly(float x) {
+    // x = j + f, j = round(x) via the 1.5 * 2^23 trick, f in [-1/2, 1/2];
+    // 2^x = p(f) * 2^j with 2^j applied through the exponent field.
+    x = fmaxf(x, -125.0f);
+    const float magic = 12582912.0f;
+    const float t = x + magic;
+    const float f = x - (t - magic);
+    const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// Two lanes at once with packed f32x2 arithmetic; same steps as ex2_poly.
+__device__ __forceinline__ void ex2_poly2(float &y0, float &y1, float x0, float x1) {
+    x0 = fmaxf(x0, -125.0f);
+    x1 = fmaxf(x1, -125.0f);
+    const float magic = 12582912.0f;
+    float t0, t1, j0, j1, f0, f1, p0, p1;
+    add2(t0, t1, x0, x1, magic, magic);
+    add2(j0, j1, t0, t1, -magic, -magic);
+    add2(f0, f1, x0, x1, -j0, -j1);
+    fma2(p0, p1, kExp2C3, kExp2C3, f0, f1, kExp2C2, kExp2C2);
+    fma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
+    fma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 }  // namespace tab

@@ -117,33 +117,6 @@ struct FwdSmem {
     int range[2][2];  // per query tile: first and last key block (inclusive)
 };
 
-__device__ __forceinline__ float ex2_poly(float x) {
-    // x = j + f, j = round(x) via the 1.5 * 2^23 trick, f in [-1/2, 1/2];
-    // 2^x = p(f) * 2^j with 2^j applied through the exponent field.
-    x = fmaxf(x, -125.0f);
-    const float magic = 12582912.0f;
-    const float t = x + magic;
-    const float f = x - (t - magic);
-    const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
-// Two lanes at once with packed f32x2 arithmetic; same steps as ex2_poly.
-__device__ __forceinline__ void ex2_poly2(float &y0, float &y1, float x0, float x1) {
-    x0 = fmaxf(x0, -125.0f);
-    x1 = fmaxf(x1, -125.0f);
-    const float magic = 12582912.0f;
-    float t0, t1, j0, j1, f0, f1, p0, p1;
-    add2(t0, t1, x0, x1, magic, magic);
-    add2(j0, j1, t0, t1, -magic, -magic);
-    add2(f0, f1, x0, x1, -j0, -j1);
-    fma2(p0, p1, kExp2C3, kExp2C3, f0, f1, kExp2C2, kExp2C2);
-    fma2(p0, p1, p0, p1, f0, f1, kExp2C1, kExp2C1);
-    fma2(p0, p1, p0, p1, f0, f1, kExp2C0, kExp2C0);
-    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // Column pairs that use the polynomial in EXP_MODE 1: one pair in eight,
 // spread through the row so MUFU and FMA work interleave.  (Measured on
 // B200 for the causal S=8192 forward: 1/8 of pairs is the fastest split; a
