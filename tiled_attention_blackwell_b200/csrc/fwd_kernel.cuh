@@ -74,6 +74,7 @@ struct FwdParams {
     int B, Hq, Hkv, Sq, Sk, group;
     int causal, window_left, window_right;
     int num_qblocks;
+    int head_group;  // (batch, head) pairs scheduled together (L2 reuse of K/V)
     float scale_log2;
     float rescale_threshold;
     long long *trace;  // clock64 event log (trace builds only), else null
@@ -165,11 +166,27 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
     const int warp = warp_id();
     const int lane = lane_id();
 
-    // Work item: heaviest query blocks first across all heads (causal load
-    // balance), then (batch, head).
+    // Work item.  (batch, head) pairs are taken in groups of head_group;
+    // within a group the heaviest query blocks come first (causal load
+    // balance) and consecutive CTAs cycle through the group's heads, so the
+    // CTAs resident at any time share the K/V of a few heads in L2.
     const int bh_count = p.Hq * p.B;
-    const int qb = p.num_qblocks - 1 - (int)(blockIdx.x / bh_count);
-    const int bh = (int)(blockIdx.x % bh_count);
+    const int G = p.head_group;
+    const int nq = p.num_qblocks;
+    const int full_groups = bh_count / G;
+    const int lin = (int)blockIdx.x;
+    int grp, r, ge;
+    if (lin < full_groups * G * nq) {
+        grp = lin / (G * nq);
+        r = lin % (G * nq);
+        ge = G;
+    } else {
+        grp = full_groups;
+        r = lin - full_groups * G * nq;
+        ge = bh_count - full_groups * G;
+    }
+    const int qb = nq - 1 - r / ge;
+    const int bh = grp * G + r % ge;
     const int hq = bh % p.Hq;
     const int b = bh / p.Hq;
     const int hkv = hq / p.group;
