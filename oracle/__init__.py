@@ -45,7 +45,7 @@ def _load():
             build()
             lib = ctypes.CDLL(_LIB_PATH)
             dims = [ctypes.c_int] * 6 + [ctypes.c_double] + [ctypes.c_int] * 3 + \
-                   [ctypes.c_void_p, ctypes.c_int]
+                   [ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_void_p]
             for name in ("oracle_attn_fwd_bf16", "oracle_attn_fwd_f64"):
                 fn = getattr(lib, name)
                 fn.restype = ctypes.c_int
@@ -95,6 +95,15 @@ def _mask_args(causal, window, doc_offsets):
     return int(bool(causal)), wl, wr, offs, int(offs.size - 1)
 
 
+def _mods(softcap, alibi_slopes, Hq):
+    if alibi_slopes is None:
+        return float(softcap or 0.0), None
+    sl = np.ascontiguousarray(np.asarray(alibi_slopes, dtype=np.float64).reshape(-1))
+    if sl.size != Hq:
+        raise ValueError("alibi_slopes must have one entry per query head")
+    return float(softcap or 0.0), sl
+
+
 def _shapes(q, k):
     B, Sq, Hq, D = q.shape
     Bk, Sk, Hkv, Dk = k.shape
@@ -104,7 +113,7 @@ def _shapes(q, k):
 
 
 def attn_fwd(q, k, v, *, scale, causal=False, window=None, doc_offsets=None,
-             rows=None):
+             rows=None, softcap=0.0, alibi_slopes=None):
     """Exact attention forward in fp64.
 
     q: [B,Sq,Hq,D], k/v: [B,Sk,Hkv,D] (bf16 torch tensors or float64 arrays).
@@ -118,6 +127,7 @@ def attn_fwd(q, k, v, *, scale, causal=False, window=None, doc_offsets=None,
         raise TypeError("q, k, v must all be bf16 or all float64")
     B, Hq, Hkv, Sq, Sk, D = _shapes(qa, ka)
     causal_i, wl, wr, offs, nd = _mask_args(causal, window, doc_offsets)
+    cap, slopes = _mods(softcap, alibi_slopes, Hq)
     if rows is None:
         o = np.zeros((B, Sq, Hq, D), dtype=np.float64)
         lse = np.zeros((B, Hq, Sq), dtype=np.float64)
@@ -129,13 +139,14 @@ def attn_fwd(q, k, v, *, scale, causal=False, window=None, doc_offsets=None,
         lse = np.zeros((n,), dtype=np.float64)
     fn = lib.oracle_attn_fwd_bf16 if qb else lib.oracle_attn_fwd_f64
     rc = fn(_ptr(qa), _ptr(ka), _ptr(va), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
-            float(scale), causal_i, wl, wr, _ptr(offs), nd, _ptr(rows_a), n)
+            float(scale), causal_i, wl, wr, _ptr(offs), nd, cap, _ptr(slopes), _ptr(rows_a), n)
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd failed with code {rc}")
     return o, lse
 
 
-def attn_bwd(q, k, v, dout, *, scale, causal=False, window=None, doc_offsets=None):
+def attn_bwd(q, k, v, dout, *, scale, causal=False, window=None, doc_offsets=None,
+             softcap=0.0, alibi_slopes=None):
     """Exact attention backward of L = sum(O * dO) in fp64.
 
     Returns (dQ, dK, dV, O, LSE) as float64 numpy arrays; dK/dV are summed
@@ -148,6 +159,7 @@ def attn_bwd(q, k, v, dout, *, scale, causal=False, window=None, doc_offsets=Non
     (qa, bf), (ka, _), (va, _), (da, _) = ins
     B, Hq, Hkv, Sq, Sk, D = _shapes(qa, ka)
     causal_i, wl, wr, offs, nd = _mask_args(causal, window, doc_offsets)
+    cap, slopes = _mods(softcap, alibi_slopes, Hq)
     dq = np.zeros((B, Sq, Hq, D))
     dk = np.zeros((B, Sk, Hkv, D))
     dv = np.zeros((B, Sk, Hkv, D))
@@ -156,7 +168,7 @@ def attn_bwd(q, k, v, dout, *, scale, causal=False, window=None, doc_offsets=Non
     fn = lib.oracle_attn_bwd_bf16 if bf else lib.oracle_attn_bwd_f64
     rc = fn(_ptr(qa), _ptr(ka), _ptr(va), _ptr(da), _ptr(dq), _ptr(dk), _ptr(dv),
             _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, float(scale), causal_i, wl, wr,
-            _ptr(offs), nd)
+            _ptr(offs), nd, cap, _ptr(slopes))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd failed with code {rc}")
     return dq, dk, dv, o, lse

@@ -28,7 +28,13 @@
  *     offsets[d] <= t < offsets[d+1]; query i may see key j only if both lie
  *     in the same document.  It combines (AND) with causal and window;
  *   - grouped heads: query head hq reads key/value head hq / (Hq / Hkv);
- *   - a row with no allowed key has O = 0 and LSE = -inf.
+ *   - a row with no allowed key has O = 0 and LSE = -inf;
+ *   - score modifiers ("El FlexAttention de PyTorch con FlashAttention-4",
+ *     intro: soft-capping and ALiBi), applied in this order to the scaled
+ *     score s = scale * <q_i, k_j>: soft-capping s <- c * tanh(s / c) for a
+ *     cap c > 0; ALiBi s <- s - slope_hq * |i + (Sk - Sq) - j| (a linear
+ *     distance penalty per query head, measured from the bottom-right
+ *     aligned diagonal); then the mask.
  *
  * Parity pins (tests, CPU only): closed forms (equal logits -> mean of V,
  * one dominant logit -> that V row, constant V -> rows of P sum to one,
@@ -58,6 +64,8 @@ typedef struct {
     int causal, window_left, window_right;
     const int *doc_offsets; /* host int32[num_docs + 1] or NULL */
     int num_docs;
+    double softcap;             /* > 0: scores pass through softcap * tanh(s / softcap) */
+    const double *alibi_slopes; /* host double[Hq] or NULL */
 } oracle_shape_t;
 
 /* ------------------------------------------------------------------ input */
@@ -122,7 +130,27 @@ static int kv_head_of(const oracle_shape_t *s, int hq) {
  * Work buffers: s (Sk), qi/kj (D).  kd/vd hold this head's K and V rows
  * already converted to double ([Sk][D]).
  */
-static void forward_row(const oracle_shape_t *s, const double *qi,
+/* The score of (i, j) from the raw dot product: scale, soft-cap, ALiBi. */
+static double modified_score(const oracle_shape_t *s, int hq, long i, long j, double dot) {
+    double x = s->scale * dot;
+    if (s->softcap > 0.0) x = s->softcap * tanh(x / s->softcap);
+    if (s->alibi_slopes) {
+        const double dist = fabs((double)(i + (long)(s->Sk - s->Sq) - j));
+        x -= s->alibi_slopes[hq] * dist;
+    }
+    return x;
+}
+
+/* d(score)/d(dot): the chain rule through the soft-cap (ALiBi is constant). */
+static double score_grad(const oracle_shape_t *s, double dot) {
+    if (s->softcap > 0.0) {
+        const double t = tanh(s->scale * dot / s->softcap);
+        return s->scale * (1.0 - t * t);
+    }
+    return s->scale;
+}
+
+static void forward_row(const oracle_shape_t *s, int hq, const double *qi,
                         const double *kd, const double *vd, long i,
                         double *srow, unsigned char *allow,
                         double *o_out, double *lse_out) {
@@ -135,7 +163,7 @@ static void forward_row(const oracle_shape_t *s, const double *qi,
         const double *kj = kd + (size_t)j * D;
         double dot = 0.0;
         for (int d = 0; d < D; ++d) dot += qi[d] * kj[d];
-        srow[j] = s->scale * dot;
+        srow[j] = modified_score(s, hq, i, j, dot);
         if (srow[j] > M) M = srow[j];
         ++n_allowed;
     }
@@ -229,7 +257,7 @@ static int attn_fwd_core(const oracle_shape_t *s, const void *q, const void *k,
                             lse_dst = lse + ((size_t)b * s->Hq + hq) * s->Sq + i;
                         }
                         load_vec(q, in_bf16, q_index(s, b, i, hq), D, qi);
-                        forward_row(s, qi, kd, vd, i, srow, allow, o_dst, lse_dst);
+                        forward_row(s, hq, qi, kd, vd, i, srow, allow, o_dst, lse_dst);
                     }
                 }
                 free(srow);
@@ -252,8 +280,10 @@ static int attn_fwd_core(const oracle_shape_t *s, const void *q, const void *k,
  *   dV_j += sum_i P_ij dO_i
  *   dP_ij = <dO_i, v_j>
  *   dS_ij = P_ij (dP_ij - D_i)
- *   dQ_i  = scale * sum_j dS_ij k_j
- *   dK_j += scale * sum_i dS_ij q_i
+ *   dQ_i  = sum_j dS_ij s'_ij k_j
+ *   dK_j += sum_i dS_ij s'_ij q_i
+ * where s'_ij is the derivative of the score w.r.t. <q_i, k_j> (scale, times
+ * 1 - tanh^2 under a soft-cap; ALiBi adds a constant).
  * dK and dV sum over the Hq/Hkv query heads of the group.  ("Hardware-Aware
  * FP4 FlashAttention-4", section "Causal Backward Cuantizado": the backward
  * reconstructs the probabilities from the saved LSE.)
@@ -293,7 +323,7 @@ static int attn_bwd_core(const oracle_shape_t *s, const void *q, const void *k,
                         double lse;
                         load_vec(q, in_bf16, q_index(s, b, i, hq), D, qi);
                         load_vec(dout, in_bf16, q_index(s, b, i, hq), D, doi);
-                        forward_row(s, qi, kd, vd, i, srow, allow, oi, &lse);
+                        forward_row(s, hq, qi, kd, vd, i, srow, allow, oi, &lse);
                         if (o_opt)
                             memcpy(o_opt + q_index(s, b, i, hq), oi, (size_t)D * sizeof(double));
                         if (lse_opt) lse_opt[((size_t)b * s->Hq + hq) * Sq + i] = lse;
@@ -309,12 +339,15 @@ static int attn_bwd_core(const oracle_shape_t *s, const void *q, const void *k,
                             double dp = 0.0;
                             for (int d = 0; d < D; ++d) dp += doi[d] * vj[d];
                             const double ds = p * (dp - Di);
+                            double dot = 0.0;
+                            for (int d = 0; d < D; ++d) dot += qi[d] * kj[d];
+                            const double g = ds * score_grad(s, dot);  /* dL/d(q_i . k_j) */
                             double *dkj = dk + kv_index(s, b, j, hkv);
                             double *dvj = dv + kv_index(s, b, j, hkv);
                             for (int d = 0; d < D; ++d) {
                                 dvj[d] += p * doi[d];
-                                dqi[d] += s->scale * ds * kj[d];
-                                dkj[d] += s->scale * ds * qi[d];
+                                dqi[d] += g * kj[d];
+                                dkj[d] += g * qi[d];
                             }
                         }
                     }
@@ -330,12 +363,13 @@ static int attn_bwd_core(const oracle_shape_t *s, const void *q, const void *k,
 
 #define ORACLE_SHAPE                                                        \
     oracle_shape_t s = {B, Hq, Hkv, Sq, Sk, D, scale, causal, window_left,  \
-                        window_right, doc_offsets, num_docs}
+                        window_right, doc_offsets, num_docs, softcap, alibi_slopes}
 
 int oracle_attn_fwd_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                          double *o, double *lse, int B, int Hq, int Hkv, int Sq,
                          int Sk, int D, double scale, int causal, int window_left,
                          int window_right, const int *doc_offsets, int num_docs,
+                         double softcap, const double *alibi_slopes,
                          const int64_t *rows, int64_t n_rows) {
     ORACLE_SHAPE;
     return attn_fwd_core(&s, q, k, v, 1, o, lse, rows, n_rows);
@@ -345,6 +379,7 @@ int oracle_attn_fwd_f64(const double *q, const double *k, const double *v,
                         double *o, double *lse, int B, int Hq, int Hkv, int Sq,
                         int Sk, int D, double scale, int causal, int window_left,
                         int window_right, const int *doc_offsets, int num_docs,
+                        double softcap, const double *alibi_slopes,
                         const int64_t *rows, int64_t n_rows) {
     ORACLE_SHAPE;
     return attn_fwd_core(&s, q, k, v, 0, o, lse, rows, n_rows);
@@ -354,7 +389,8 @@ int oracle_attn_bwd_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v
                          const uint16_t *dout, double *dq, double *dk, double *dv,
                          double *o, double *lse, int B, int Hq, int Hkv, int Sq,
                          int Sk, int D, double scale, int causal, int window_left,
-                         int window_right, const int *doc_offsets, int num_docs) {
+                         int window_right, const int *doc_offsets, int num_docs,
+                         double softcap, const double *alibi_slopes) {
     ORACLE_SHAPE;
     return attn_bwd_core(&s, q, k, v, dout, 1, dq, dk, dv, o, lse);
 }
@@ -363,7 +399,8 @@ int oracle_attn_bwd_f64(const double *q, const double *k, const double *v,
                         const double *dout, double *dq, double *dk, double *dv,
                         double *o, double *lse, int B, int Hq, int Hkv, int Sq,
                         int Sk, int D, double scale, int causal, int window_left,
-                        int window_right, const int *doc_offsets, int num_docs) {
+                        int window_right, const int *doc_offsets, int num_docs,
+                        double softcap, const double *alibi_slopes) {
     ORACLE_SHAPE;
     return attn_bwd_core(&s, q, k, v, dout, 0, dq, dk, dv, o, lse);
 }

@@ -321,3 +321,86 @@ def test_backward_matches_torch_autograd_float64():
     np.testing.assert_allclose(dq, tq.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
     np.testing.assert_allclose(dk, tk.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
     np.testing.assert_allclose(dv, tv.grad.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+
+
+# ------------------------------------------- score modifiers (soft-cap, ALiBi)
+
+def test_alibi_equal_logits_give_geometric_weights():
+    """Q = 0 and a causal mask leave only the ALiBi bias -m (i - j): weights
+    r^(i-j) / sum_t r^t with r = e^-m, so LSE_i = log((1 - r^(i+1)) / (1 - r))."""
+    S, D, m = 23, 4, 0.37
+    q = np.zeros((1, S, 2, D))
+    k, v = randn(1, S, 1, D), randn(1, S, 1, D)
+    slopes = [m, 2 * m]
+    o, lse = oracle.attn_fwd(q, k, v, scale=0.5, causal=True, alibi_slopes=slopes)
+    for h, mh in enumerate(slopes):
+        r = math.exp(-mh)
+        for i in range(S):
+            w = r ** (i - np.arange(i + 1))
+            np.testing.assert_allclose(o[0, i, h], (w[:, None] * v[0, :i + 1, 0]).sum(0) / w.sum(),
+                                       atol=1e-13)
+            assert abs(lse[0, h, i] - math.log((1 - r ** (i + 1)) / (1 - r))) < 1e-12
+
+
+def test_softcap_two_keys_is_logistic_of_capped_gap():
+    """Two keys with scaled scores 0 and a: the cap maps a to c tanh(a / c),
+    so the weights are the logistic function of that value."""
+    c, a = 2.5, 4.0
+    q = np.array([[a, 0.0]]).reshape(1, 1, 1, 2)
+    k = np.array([[0.0, 0.0], [1.0, 0.0]]).reshape(1, 2, 1, 2)
+    v = np.array([[1.0, 0.0], [0.0, 1.0]]).reshape(1, 2, 1, 2)
+    o, lse = oracle.attn_fwd(q, k, v, scale=1.0, softcap=c)
+    z = c * math.tanh(a / c)
+    np.testing.assert_allclose(o[0, 0, 0], [1 / (1 + math.exp(z)), math.exp(z) / (1 + math.exp(z))],
+                               atol=1e-15)
+    assert abs(lse[0, 0, 0] - math.log1p(math.exp(z))) < 1e-14
+
+
+def test_huge_softcap_is_no_softcap():
+    q, k, v = randn(1, 30, 2, 8), randn(1, 30, 2, 8), randn(1, 30, 2, 8)
+    o1, l1 = oracle.attn_fwd(q, k, v, scale=0.3, causal=True)
+    o2, l2 = oracle.attn_fwd(q, k, v, scale=0.3, causal=True, softcap=1e9)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,Sq", [(True, 40), (False, 40), (True, 25)])
+def test_modifiers_match_scipy_on_dense_scores(causal, Sq):
+    B, Sk, Hq, Hkv, D = 1, 40, 4, 2, 8
+    q, k, v = randn(B, Sq, Hq, D, scale=3.0), randn(B, Sk, Hkv, D, scale=3.0), randn(B, Sk, Hkv, D)
+    cap, slopes = 3.0, np.array([0.5, 0.25, 0.125, 0.0625])
+    mask = dense_mask(Sq, Sk, causal)
+    dist = np.abs(np.arange(Sq)[:, None] + (Sk - Sq) - np.arange(Sk)[None, :])
+    o_ref = np.zeros_like(q)
+    lse_ref = np.zeros((B, Hq, Sq))
+    g = Hq // Hkv
+    for h in range(Hq):
+        s = 0.4 * q[0, :, h, :] @ k[0, :, h // g, :].T
+        s = cap * np.tanh(s / cap) - slopes[h] * dist
+        s = np.where(mask, s, -np.inf)
+        lse_ref[0, h] = scipy.special.logsumexp(s, axis=1)
+        o_ref[0, :, h, :] = scipy.special.softmax(s, axis=1) @ v[0, :, h // g, :]
+    o, lse = oracle.attn_fwd(q, k, v, scale=0.4, causal=causal, softcap=cap, alibi_slopes=slopes)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+
+
+@pytest.mark.parametrize("mods", [dict(softcap=1.5), dict(alibi_slopes=[0.3, 0.7]),
+                                  dict(softcap=2.0, alibi_slopes=[0.2, 0.05])])
+def test_backward_with_modifiers_matches_central_differences(mods):
+    B, S, Hq, Hkv, D = 1, 6, 2, 1, 3
+    q, k, v = randn(B, S, Hq, D, scale=2.0), randn(B, S, Hkv, D, scale=2.0), randn(B, S, Hkv, D)
+    dout = randn(B, S, Hq, D)
+    kw = dict(mods, scale=0.9, causal=True)
+    dq, dk, dv, _, _ = oracle.attn_bwd(q, k, v, dout, **kw)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = {"q": q, "k": k, "v": v}
+            fd[idx] = (_loss(**{**args, name: xp}, dout=dout, **kw) -
+                       _loss(**{**args, name: xm}, dout=dout, **kw)) / (2 * h)
+        np.testing.assert_allclose(g, fd, atol=2e-8, rtol=1e-6, err_msg=name)
