@@ -86,7 +86,17 @@ typedef struct {
      * units).  0 = all on the MUFU ex2 unit; 1 = the tuned split
      * (default); 2 = every column of unmasked tiles by polynomial. */
     int exp2_mode;
-    int reserved[6]; /* must be zero */
+    /* Bound of every device-side wait of the forward, in microseconds
+     * (0 = the default, 1 s).  A wait that runs out makes the kernel record
+     * ATTN_ERR_DEVICE_TIMEOUT, finish its in-flight copies and MMAs, free its
+     * tensor memory and return.  Valid range [0, 60000000]. */
+    int wait_timeout_us;
+    /* Testing only (keep 0): 1 makes the first CTA withhold the copy of its
+     * first key block, so its MMA warp's wait runs out and the call reports
+     * ATTN_ERR_DEVICE_TIMEOUT through attn_get_device_status().  Nothing
+     * faults; the outputs of that CTA are left unwritten. */
+    int debug_withhold_kv;
+    int reserved[4]; /* must be zero */
 } attn_fwd_options_t;
 
 /* Fills *opts with the defaults. */

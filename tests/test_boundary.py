@@ -51,7 +51,8 @@ def test_status_strings_and_version(L):
 
 def test_default_options(L):
     o = attn.default_options()
-    assert o.rescale_threshold == 8.0 and o.exp2_mode == 1 and list(o.reserved) == [0] * 6
+    assert o.rescale_threshold == 8.0 and o.exp2_mode == 1 and list(o.reserved) == [0] * 4
+    assert o.wait_timeout_us == 0 and o.debug_withhold_kv == 0
 
 
 # Fake, 16-byte-aligned device addresses: validation must reject the call
@@ -103,7 +104,10 @@ def test_invalid_arguments_rejected_before_launch(L, kw, status):
 @pytest.mark.parametrize("field,value", [("rescale_threshold", -1.0),
                                          ("rescale_threshold", 17.0),
                                          ("rescale_threshold", float("nan")),
-                                         ("exp2_mode", 3), ("exp2_mode", -1)])
+                                         ("exp2_mode", 3), ("exp2_mode", -1),
+                                         ("wait_timeout_us", -1),
+                                         ("wait_timeout_us", 60000001),
+                                         ("debug_withhold_kv", 2)])
 def test_invalid_options_rejected(L, field, value):
     opts = attn.default_options()
     setattr(opts, field, value)

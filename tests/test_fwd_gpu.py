@@ -193,3 +193,21 @@ def test_full_size_workload_sampled(name):
     assert err.max() <= O_MAX, f"{name}: O max-abs {err.max():.3e}"
     assert err.mean() <= O_MEAN, f"{name}: O mean-abs {err.mean():.3e}"
     assert np.abs(lse_s - lse_ref).max() <= LSE_TOL
+
+
+# ----------------------------------------------------------- failure path
+
+def test_device_wait_timeout_is_reported_and_recoverable():
+    """A wait that runs out (the first CTA withholds a key copy, nothing
+    faults) makes the call report ATTN_ERR_DEVICE_TIMEOUT through the status
+    word; reading clears it, and the device keeps computing correct results."""
+    t = make_tensors(1, 2, 2, 512, 512, 128, seed=81)
+    q, k, v = (t[n].to(DEV) for n in ("q", "k", "v"))
+    opts = attn.default_options(wait_timeout_us=20000, debug_withhold_kv=1)
+    attn.attention(q, k, v, causal=True, options=opts)
+    assert attn.device_status() == attn.ATTN_ERR_DEVICE_TIMEOUT
+    assert attn.device_status() == attn.ATTN_OK
+    o, lse = run_gpu(t, causal=True, scale=1 / math.sqrt(128))
+    o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=1 / math.sqrt(128),
+                                     causal=True)
+    check(o, lse, o_ref, lse_ref, "after a timeout")

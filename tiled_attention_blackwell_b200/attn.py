@@ -39,7 +39,8 @@ class AttnError(RuntimeError):
 class FwdOptions(ctypes.Structure):
     """Mirror of attn_fwd_options_t."""
     _fields_ = [("rescale_threshold", ctypes.c_float), ("exp2_mode", ctypes.c_int),
-                ("reserved", ctypes.c_int * 6)]
+                ("wait_timeout_us", ctypes.c_int), ("debug_withhold_kv", ctypes.c_int),
+                ("reserved", ctypes.c_int * 4)]
 
 
 _FWD_ARGS = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [ctypes.c_float] + \

@@ -285,6 +285,10 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
         return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must lie in [0, 16]");
     if (op.exp2_mode < 0 || op.exp2_mode > 2)
         return fail(ATTN_ERR_INVALID_ARG, "exp2_mode must be 0, 1 or 2");
+    if (op.wait_timeout_us < 0 || op.wait_timeout_us > 60000000)
+        return fail(ATTN_ERR_INVALID_ARG, "wait_timeout_us must lie in [0, 60000000]");
+    if (op.debug_withhold_kv != 0 && op.debug_withhold_kv != 1)
+        return fail(ATTN_ERR_INVALID_ARG, "debug_withhold_kv must be 0 or 1");
     for (int r : op.reserved)
         if (r != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved option fields must be zero");
     const long long num_qblocks = (Sq + 2LL * tab::kBlockM - 1) / (2LL * tab::kBlockM);
@@ -319,6 +323,9 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
     p.head_group = std::min(B * Hq, kFwdHeadGroup * (Hq / Hkv));
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     p.rescale_threshold = op.rescale_threshold;
+    p.timeout_ns = op.wait_timeout_us > 0 ? 1000ull * (unsigned long long)op.wait_timeout_us
+                                          : tab::kWaitTimeoutNs;
+    p.debug_withhold_kv = op.debug_withhold_kv;
 #ifdef ATTN_TRACE
     p.trace = g_trace;
     p.trace_ctas = g_trace_ctas;

@@ -79,6 +79,8 @@ struct FwdParams {
     float rescale_threshold;
     long long *trace;  // clock64 event log (trace builds only), else null
     int trace_ctas;
+    unsigned long long timeout_ns;  // bound of every wait
+    int debug_withhold_kv;          // testing: CTA 0 skips its first K copy
 };
 
 // Opt-in event trace (compile with -DATTN_TRACE): lane 0 of warps 0 and 4
@@ -279,8 +281,11 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                     for (int which = 0; which < 2 && ok; ++which, ++it) {
                         const uint32_t slot = it % NS;
                         ok = wait_bounded(&sm.kv_empty[slot], ((it / NS) & 1u) ^ 1u, abort_flag,
-                                          p.status);
+                                          p.status, true, p.timeout_ns);
                         if (!ok) break;
+                        // Testing only: the first CTA withholds its first K copy (the
+                        // loop increment still advances the ring position).
+                        if (p.debug_withhold_kv && blockIdx.x == 0 && it == 0) continue;
                         mbar_arrive_expect_tx(&sm.kv_full[slot], kTileBytes);
                         const CUtensorMap *map = which ? &p.tm_v : &p.tm_k;
                         for (int c = 0; c < Smem::kChunks; ++c)
@@ -290,10 +295,10 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 // Every copy still in flight lands before the CTA can exit (only
                 // the last NS loads can be outstanding; on the normal path they
                 // have been consumed already).
-                wait_bounded(&sm.q_full, 0, abort_flag, p.status, false);
+                wait_bounded(&sm.q_full, 0, abort_flag, p.status, false, p.timeout_ns);
                 const uint32_t first = it > NS ? it - NS : 0;
                 for (uint32_t L = first; L < it; ++L)
-                    wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status, false);
+                    wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status, false, p.timeout_ns);
             }
             __syncwarp();
         } else if (warp == 8) {
@@ -314,7 +319,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 const uint64_t v_desc =
                     smem_desc_sw128(smem_u32(&sm.kv[0][0][0]), kChunkBytes, 1024);
                 bool ok = __all_sync(0xffffffffu,
-                                     wait_bounded(&sm.q_full, 0, abort_flag, p.status));
+                                     wait_bounded(&sm.q_full, 0, abort_flag, p.status, true, p.timeout_ns));
                 tc_fence_after();
                 int k_ready = ulo - 1;  // last key block whose K slot was waited on
                 auto ring_pos = [&](int j, int which) -> uint32_t {
@@ -325,7 +330,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                     if (ok)
                         ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[L % NS],
                                                                   (L / NS) & 1u, abort_flag,
-                                                                  p.status));
+                                                                  p.status, true, p.timeout_ns));
                     tc_fence_after();
                     k_ready = j;
                 };
@@ -361,7 +366,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                     const uint32_t vslot = Lv % NS;
                     ATTN_TRACE_EVENT(2, j - ulo, 0);
                     ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[vslot], (Lv / NS) & 1u,
-                                                              abort_flag, p.status));
+                                                              abort_flag, p.status, true, p.timeout_ns));
                     ATTN_TRACE_EVENT(2, j - ulo, 1);
                     if (!ok) break;
                     tc_fence_after();
@@ -379,7 +384,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                             // (SBO), 64-column chunks kChunkBytes apart (LBO).
                             ATTN_TRACE_EVENT(2, j - ulo, 2 + 3 * i);
                             ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_half[i], par,
-                                                                      abort_flag, p.status));
+                                                                      abort_flag, p.status, true, p.timeout_ns));
                             if (!ok) break;
                             tc_fence_after();
                             if (leader) {
@@ -390,7 +395,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                             }
                             __syncwarp();
                             ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_full[i], par,
-                                                                      abort_flag, p.status));
+                                                                      abort_flag, p.status, true, p.timeout_ns));
                             ATTN_TRACE_EVENT(2, j - ulo, 3 + 3 * i);
                             if (!ok) break;
                             tc_fence_after();
@@ -419,7 +424,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                     // Let every MMA already issued finish before TMEM is freed.
                     if (leader) tc_commit(&sm.drain);
                     __syncwarp();
-                    wait_bounded(&sm.drain, 0, abort_flag, p.status, false);
+                    wait_bounded(&sm.drain, 0, abort_flag, p.status, false, p.timeout_ns);
                 }
             }
             __syncwarp();
@@ -446,7 +451,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         for (int j = lo_b; j <= hi_b; ++j) {
             const int t = j - lo_b;
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 0);
-            ok = wait_bounded(&sm.s_full[i], (uint32_t)t & 1u, abort_flag, p.status);
+            ok = wait_bounded(&sm.s_full[i], (uint32_t)t & 1u, abort_flag, p.status, true, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
@@ -557,7 +562,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         // ----------------------------------------------------------- epilogue
         const bool has_blocks = lo_b <= hi_b;
         if (ok && has_blocks) {
-            ok = wait_bounded(&sm.o_final[i], 0, abort_flag, p.status);
+            ok = wait_bounded(&sm.o_final[i], 0, abort_flag, p.status, true, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
         }
