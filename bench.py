@@ -236,10 +236,15 @@ def oracle_sample(w, inputs, n_rows: int, seed: int = 0):
 
 
 def rows_for_seconds(w, inputs, seconds: float) -> int:
-    """Calibrate the row count so the oracle runs for about `seconds`."""
-    n = 500
-    dt, _, _ = oracle_sample(w, inputs, n, seed=123)
-    return max(100, int(n * seconds / max(dt, 1e-3)))
+    """Calibrate the row count so the oracle runs for about `seconds`.  Each
+    call has a fixed cost (converting the inputs) besides the per-row work, so
+    two sample sizes give both terms."""
+    n1, n2 = 200, 1200
+    t1, _, _ = oracle_sample(w, inputs, n1, seed=123)
+    t2, _, _ = oracle_sample(w, inputs, n2, seed=124)
+    per_row = max((t2 - t1) / (n2 - n1), 1e-7)
+    fixed = max(t1 - n1 * per_row, 0.0)
+    return max(100, int(max(seconds - fixed, 0.0) / per_row))
 
 
 def workload_config(w, doc_offsets):

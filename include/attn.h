@@ -96,8 +96,29 @@ typedef struct {
      * ATTN_ERR_DEVICE_TIMEOUT through attn_get_device_status().  Nothing
      * faults; the outputs of that CTA are left unwritten. */
     int debug_withhold_kv;
+    /* Score modifiers ("El FlexAttention de PyTorch con FlashAttention-4",
+     * intro: soft-capping, ALiBi), applied in this order to the scaled score
+     * s = scale * <q_i, k_j> before the mask:
+     *   softcap > 0        : s <- softcap * tanh(s / softcap)
+     *   alibi_slopes != 0  : s <- s - alibi_slopes[hq] * |i + (Sk - Sq) - j|
+     * softcap = 0 and alibi_slopes = NULL (the defaults) leave s unchanged.
+     * alibi_slopes is device memory, fp32 [Hq], 4-byte aligned.  With a
+     * modifier the exponentials all run on MUFU (exp2_mode is ignored). */
+    float softcap;
+    int reserved0; /* must be zero */
+    const float *alibi_slopes;
     int reserved[4]; /* must be zero */
 } attn_fwd_options_t;
+
+/* Score modifiers of the backward: the same meaning as in
+ * attn_fwd_options_t, and they must match the forward that produced O and
+ * LSE.  Pass NULL to attn_bwd_ex for none. */
+typedef struct {
+    float softcap;
+    int reserved0; /* must be zero */
+    const float *alibi_slopes;
+    int reserved[4]; /* must be zero */
+} attn_bwd_options_t;
 
 /* Fills *opts with the defaults. */
 ATTN_API void attn_fwd_default_options(attn_fwd_options_t *opts);
@@ -148,6 +169,17 @@ ATTN_API attn_status_t attn_bwd(const void *q, const void *k, const void *v, con
                                 float scale, int causal, int window_left, int window_right,
                                 const int *doc_offsets, int num_docs, void *workspace,
                                 size_t workspace_bytes, void *stream);
+
+/* attn_bwd with score modifiers (NULL = none).  Under a soft-cap the
+ * gradients carry the cap's derivative: dL/d<q_i,k_j> = dS_ij * scale *
+ * (1 - tanh^2(s_ij / softcap)). */
+ATTN_API attn_status_t attn_bwd_ex(const void *q, const void *k, const void *v, const void *o,
+                                   const float *lse, const void *dout, float *dq, void *dk,
+                                   void *dv, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                                   float scale, int causal, int window_left, int window_right,
+                                   const int *doc_offsets, int num_docs, void *workspace,
+                                   size_t workspace_bytes, const attn_bwd_options_t *opts,
+                                   void *stream);
 
 /*
  * attn_bwd without a workspace argument, for callers that cannot allocate

@@ -118,6 +118,29 @@ def test_reserved_options_must_be_zero(L):
     opts = attn.default_options()
     opts.reserved[2] = 1
     assert call(L, opts=opts) == attn.ATTN_ERR_INVALID_ARG
+    opts = attn.default_options()
+    opts.reserved0 = 1
+    assert call(L, opts=opts) == attn.ATTN_ERR_INVALID_ARG
+
+
+def test_default_options_select_no_modifier(L):
+    o = attn.default_options()
+    assert o.softcap == 0.0 and o.alibi_slopes is None and o.reserved0 == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("softcap", -1.0, attn.ATTN_ERR_INVALID_ARG),
+    ("softcap", float("nan"), attn.ATTN_ERR_INVALID_ARG),
+    ("softcap", float("inf"), attn.ATTN_ERR_INVALID_ARG),
+    ("alibi_slopes", P + 2, attn.ATTN_ERR_MISALIGNED),
+])
+def test_invalid_modifiers_rejected(L, field, value, status):
+    opts = attn.default_options()
+    setattr(opts, field, value)
+    assert call(L, opts=opts) == status
+    bopts = attn.BwdOptions()
+    setattr(bopts, field, value)
+    assert call_bwd(L, opts=bopts) == status
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
@@ -127,15 +150,18 @@ def test_valid_call_without_gpu_reports_cuda_error(L):
 
 def call_bwd(L, **kw):
     a = dict(ptr=P, lse=P, ws=P, B=1, Hq=2, Hkv=2, Sq=16, Sk=16, D=128, scale=0.1, causal=1,
-             wl=-1, wr=-1, docs=None, nd=0, wsb=1 << 20)
+             wl=-1, wr=-1, docs=None, nd=0, wsb=1 << 20, opts=None)
     a.update(kw)
     vp = ctypes.c_void_p
     ptrs = [vp(a.get(n, a["ptr"])) for n in ("q", "k", "v", "o")]
     ptrs += [vp(a["lse"])]
     ptrs += [vp(a.get(n, a["ptr"])) for n in ("dout", "dq", "dk", "dv")]
-    return L.attn_bwd(*ptrs, a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Sk"], a["D"], a["scale"],
-                      a["causal"], a["wl"], a["wr"], vp(a["docs"]) if a["docs"] else None, a["nd"],
-                      vp(a["ws"]), a["wsb"], None)
+    args = ptrs + [a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Sk"], a["D"], a["scale"], a["causal"],
+                   a["wl"], a["wr"], vp(a["docs"]) if a["docs"] else None, a["nd"], vp(a["ws"]),
+                   a["wsb"]]
+    if a["opts"] is None:
+        return L.attn_bwd(*args, None)
+    return L.attn_bwd_ex(*args, ctypes.byref(a["opts"]), None)
 
 
 def test_bwd_workspace_size(L):
@@ -157,6 +183,13 @@ def test_bwd_workspace_size(L):
 ])
 def test_bwd_invalid_arguments_rejected_before_launch(L, kw, status):
     assert call_bwd(L, **kw) == status
+    assert call_bwd(L, opts=attn.BwdOptions(), **kw) == status
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
+def test_valid_bwd_calls_without_gpu_report_cuda_error(L):
+    assert call_bwd(L) == attn.ATTN_ERR_CUDA
+    assert call_bwd(L, opts=attn.BwdOptions(softcap=30.0, alibi_slopes=P)) == attn.ATTN_ERR_CUDA
 
 
 def test_binding_refuses_cpu_tensors(L):

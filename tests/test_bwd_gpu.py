@@ -31,13 +31,17 @@ def _lib():
     assert attn.device_status() == attn.ATTN_OK
 
 
-def gpu_grads(t, *, scale, causal=False, window=None, doc_offsets=None):
+def gpu_grads(t, *, scale, causal=False, window=None, doc_offsets=None, softcap=None,
+              alibi_slopes=None):
     q, k, v, dout = (t[n].to(DEV) for n in ("q", "k", "v", "dout"))
     docs = None if doc_offsets is None else torch.as_tensor(doc_offsets, dtype=torch.int32,
                                                              device=DEV)
-    o, lse = attn.attention(q, k, v, scale=scale, causal=causal, window=window, doc_offsets=docs)
+    slopes = None if alibi_slopes is None else torch.as_tensor(alibi_slopes, device=DEV)
+    o, lse = attn.attention(q, k, v, scale=scale, causal=causal, window=window, doc_offsets=docs,
+                            softcap=softcap, alibi_slopes=slopes)
     dq, dk, dv = attn.attention_backward(q, k, v, o, lse, dout, scale=scale, causal=causal,
-                                         window=window, doc_offsets=docs)
+                                         window=window, doc_offsets=docs, softcap=softcap,
+                                         alibi_slopes=slopes)
     torch.cuda.synchronize()
     return [x.float().cpu().numpy().astype(np.float64) for x in (dq, dk, dv)]
 
@@ -53,13 +57,45 @@ def check_grads(got, ref, what):
         assert err <= GRAD_TOL * scale, f"{what}: {name} max-abs {err:.3e} vs {GRAD_TOL}*{scale:.3e}"
 
 
-def case(B, Hq, Hkv, Sq, Sk, D, seed, *, causal=False, window=None, docs=None):
-    t = make_tensors(B, Hq, Hkv, Sq, Sk, D, seed, with_dout=True)
+def case(B, Hq, Hkv, Sq, Sk, D, seed, *, causal=False, window=None, docs=None, softcap=None,
+         alibi_slopes=None, qk_std=1.0):
+    t = make_tensors(B, Hq, Hkv, Sq, Sk, D, seed, with_dout=True, qk_std=qk_std)
     scale = 1.0 / math.sqrt(D)
-    got = gpu_grads(t, scale=scale, causal=causal, window=window, doc_offsets=docs)
+    got = gpu_grads(t, scale=scale, causal=causal, window=window, doc_offsets=docs,
+                    softcap=softcap, alibi_slopes=alibi_slopes)
     dq, dk, dv, _, _ = oracle.attn_bwd(t["q"], t["k"], t["v"], t["dout"], scale=scale,
-                                       causal=causal, window=window, doc_offsets=docs)
-    check_grads(got, (dq, dk, dv), f"B{B} Hq{Hq} Hkv{Hkv} Sq{Sq} Sk{Sk} D{D} causal={causal}")
+                                       causal=causal, window=window, doc_offsets=docs,
+                                       softcap=softcap or 0.0, alibi_slopes=alibi_slopes)
+    check_grads(got, (dq, dk, dv), f"B{B} Hq{Hq} Hkv{Hkv} Sq{Sq} Sk{Sk} D{D} causal={causal} "
+                                   f"softcap={softcap} alibi={alibi_slopes is not None}")
+
+
+def geometric_slopes(H):
+    """Per-head ALiBi slopes 2^(-8 (h+1) / H) as fp32 (an input, like Q)."""
+    return np.float32(2.0) ** (-8.0 * np.arange(1, H + 1, dtype=np.float32) / H)
+
+
+@pytest.mark.parametrize("softcap", [3.0, 30.0])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_softcap_backward(softcap, D, causal):
+    case(1, 2, 2, 400, 400, D, seed=301, causal=causal, softcap=softcap, qk_std=2.0)
+
+
+@pytest.mark.parametrize("Sq,Sk", [(400, 400), (200, 520), (520, 200)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_alibi_backward(Sq, Sk, causal):
+    case(1, 4, 4, Sq, Sk, 128, seed=302, causal=causal, alibi_slopes=geometric_slopes(4))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_softcap_and_alibi_backward_with_gqa_window_and_documents(D):
+    case(2, 4, 2, 450, 450, D, seed=303, causal=True, softcap=6.0,
+         alibi_slopes=geometric_slopes(4), qk_std=1.5)
+    case(1, 4, 1, 450, 450, D, seed=304, window=(100, 30), softcap=6.0,
+         alibi_slopes=geometric_slopes(4))
+    case(1, 2, 2, 400, 400, D, seed=305, causal=True, docs=[0, 1, 129, 250, 400], softcap=10.0,
+         alibi_slopes=geometric_slopes(2))
 
 
 @pytest.mark.parametrize("D", [64, 128])

@@ -49,7 +49,7 @@ def check(o, lse, o_ref, lse_ref, what=""):
     err = np.abs(o - o_ref)
     assert err.max() <= O_MAX, f"{what}: O max-abs {err.max():.3e}"
     assert err.mean() <= O_MEAN, f"{what}: O mean-abs {err.mean():.3e}"
-    lse_err = np.abs(np.where(empty, 0.0, lse - lse_ref))
+    lse_err = np.abs(np.where(empty, 0.0, lse) - np.where(empty, 0.0, lse_ref))
     assert lse_err.max() <= LSE_TOL, f"{what}: LSE abs {lse_err.max():.3e}"
     if empty.any():
         # rows with no key: O exactly zero (LSE layout [B,H,S] vs O [B,S,H,D])
@@ -128,6 +128,69 @@ def test_large_logits_stay_finite():
         o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=1 / math.sqrt(128),
                                          causal=True)
         check(o, lse, o_ref, lse_ref, f"large logits exp2_mode={exp2_mode}")
+
+
+# ---------------------------------------------------------- score modifiers
+
+def geometric_slopes(H):
+    """Per-head ALiBi slopes 2^(-8 (h+1) / H) as fp32 (an input, like Q)."""
+    return np.float32(2.0) ** (-8.0 * np.arange(1, H + 1, dtype=np.float32) / H)
+
+
+def modifier_case(B, Hq, Hkv, Sq, Sk, D, seed, *, softcap=None, alibi=False, causal=False,
+                  window=None, doc_offsets=None, qk_std=1.0):
+    t = make_tensors(B, Hq, Hkv, Sq, Sk, D, seed, qk_std=qk_std)
+    scale = 1.0 / math.sqrt(D)
+    slopes = geometric_slopes(Hq) if alibi else None
+    q, k, v = (t[n].to(DEV) for n in ("q", "k", "v"))
+    docs = None if doc_offsets is None else torch.as_tensor(doc_offsets, dtype=torch.int32,
+                                                             device=DEV)
+    o, lse = attn.attention(q, k, v, scale=scale, causal=causal, window=window, doc_offsets=docs,
+                            softcap=softcap,
+                            alibi_slopes=None if slopes is None else torch.from_numpy(slopes).to(DEV))
+    torch.cuda.synchronize()
+    o = o.float().cpu().numpy().astype(np.float64)
+    lse = lse.cpu().numpy().astype(np.float64)
+    o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=scale, causal=causal,
+                                     window=window, doc_offsets=doc_offsets,
+                                     softcap=softcap or 0.0, alibi_slopes=slopes)
+    check(o, lse, o_ref, lse_ref, f"softcap={softcap} alibi={alibi} causal={causal} D{D}")
+
+
+@pytest.mark.parametrize("softcap", [2.0, 5.0, 30.0])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_softcap(softcap, D, causal):
+    # qk_std 2 gives scaled scores of std ~4, so a cap of 2 or 5 is active.
+    modifier_case(2, 2, 2, 700, 700, D, seed=71, softcap=softcap, causal=causal, qk_std=2.0)
+
+
+@pytest.mark.parametrize("Sq,Sk", [(700, 700), (300, 1000), (1000, 300), (1, 515)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_alibi(Sq, Sk, causal):
+    modifier_case(1, 8, 8, Sq, Sk, 128, seed=72, alibi=True, causal=causal)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_softcap_and_alibi_with_gqa_window_and_documents(D):
+    modifier_case(2, 8, 2, 900, 900, D, seed=73, softcap=8.0, alibi=True, causal=True,
+                  qk_std=1.5)
+    modifier_case(1, 4, 2, 900, 900, D, seed=74, softcap=8.0, alibi=True, window=(200, 50))
+    modifier_case(1, 4, 1, 700, 700, D, seed=75, softcap=20.0, alibi=True, causal=True,
+                  doc_offsets=[0, 1, 130, 400, 700])
+
+
+def test_modifier_options_struct_path():
+    """The same modifiers given through the options struct instead of the
+    keyword arguments."""
+    t = make_tensors(1, 4, 4, 333, 333, 128, seed=76, qk_std=2.0)
+    slopes = torch.from_numpy(geometric_slopes(4)).to(DEV)
+    opts = attn.default_options(softcap=6.0, alibi_slopes=slopes.data_ptr())
+    o, lse = run_gpu(t, causal=True, scale=1 / math.sqrt(128), options=opts)
+    o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=1 / math.sqrt(128),
+                                     causal=True, softcap=6.0,
+                                     alibi_slopes=geometric_slopes(4))
+    check(o, lse, o_ref, lse_ref, "options struct")
 
 
 # -------------------------------------------------------- memory discipline

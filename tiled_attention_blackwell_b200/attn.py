@@ -26,7 +26,7 @@ ATTN_ERR_DEVICE_TIMEOUT = 5
 ATTN_ERR_CUDA = 6
 
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_default_options", "attn_bwd",
-            "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_status",
+            "attn_bwd_ex", "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_status",
             "attn_status_string", "attn_last_error_detail", "attn_abi_version")
 
 
@@ -40,7 +40,14 @@ class FwdOptions(ctypes.Structure):
     """Mirror of attn_fwd_options_t."""
     _fields_ = [("rescale_threshold", ctypes.c_float), ("exp2_mode", ctypes.c_int),
                 ("wait_timeout_us", ctypes.c_int), ("debug_withhold_kv", ctypes.c_int),
-                ("reserved", ctypes.c_int * 4)]
+                ("softcap", ctypes.c_float), ("reserved0", ctypes.c_int),
+                ("alibi_slopes", ctypes.c_void_p), ("reserved", ctypes.c_int * 4)]
+
+
+class BwdOptions(ctypes.Structure):
+    """Mirror of attn_bwd_options_t."""
+    _fields_ = [("softcap", ctypes.c_float), ("reserved0", ctypes.c_int),
+                ("alibi_slopes", ctypes.c_void_p), ("reserved", ctypes.c_int * 4)]
 
 
 _FWD_ARGS = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [ctypes.c_float] + \
@@ -80,6 +87,9 @@ def lib():
                 [ctypes.c_float] + [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int,
                                                          ctypes.c_void_p, ctypes.c_size_t,
                                                          ctypes.c_void_p]
+            L.attn_bwd_ex.restype = ctypes.c_int
+            L.attn_bwd_ex.argtypes = L.attn_bwd.argtypes[:-1] + [ctypes.POINTER(BwdOptions),
+                                                                 ctypes.c_void_p]
             L.attn_bwd_noalloc.restype = ctypes.c_int
             L.attn_bwd_noalloc.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int] * 6 + \
                 [ctypes.c_float] + [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int,
@@ -113,12 +123,29 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _slopes(alibi_slopes, Hq, device, stream):
+    """ALiBi slopes as a contiguous CUDA fp32 [Hq] tensor that stays valid
+    until the kernel that reads it has run on `stream`."""
+    if alibi_slopes is None:
+        return None
+    if not torch.is_tensor(alibi_slopes) or not alibi_slopes.is_cuda:
+        alibi_slopes = torch.as_tensor(alibi_slopes, dtype=torch.float32).to(device)
+        if stream is not None:
+            alibi_slopes.record_stream(stream)
+    if alibi_slopes.dtype != torch.float32 or not alibi_slopes.is_contiguous() \
+            or alibi_slopes.numel() != Hq:
+        raise TypeError("alibi_slopes must be a contiguous fp32 tensor of Hq entries")
+    return alibi_slopes
+
+
 def attn_fwd(q, k, v, o, lse, *, scale, causal=False, window=None, doc_offsets=None,
-             options=None, stream=None):
+             options=None, stream=None, softcap=None, alibi_slopes=None):
     """Enqueue the forward on `stream` (default: torch's current stream).
 
     q, o: bf16 CUDA [B,Sq,Hq,D]; k, v: bf16 CUDA [B,Sk,Hkv,D]; lse: fp32 CUDA
     [B,Hq,Sq]; doc_offsets: int32 CUDA [num_docs+1] or None.  All contiguous.
+    softcap (> 0) and alibi_slopes (fp32 [Hq]) select the score modifiers;
+    they override the same fields of `options`.
     """
     for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
                         ("v", v, torch.bfloat16), ("o", o, torch.bfloat16),
@@ -137,6 +164,16 @@ def attn_fwd(q, k, v, o, lse, *, scale, causal=False, window=None, doc_offsets=N
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
             float(scale), int(bool(causal)), wl, wr, docs_ptr, nd]
     L = lib()
+    slopes = _slopes(alibi_slopes, Hq, q.device, stream)
+    if softcap is not None or slopes is not None:
+        if options is None:
+            options = default_options()
+        else:
+            options = FwdOptions.from_buffer_copy(options)
+        if softcap is not None:
+            options.softcap = float(softcap)
+        if slopes is not None:
+            options.alibi_slopes = slopes.data_ptr()
     if options is None:
         st = L.attn_fwd(*args, _stream_handle(stream))
     else:
@@ -145,7 +182,7 @@ def attn_fwd(q, k, v, o, lse, *, scale, causal=False, window=None, doc_offsets=N
 
 
 def attention(q, k, v, *, scale=None, causal=False, window=None, doc_offsets=None,
-              options=None, stream=None):
+              options=None, stream=None, softcap=None, alibi_slopes=None):
     """Allocate O and LSE with torch and run the forward.  Returns (O, LSE)."""
     B, Sq, Hq, D = q.shape
     if scale is None:
@@ -157,7 +194,8 @@ def attention(q, k, v, *, scale=None, causal=False, window=None, doc_offsets=Non
     if doc_offsets is not None and not doc_offsets.is_cuda:
         doc_offsets = doc_offsets.to(q.device)
     attn_fwd(q, k, v, o, lse, scale=scale, causal=causal, window=window,
-             doc_offsets=doc_offsets, options=options, stream=stream)
+             doc_offsets=doc_offsets, options=options, stream=stream, softcap=softcap,
+             alibi_slopes=alibi_slopes)
     return o, lse
 
 
@@ -167,10 +205,11 @@ def bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D) -> int:
 
 
 def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, *, scale, causal=False, window=None,
-             doc_offsets=None, stream=None):
+             doc_offsets=None, stream=None, softcap=None, alibi_slopes=None):
     """Enqueue the backward on `stream`.  dq fp32 [B,Sq,Hq,D]; dk, dv bf16
     [B,Sk,Hkv,D]; workspace a CUDA uint8 tensor of at least
-    bwd_workspace_size() bytes."""
+    bwd_workspace_size() bytes.  softcap / alibi_slopes must match the
+    forward that produced o and lse."""
     for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
                         ("v", v, torch.bfloat16), ("o", o, torch.bfloat16),
                         ("lse", lse, torch.float32), ("dout", dout, torch.bfloat16),
@@ -189,15 +228,22 @@ def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, *, scale, causal=Fals
         docs_ptr, nd = _ptr(doc_offsets), doc_offsets.numel() - 1
     else:
         docs_ptr, nd = None, 0
-    st = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
-                        _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, D, float(scale),
-                        int(bool(causal)), wl, wr, docs_ptr, nd, _ptr(workspace),
-                        workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+            _ptr(dv), B, Hq, Hkv, Sq, Sk, D, float(scale), int(bool(causal)), wl, wr,
+            docs_ptr, nd, _ptr(workspace), workspace.numel() * workspace.element_size()]
+    slopes = _slopes(alibi_slopes, Hq, q.device, stream)
+    if softcap is None and slopes is None:
+        st = lib().attn_bwd(*args, _stream_handle(stream))
+    else:
+        opts = BwdOptions()
+        opts.softcap = float(softcap or 0.0)
+        opts.alibi_slopes = None if slopes is None else slopes.data_ptr()
+        st = lib().attn_bwd_ex(*args, ctypes.byref(opts), _stream_handle(stream))
     _check(st, "attn_bwd")
 
 
 def attention_backward(q, k, v, o, lse, dout, *, scale=None, causal=False, window=None,
-                       doc_offsets=None, stream=None):
+                       doc_offsets=None, stream=None, softcap=None, alibi_slopes=None):
     """Allocate dQ (fp32), dK, dV (bf16) and the workspace with torch and run
     the backward.  Returns (dQ, dK, dV)."""
     B, Sq, Hq, D = q.shape
@@ -214,7 +260,7 @@ def attention_backward(q, k, v, o, lse, dout, *, scale=None, causal=False, windo
     if doc_offsets is not None and not doc_offsets.is_cuda:
         doc_offsets = doc_offsets.to(q.device)
     attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, ws, scale=scale, causal=causal, window=window,
-             doc_offsets=doc_offsets, stream=stream)
+             doc_offsets=doc_offsets, stream=stream, softcap=softcap, alibi_slopes=alibi_slopes)
     return dq, dk, dv
 
 

@@ -104,12 +104,12 @@ attn_status_t make_map(CUtensorMap *map, const void *base, int B, int S, int H, 
 
 // --------------------------------------------------------------- launching
 
-template <int D, int NS, int EXP>
+template <int D, int NS, int EXP, int MOD = 0>
 attn_status_t launch_fwd(const tab::FwdParams &p, int grid, cudaStream_t stream) {
     using Smem = tab::FwdSmem<D, NS>;
     constexpr size_t smem = sizeof(Smem) + 1024;
     static_assert(smem <= 232448, "shared memory budget");
-    auto kernel = tab::attn_fwd_kernel<D, NS, EXP>;
+    auto kernel = tab::attn_fwd_kernel<D, NS, EXP, MOD>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     int dev = 0;
@@ -148,7 +148,15 @@ constexpr int kFwdHeadGroup = 8;
 constexpr int kStagesD64 = 8;
 
 template <int D, int NS>
-attn_status_t dispatch_exp(const tab::FwdParams &p, int grid, int exp_mode, cudaStream_t s) {
+attn_status_t dispatch_exp(const tab::FwdParams &p, int grid, int exp_mode, int mod,
+                           cudaStream_t s) {
+    // With a score modifier the exponentials all run on MUFU.
+    switch (mod) {
+        case 1: return launch_fwd<D, NS, 0, 1>(p, grid, s);
+        case 2: return launch_fwd<D, NS, 0, 2>(p, grid, s);
+        case 3: return launch_fwd<D, NS, 0, 3>(p, grid, s);
+        default: break;
+    }
     switch (exp_mode) {
         case 0: return launch_fwd<D, NS, 0>(p, grid, s);
         case 1: return launch_fwd<D, NS, 1>(p, grid, s);
@@ -203,7 +211,7 @@ attn_status_t prepare_kernel(Kernel kernel, size_t smem, int threads, int min_re
 constexpr int kBwdStagesQ = 2;
 constexpr int kBwdStagesKV = 4;
 
-template <int D>
+template <int D, int MOD>
 attn_status_t launch_bwd(const tab::BwdParams &p, cudaStream_t stream) {
     using DkdvS = tab::DkdvSmem<D, kBwdStagesQ>;
     using DqS = tab::DqSmem<D, kBwdStagesKV>;
@@ -211,8 +219,8 @@ attn_status_t launch_bwd(const tab::BwdParams &p, cudaStream_t stream) {
     constexpr size_t smem_dq = sizeof(DqS) + 1024;
     static_assert(smem_dkdv <= 232448 && smem_dq <= 232448, "shared memory budget");
     auto k_pre = tab::attn_bwd_preprocess_kernel<D>;
-    auto k_dkdv = tab::attn_bwd_dkdv_kernel<D, kBwdStagesQ>;
-    auto k_dq = tab::attn_bwd_dq_kernel<D, kBwdStagesKV>;
+    auto k_dkdv = tab::attn_bwd_dkdv_kernel<D, kBwdStagesQ, MOD>;
+    auto k_dq = tab::attn_bwd_dq_kernel<D, kBwdStagesKV, MOD>;
     static std::once_flag once[kMaxDevices];
     static attn_status_t prep[kMaxDevices];
     int dev = 0;
@@ -229,6 +237,29 @@ attn_status_t launch_bwd(const tab::BwdParams &p, cudaStream_t stream) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ATTN_ERR_LAUNCH, "launch: %s", cudaGetErrorString(e));
     return ok();
+}
+
+template <int D>
+attn_status_t dispatch_bwd(const tab::BwdParams &p, int mod, cudaStream_t stream) {
+    switch (mod) {
+        case 1: return launch_bwd<D, 1>(p, stream);
+        case 2: return launch_bwd<D, 2>(p, stream);
+        case 3: return launch_bwd<D, 3>(p, stream);
+        default: return launch_bwd<D, 0>(p, stream);
+    }
+}
+
+// Shared checks of the score-modifier fields of both option structs.
+attn_status_t check_modifiers(float softcap, int reserved0, const float *alibi_slopes,
+                              const int *reserved, int n_reserved) {
+    for (int i = 0; i < n_reserved; ++i)
+        if (reserved[i] != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved option fields must be zero");
+    if (reserved0 != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved option fields must be zero");
+    if (!(softcap >= 0.0f) || !std::isfinite(softcap))
+        return fail(ATTN_ERR_INVALID_ARG, "softcap must be >= 0 and finite");
+    if ((reinterpret_cast<uintptr_t>(alibi_slopes) & 3u) != 0)
+        return fail(ATTN_ERR_MISALIGNED, "alibi_slopes must be 4-byte aligned");
+    return ATTN_OK;
 }
 
 #ifdef ATTN_TRACE
@@ -289,8 +320,10 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
         return fail(ATTN_ERR_INVALID_ARG, "wait_timeout_us must lie in [0, 60000000]");
     if (op.debug_withhold_kv != 0 && op.debug_withhold_kv != 1)
         return fail(ATTN_ERR_INVALID_ARG, "debug_withhold_kv must be 0 or 1");
-    for (int r : op.reserved)
-        if (r != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved option fields must be zero");
+    {
+        attn_status_t c = check_modifiers(op.softcap, op.reserved0, op.alibi_slopes, op.reserved, 4);
+        if (c != ATTN_OK) return c;
+    }
     const long long num_qblocks = (Sq + 2LL * tab::kBlockM - 1) / (2LL * tab::kBlockM);
     const long long grid = num_qblocks * Hq * B;
     if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
@@ -326,14 +359,20 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
     p.timeout_ns = op.wait_timeout_us > 0 ? 1000ull * (unsigned long long)op.wait_timeout_us
                                           : tab::kWaitTimeoutNs;
     p.debug_withhold_kv = op.debug_withhold_kv;
+    const int mod = (op.softcap > 0.0f ? 1 : 0) | (op.alibi_slopes ? 2 : 0);
+    if (op.softcap > 0.0f) {
+        p.softcap_in = (float)((double)scale / op.softcap);
+        p.softcap_out = (float)((double)op.softcap * 1.4426950408889634);
+    }
+    p.alibi_slopes = op.alibi_slopes;
 #ifdef ATTN_TRACE
     p.trace = g_trace;
     p.trace_ctas = g_trace_ctas;
 #endif
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (D == 128) return dispatch_exp<128, kStagesD128>(p, (int)grid, op.exp2_mode, cs);
-    return dispatch_exp<64, kStagesD64>(p, (int)grid, op.exp2_mode, cs);
+    if (D == 128) return dispatch_exp<128, kStagesD128>(p, (int)grid, op.exp2_mode, mod, cs);
+    return dispatch_exp<64, kStagesD64>(p, (int)grid, op.exp2_mode, mod, cs);
 }
 
 attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -358,11 +397,28 @@ attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *
                        int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
                        int window_left, int window_right, const int *doc_offsets, int num_docs,
                        void *workspace, size_t workspace_bytes, void *stream) {
+    return attn_bwd_ex(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D, scale, causal,
+                       window_left, window_right, doc_offsets, num_docs, workspace,
+                       workspace_bytes, nullptr, stream);
+}
+
+attn_status_t attn_bwd_ex(const void *q, const void *k, const void *v, const void *o,
+                          const float *lse, const void *dout, float *dq, void *dk, void *dv,
+                          int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                          int causal, int window_left, int window_right,
+                          const int *doc_offsets, int num_docs, void *workspace,
+                          size_t workspace_bytes, const attn_bwd_options_t *opts,
+                          void *stream) {
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
         return fail(ATTN_ERR_INVALID_ARG, "null pointer");
     attn_status_t s = check_common(B, Hq, Hkv, Sq, Sk, D, scale, window_left, window_right,
                                    doc_offsets, num_docs);
     if (s != ATTN_OK) return s;
+    attn_bwd_options_t op;
+    memset(&op, 0, sizeof op);
+    if (opts) op = *opts;
+    if ((s = check_modifiers(op.softcap, op.reserved0, op.alibi_slopes, op.reserved, 4)) != ATTN_OK)
+        return s;
     for (const void *ptr : {q, k, v, o, dout, (const void *)dq, (const void *)dk, (const void *)dv,
                             (const void *)workspace})
         if (!aligned16(ptr)) return fail(ATTN_ERR_MISALIGNED, "tensors and workspace must be 16-byte aligned");
@@ -406,12 +462,18 @@ attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *
     p.num_kb = (int)num_kb;
     p.scale = scale;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    const int mod = (op.softcap > 0.0f ? 1 : 0) | (op.alibi_slopes ? 2 : 0);
+    if (op.softcap > 0.0f) {
+        p.softcap_in = (float)((double)scale / op.softcap);
+        p.softcap_out = (float)((double)op.softcap * 1.4426950408889634);
+    }
+    p.alibi_slopes = op.alibi_slopes;
 #ifdef ATTN_TRACE
     p.trace = g_trace;
     p.trace_ctas = g_trace_ctas;
 #endif
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    return D == 128 ? launch_bwd<128>(p, cs) : launch_bwd<64>(p, cs);
+    return D == 128 ? dispatch_bwd<128>(p, mod, cs) : dispatch_bwd<64>(p, mod, cs);
 }
 
 attn_status_t attn_bwd_noalloc(const void *q, const void *k, const void *v, const void *o,

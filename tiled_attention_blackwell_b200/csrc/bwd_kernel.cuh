@@ -75,7 +75,34 @@ struct BwdParams {
     float scale_log2;
     long long *trace;  // clock64 event log (trace builds only), else null
     int trace_ctas;
+    // Score modifiers (MOD != 0 kernels), as in the forward: soft-cap
+    // softcap_out * tanh(raw * softcap_in) in log2 units; ALiBi slopes per
+    // query head (device fp32 [Hq]) or null.
+    float softcap_in;   // scale / cap
+    float softcap_out;  // cap * log2(e)
+    const float *alibi_slopes;
 };
+
+// Modified score of one element in log2 units (MOD bit 0 soft-cap, bit 1
+// ALiBi at distance `dist` = i + (Sk - Sq) - j) and, in *dfac, its
+// derivative with respect to the scaled score scale * raw: 1 - tanh^2 under
+// the cap, else 1 (the ALiBi bias is constant).
+template <int MOD>
+__device__ __forceinline__ float bwd_modified(float raw, float c, float softcap_in,
+                                              float softcap_out, float slope2, float dist,
+                                              float *dfac) {
+    float x;
+    if (MOD & 1) {
+        const float t = tanh_full(raw * softcap_in);
+        x = softcap_out * t;
+        *dfac = fmaf(-t, t, 1.0f);
+    } else {
+        x = raw * c;
+        *dfac = 1.0f;
+    }
+    if (MOD & 2) x = fmaf(-slope2, fabsf(dist), x);
+    return x;
+}
 
 // Opt-in event trace of the dK/dV kernel (compile with -DATTN_TRACE), same
 // layout as the forward's: [cta][role][item][event], roles 0 = elementwise
@@ -148,7 +175,7 @@ struct DkdvSmem {
     int qb_lo, qb_hi;
 };
 
-template <int D, int NSQ>
+template <int D, int NSQ, int MOD = 0>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
     using Smem = DkdvSmem<D, NSQ>;
@@ -445,7 +472,33 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
             const bool full = sm.full[s] != 0;
             const float4 *l4 = reinterpret_cast<const float4 *>(sm.lse2[s] + h * 64);
             uint32_t pk[32];
-            if (full) {
+            if (MOD) {
+                // Modified scores: P from the transformed score; pv keeps
+                // P * d(modified)/d(scaled) for dS, pk the plain P for dV.
+                const int qb = qb_lo + it % n_qb;
+                const int hq = hkv * p.group + it / n_qb;
+                const float slope2 = (MOD & 2) ? __ldg(p.alibi_slopes + hq) * kLog2e : 0.0f;
+                const float dist0 = (float)(qb * 128 + h * 64 + p.Sk - p.Sq - key);
+                const int *rlo = sm.rlo[s] + h * 64;
+                const int *rhi = sm.rhi[s] + h * 64;
+                const float *l2 = sm.lse2[s] + h * 64;
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    float pr[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int r = e + u;
+                        float dfac;
+                        const float x = bwd_modified<MOD>(pv[r], c, p.softcap_in, p.softcap_out,
+                                                          slope2, dist0 + (float)r, &dfac);
+                        const bool in = full || (rlo[r] <= key && key <= rhi[r]);
+                        const float pe = ex2_mufu(x - l2[r]);
+                        pr[u] = in ? pe : 0.0f;
+                        pv[r] = pr[u] * dfac;
+                    }
+                    pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+                }
+            } else if (full) {
 #pragma unroll
                 for (int e = 0; e < 64; e += 4) {
                     const float4 l = l4[e >> 2];
@@ -472,6 +525,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
                     pk[(e >> 1) + 1] = pack_bf16x2(pv[e + 2], pv[e + 3]);
                 }
             }
+            __syncwarp();  // tcgen05.st is warp-collective
             tmem_st32(s_col, pk);
             tmem_wait_st();
             tc_fence_before();
@@ -500,6 +554,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
                 pk[(e >> 1) + 0] = pack_bf16x2(g0, g1);
                 pk[(e >> 1) + 1] = pack_bf16x2(g2, g3);
             }
+            __syncwarp();
             tmem_st32(dp_col, pk);
             tmem_wait_st();
             tc_fence_before();
@@ -572,7 +627,7 @@ struct DqSmem {
     int range[2];
 };
 
-template <int D, int NS>
+template <int D, int NS, int MOD = 0>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
     using Smem = DqSmem<D, NS>;
@@ -782,6 +837,7 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
         const float l2 = row_ok ? __ldg(p.lse + ri) * kLog2e : INFINITY;
         const float dval = row_ok ? p.dval[ri] : 0.0f;
         const float c = p.scale_log2;
+        const float slope2 = (MOD & 2) ? __ldg(p.alibi_slopes + hq) * kLog2e : 0.0f;
         bool ok = true;
         for (int t = 0; t < n_blocks; ++t) {
             const int j = lo_b + t;
@@ -805,7 +861,20 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
             float *pv = reinterpret_cast<float *>(sr);
             const int key0 = j * 128 + h * 64;
             const bool masked = __any_sync(0xffffffffu, key0 < kr.lo || key0 + 63 > kr.hi);
-            if (masked) {
+            if (MOD) {
+                // pv becomes P * d(modified)/d(scaled), all dS needs.
+                const float dist0 = (float)(row + p.Sk - p.Sq - key0);
+#pragma unroll
+                for (int e = 0; e < 64; ++e) {
+                    const int key = key0 + e;
+                    float dfac;
+                    const float x = bwd_modified<MOD>(pv[e], c, p.softcap_in, p.softcap_out,
+                                                      slope2, dist0 - (float)e, &dfac);
+                    const bool in = !masked || (key >= kr.lo && key <= kr.hi);
+                    const float pe = ex2_mufu(x - l2) * dfac;
+                    pv[e] = in ? pe : 0.0f;
+                }
+            } else if (masked) {
 #pragma unroll
                 for (int e = 0; e < 64; ++e) {
                     const int key = key0 + e;
@@ -822,6 +891,7 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                 const float g1 = pv[e + 1] * (__uint_as_float(dr[e + 1]) - dval);
                 pk[e / 2] = pack_bf16x2(g0, g1);
             }
+            __syncwarp();
             tmem_st32(s_col, pk);
             tmem_wait_st();
             tc_fence_before();

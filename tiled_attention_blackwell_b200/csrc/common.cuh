@@ -62,6 +62,19 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
     }
 }
 
+constexpr float kLog2eF = 1.4426950408889634f;
+
+// tanh to fp32 accuracy from the identity tanh(y) = 1 - 2 / (e^(2y) + 1):
+// one ex2 and one fast division (the MUFU tanh approximation is too coarse
+// for soft-capped logits: its error is multiplied by the cap).  |y| is
+// clamped to 20, where tanh is +-1 in fp32, so nothing overflows; a NaN
+// input stays NaN.
+__device__ __forceinline__ float tanh_full(float y) {
+    y = fminf(fmaxf(y, -20.0f), 20.0f);
+    const float e = ex2_mufu(y * 2.8853900817779268f);  // e^(2y), at most e^40
+    return 1.0f - __fdividef(2.0f, e + 1.0f);
+}
+
 // Software 2^x for the FMA pipe ("La ventaja técnica", ainvest.com page:
 // part of the exponentials as a cubic on the CUDA cores): our minimax cubic
 // (exp2_poly.cuh, fitted by fit_exp2.py) with 2^round(x) applied through the

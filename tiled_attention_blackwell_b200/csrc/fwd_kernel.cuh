@@ -81,6 +81,12 @@ struct FwdParams {
     int trace_ctas;
     unsigned long long timeout_ns;  // bound of every wait
     int debug_withhold_kv;          // testing: CTA 0 skips its first K copy
+    // Score modifiers (MOD != 0 kernels): soft-cap s <- cap tanh(s / cap)
+    // as softcap_out * tanh(raw * softcap_in) in log2 units; ALiBi slope per
+    // query head (device fp32 [Hq]) or null.
+    float softcap_in;   // scale / cap
+    float softcap_out;  // cap * log2(e)
+    const float *alibi_slopes;
 };
 
 // Opt-in event trace (compile with -DATTN_TRACE): lane 0 of warps 0 and 4
@@ -157,7 +163,19 @@ __device__ __forceinline__ float exp_pack_half(const float *s, float c, float ne
     return (sum0 + sum1) + (sum2 + sum3);
 }
 
-template <int D, int NS, int EXP_MODE>
+// Score modifier, in log2 units: MOD bit 0 soft-cap, bit 1 ALiBi.  `raw` is
+// <q_i, k_j>; `dist` is i + (Sk - Sq) - j as a float.
+template <int MOD>
+__device__ __forceinline__ float modified_score(float raw, float c, float softcap_in,
+                                                float softcap_out, float slope2, float dist) {
+    float x;
+    if (MOD & 1) x = softcap_out * tanh_full(raw * softcap_in);
+    else x = raw * c;
+    if (MOD & 2) x = fmaf(-slope2, fabsf(dist), x);
+    return x;
+}
+
+template <int D, int NS, int EXP_MODE, int MOD = 0>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ FwdParams p) {
     using Smem = FwdSmem<D, NS>;
@@ -444,6 +462,11 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         const int hi_b = i == 0 ? hi0 : hi1;
         const float c = p.scale_log2;
         const float tau = p.rescale_threshold;
+        // With a modifier the scores are transformed into log2 units before
+        // the max, so the exponent step multiplies by 1 instead of c.
+        const float c_exp = MOD ? 1.0f : c;
+        const float slope2 = (MOD & 2) ? __ldg(p.alibi_slopes + hq) * kLog2eF : 0.0f;
+        const float diag_f = (float)(row + p.Sk - p.Sq);
         float m_run = -INFINITY;
         float l_run = 0.0f;
         bool ok = true;
@@ -470,6 +493,13 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             float *s = reinterpret_cast<float *>(sr);
 
             const int key0 = j * kBlockN;
+            const float dist0 = diag_f - (float)key0;  // distance to key0 of this block
+            if (MOD) {
+#pragma unroll
+                for (int e = 0; e < kBlockN / 2; ++e)
+                    s[e] = modified_score<MOD>(s[e], c, p.softcap_in, p.softcap_out, slope2,
+                                               dist0 - (float)e);
+            }
             const bool need_mask = key0 < kr.lo || key0 + kBlockN - 1 > kr.hi;
             const bool masked = __any_sync(0xffffffffu, need_mask);
             if (masked) {
@@ -491,6 +521,12 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             tmem_wait_ld();
             reg_fence32(sr + 64);
             reg_fence32(sr + 96);
+            if (MOD) {
+#pragma unroll
+                for (int e = kBlockN / 2; e < kBlockN; ++e)
+                    s[e] = modified_score<MOD>(s[e], c, p.softcap_in, p.softcap_out, slope2,
+                                               dist0 - (float)e);
+            }
             if (masked) {
 #pragma unroll
                 for (int e = kBlockN / 2; e < kBlockN; ++e) {
@@ -504,7 +540,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], s[e + u], s[e + 4 + u]);
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 2);
             const float row_max = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
-            const float m_cand = row_max * c;
+            const float m_cand = MOD ? row_max : row_max * c;
             float alpha = 1.0f;
             if (m_cand > m_run + tau) {
                 alpha = ex2_mufu(m_run - m_cand);
@@ -543,14 +579,15 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             // this warp computes keys [64, 128).  Masked blocks (-inf scores)
             // use MUFU only: ex2(-inf) = 0 exactly.
             uint32_t pk[kBlockN / 2];
-            l_run += masked ? exp_pack_half<0>(s, c, neg_m, pk)
-                            : exp_pack_half<EXP_MODE>(s, c, neg_m, pk);
+            if (MOD) __syncwarp();  // converged before the warp-collective TMEM store
+            l_run += masked ? exp_pack_half<0>(s, c_exp, neg_m, pk)
+                            : exp_pack_half<EXP_MODE>(s, c_exp, neg_m, pk);
             tmem_st32(s_tmem + 0, pk + 0);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_half[i]);
-            l_run += masked ? exp_pack_half<0>(s + 64, c, neg_m, pk + 32)
-                            : exp_pack_half<EXP_MODE>(s + 64, c, neg_m, pk + 32);
+            l_run += masked ? exp_pack_half<0>(s + 64, c_exp, neg_m, pk + 32)
+                            : exp_pack_half<EXP_MODE>(s + 64, c_exp, neg_m, pk + 32);
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
             tmem_st32(s_tmem + 32, pk + 32);
             tmem_wait_st();
