@@ -54,6 +54,11 @@ def _load():
                 fn = getattr(lib, name)
                 fn.restype = ctypes.c_int
                 fn.argtypes = [ctypes.c_void_p] * 9 + dims
+            lib.oracle_attn_fwd_e4m3.restype = ctypes.c_int
+            lib.oracle_attn_fwd_e4m3.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_double] * 3 + \
+                [ctypes.c_void_p] * 2 + dims[:-2] + [ctypes.c_void_p, ctypes.c_int64]
+            lib.oracle_e4m3_to_double.restype = ctypes.c_double
+            lib.oracle_e4m3_to_double.argtypes = [ctypes.c_int]
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -142,6 +147,55 @@ def attn_fwd(q, k, v, *, scale, causal=False, window=None, doc_offsets=None,
             float(scale), causal_i, wl, wr, _ptr(offs), nd, cap, _ptr(slopes), _ptr(rows_a), n)
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd failed with code {rc}")
+    return o, lse
+
+
+def e4m3_to_float(code: int) -> float:
+    """The value of one fp8 e4m3 code (0..255), decoded by the oracle."""
+    return float(_load().oracle_e4m3_to_double(int(code)))
+
+
+def _as_codes(x):
+    """fp8 e4m3 codes as a contiguous uint8 array (from a torch float8_e4m3fn
+    or uint8 tensor, or a numpy uint8 array)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype != torch.uint8:
+                x = x.view(torch.uint8)
+            return x.numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint8:
+        raise TypeError("fp8 inputs must be e4m3 codes (uint8)")
+    return x
+
+
+def attn_fwd_fp8(q, k, v, *, q_descale, k_descale, v_descale, scale, causal=False,
+                 window=None, doc_offsets=None, rows=None):
+    """Exact attention in fp64 of fp8 e4m3 inputs: Q = q_descale * decode(q),
+    likewise K and V.  Shapes and return values as attn_fwd."""
+    lib = _load()
+    qa, ka, va = _as_codes(q), _as_codes(k), _as_codes(v)
+    B, Hq, Hkv, Sq, Sk, D = _shapes(qa, ka)
+    causal_i, wl, wr, offs, nd = _mask_args(causal, window, doc_offsets)
+    if rows is None:
+        o = np.zeros((B, Sq, Hq, D), dtype=np.float64)
+        lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+        rows_a, n = None, 0
+    else:
+        rows_a = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+        n = rows_a.shape[0]
+        o = np.zeros((n, D), dtype=np.float64)
+        lse = np.zeros((n,), dtype=np.float64)
+    rc = lib.oracle_attn_fwd_e4m3(_ptr(qa), _ptr(ka), _ptr(va), float(q_descale),
+                                  float(k_descale), float(v_descale), _ptr(o), _ptr(lse),
+                                  B, Hq, Hkv, Sq, Sk, D, float(scale), causal_i, wl, wr,
+                                  _ptr(offs), nd, _ptr(rows_a), n)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_e4m3 failed with code {rc}")
     return o, lse
 
 

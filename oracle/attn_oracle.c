@@ -39,8 +39,9 @@
  * Parity pins (tests, CPU only): closed forms (equal logits -> mean of V,
  * one dominant logit -> that V row, constant V -> rows of P sum to one,
  * causal row 0), library softmax / logsumexp on dense masked scores, mask
- * and GQA invariants, finite differences for the backward.  Nothing here is
- * "parity unpinned".
+ * and GQA invariants, finite differences for the backward; the e4m3 decoder
+ * against torch's float8_e4m3fn conversion for all 256 codes.  Nothing here
+ * is "parity unpinned".
  *
  * Layouts (row-major, contiguous):
  *   q, o, dq, do : [B, Sq, Hq,  D]
@@ -383,6 +384,57 @@ int oracle_attn_fwd_f64(const double *q, const double *k, const double *v,
                         const int64_t *rows, int64_t n_rows) {
     ORACLE_SHAPE;
     return attn_fwd_core(&s, q, k, v, 0, o, lse, rows, n_rows);
+}
+
+/* ------------------------------------------------------- fp8 (e4m3) inputs
+ * The low-precision forward ("Hardware-Aware FP4 FlashAttention-4", the
+ * "HAO" FP8 path that "Precisión" compares against): Q, K, V arrive as fp8
+ * e4m3 codes with one fp32 dequantisation factor per tensor.  The oracle
+ * decodes every code exactly, multiplies by its factor in fp64 and computes
+ * exact attention of those values -- the result the fp8 path approximates.
+ *
+ * e4m3 (the variant without infinities): bit 7 sign, bits 6-3 exponent with
+ * bias 7, bits 2-0 mantissa.  Exponent field 0 encodes the subnormals
+ * m/8 * 2^-6; the code with all exponent and mantissa bits set is NaN; the
+ * largest finite magnitude is 1.75 * 2^8 = 448. */
+static double e4m3_to_double(uint8_t c) {
+    const int e = (c >> 3) & 15, m = c & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m / 8.0, -6);
+    else mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (c & 0x80) ? -mag : mag;
+}
+
+double oracle_e4m3_to_double(int code) { return e4m3_to_double((uint8_t)code); }
+
+static double *decode_e4m3(const uint8_t *x, size_t n, double mul) {
+    double *d = (double *)malloc((n ? n : 1) * sizeof(double));
+    if (!d) return NULL;
+    for (size_t t = 0; t < n; ++t) d[t] = e4m3_to_double(x[t]) * mul;
+    return d;
+}
+
+int oracle_attn_fwd_e4m3(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                         double q_descale, double k_descale, double v_descale,
+                         double *o, double *lse, int B, int Hq, int Hkv, int Sq,
+                         int Sk, int D, double scale, int causal, int window_left,
+                         int window_right, const int *doc_offsets, int num_docs,
+                         const int64_t *rows, int64_t n_rows) {
+    const double softcap = 0.0;
+    const double *alibi_slopes = NULL;
+    ORACLE_SHAPE;
+    if (!shape_ok(&s)) return -1;
+    const size_t nq = (size_t)B * Sq * Hq * D, nkv = (size_t)B * Sk * Hkv * D;
+    double *qd = decode_e4m3(q, nq, q_descale);
+    double *kd = decode_e4m3(k, nkv, k_descale);
+    double *vd = decode_e4m3(v, nkv, v_descale);
+    int status = -2;
+    if (qd && kd && vd) status = attn_fwd_core(&s, qd, kd, vd, 0, o, lse, rows, n_rows);
+    free(qd);
+    free(kd);
+    free(vd);
+    return status;
 }
 
 int oracle_attn_bwd_bf16(const uint16_t *q, const uint16_t *k, const uint16_t *v,

@@ -404,3 +404,83 @@ def test_backward_with_modifiers_matches_central_differences(mods):
             fd[idx] = (_loss(**{**args, name: xp}, dout=dout, **kw) -
                        _loss(**{**args, name: xm}, dout=dout, **kw)) / (2 * h)
         np.testing.assert_allclose(g, fd, atol=2e-8, rtol=1e-6, err_msg=name)
+
+
+# ------------------------------------------------------------- fp8 (e4m3) inputs
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    """All 256 e4m3 codes against torch's float8_e4m3fn conversion."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_to_float(c) for c in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    np.testing.assert_array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+
+
+@pytest.mark.parametrize("code,value", [(0x38, 1.0), (0xB8, -1.0), (0x7E, 448.0),
+                                        (0x08, 2.0 ** -6), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9),
+                                        (0x3C, 1.5), (0x00, 0.0)])
+def test_e4m3_known_codes(code, value):
+    # The format's own corner values: one, the largest finite value, the
+    # smallest normal and subnormal, a mantissa step.
+    assert oracle.e4m3_to_float(code) == value
+
+
+def quantize_e4m3(x, amax_target=448.0):
+    """Per-tensor e4m3 quantisation with torch: codes and the descale factor."""
+    descale = float(x.abs().max()) / amax_target
+    return (x / descale).to(torch.float8_e4m3fn), descale
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_forward_is_exact_attention_of_the_dequantized_inputs(causal):
+    g = torch.Generator().manual_seed(21)
+    B, S, Hq, Hkv, D = 2, 37, 4, 2, 16
+    q8, qd = quantize_e4m3(torch.randn(B, S, Hq, D, generator=g) * 2)
+    k8, kd = quantize_e4m3(torch.randn(B, S, Hkv, D, generator=g))
+    v8, vd = quantize_e4m3(torch.randn(B, S, Hkv, D, generator=g) * 3)
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, q_descale=qd, k_descale=kd, v_descale=vd,
+                                 scale=0.3, causal=causal)
+    # independent dequantisation (torch's decode), then the dense scipy reference
+    deq = [x.to(torch.float64).numpy() * d for x, d in ((q8, qd), (k8, kd), (v8, vd))]
+    o_ref, lse_ref = dense_reference(*deq, 0.3, dense_mask(S, S, causal=causal))
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+
+
+def test_fp8_descales_act_on_their_own_tensor():
+    g = torch.Generator().manual_seed(22)
+    q8, _ = quantize_e4m3(torch.randn(1, 20, 2, 8, generator=g))
+    k8, _ = quantize_e4m3(torch.randn(1, 20, 2, 8, generator=g))
+    v8, _ = quantize_e4m3(torch.randn(1, 20, 2, 8, generator=g))
+    base = oracle.attn_fwd_fp8(q8, k8, v8, q_descale=0.01, k_descale=0.02, v_descale=0.03,
+                               scale=0.5)
+    # V's factor scales O only; Q's and K's enter the scores as a product.
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, q_descale=0.01, k_descale=0.02, v_descale=0.09,
+                                 scale=0.5)
+    np.testing.assert_allclose(o, 3 * base[0], rtol=1e-13)
+    np.testing.assert_allclose(lse, base[1], rtol=1e-13)
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, q_descale=0.04, k_descale=0.005, v_descale=0.03,
+                                 scale=0.5)
+    np.testing.assert_allclose(o, base[0], rtol=1e-12)
+    np.testing.assert_allclose(lse, base[1], rtol=1e-12)
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, q_descale=0.02, k_descale=0.02, v_descale=0.03,
+                                 scale=0.5)
+    o2, lse2 = oracle.attn_fwd_fp8(q8, k8, v8, q_descale=0.01, k_descale=0.02, v_descale=0.03,
+                                   scale=1.0)
+    np.testing.assert_allclose(o, o2, rtol=1e-12)
+    np.testing.assert_allclose(lse, lse2, rtol=1e-12)
+
+
+def test_fp8_row_subset_matches_full():
+    g = torch.Generator().manual_seed(23)
+    q8, qd = quantize_e4m3(torch.randn(1, 60, 2, 8, generator=g))
+    k8, kd = quantize_e4m3(torch.randn(1, 60, 1, 8, generator=g))
+    v8, vd = quantize_e4m3(torch.randn(1, 60, 1, 8, generator=g))
+    kw = dict(q_descale=qd, k_descale=kd, v_descale=vd, scale=0.4, causal=True)
+    o, lse = oracle.attn_fwd_fp8(q8, k8, v8, **kw)
+    rows = np.array([[0, 1, 59], [0, 0, 3]])
+    o_r, lse_r = oracle.attn_fwd_fp8(q8, k8, v8, rows=rows, **kw)
+    for n, (b, h, i) in enumerate(rows):
+        np.testing.assert_array_equal(o_r[n], o[b, i, h])
+        assert lse_r[n] == lse[b, h, i]
