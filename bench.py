@@ -228,10 +228,16 @@ def oracle_sample(w, inputs, n_rows: int, seed: int = 0):
                      rng.integers(0, w.S, n_rows)], axis=1).astype(np.int64)
     keys = allowed_keys_per_row(w, inputs["doc_offsets"])
     flops = float((4.0 * w.D * keys[rows[:, 2]]).sum())
+    window = None if w.window == (-1, -1) else w.window
     t0 = time.perf_counter()
-    oracle.attn_fwd(inputs["q"], inputs["k"], inputs["v"], scale=w.scale, causal=w.causal,
-                    window=None if w.window == (-1, -1) else w.window,
-                    doc_offsets=inputs["doc_offsets"], rows=rows)
+    if w.dtype == "fp8":
+        oracle.attn_fwd_fp8(inputs["q"], inputs["k"], inputs["v"],
+                            q_descale=inputs["q_descale"], k_descale=inputs["k_descale"],
+                            v_descale=inputs["v_descale"], scale=w.scale, causal=w.causal,
+                            window=window, doc_offsets=inputs["doc_offsets"], rows=rows)
+    else:
+        oracle.attn_fwd(inputs["q"], inputs["k"], inputs["v"], scale=w.scale, causal=w.causal,
+                        window=window, doc_offsets=inputs["doc_offsets"], rows=rows)
     return time.perf_counter() - t0, flops, oracle.num_threads()
 
 
@@ -254,7 +260,9 @@ def workload_config(w, doc_offsets):
            "scale": w.scale}
     if doc_offsets is not None:
         cfg["num_docs"] = int(len(doc_offsets) - 1)
-    io_bytes = 2 * (2 * w.B * w.S * w.Hq * w.D + 2 * w.B * w.S * w.Hkv * w.D) + 4 * w.B * w.Hq * w.S
+    eb = 1 if w.dtype == "fp8" else 2  # bytes per Q/K/V element; O is bf16
+    io_bytes = (eb * (w.B * w.S * w.Hq * w.D + 2 * w.B * w.S * w.Hkv * w.D)
+                + 2 * w.B * w.S * w.Hq * w.D + 4 * w.B * w.Hq * w.S)
     cfg["io_bytes"] = io_bytes
     cfg["l2"] = (f"inputs+outputs {io_bytes / 2**20:.0f} MiB > L2 126 MiB; no flush"
                  if io_bytes > L2_BYTES else "L2 flushed between steps")
@@ -280,7 +288,8 @@ def run_ours(args):
     host = {n: inp[n].pin_memory() for n in ("q", "k", "v")}
     dev = {n: host[n].to(device) for n in host}
     docs = None if docs_np is None else torch.as_tensor(docs_np, dtype=torch.int32, device=device)
-    o = torch.empty_like(dev["q"])
+    fp8 = w.dtype == "fp8"
+    o = torch.empty(dev["q"].shape, dtype=torch.bfloat16, device=device)
     lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=device)
     window = None if w.window == (-1, -1) else w.window
     if w.backward:
@@ -317,6 +326,11 @@ def run_ours(args):
             attn.attn_bwd(dev["q"], dev["k"], dev["v"], dev["o"], dev["lse"], dev["dout"], g_dq,
                           g_dk, g_dv, ws, scale=w.scale, causal=w.causal, window=window,
                           doc_offsets=docs, stream=stream)
+        elif fp8:
+            attn.attn_fwd_fp8(dev["q"], dev["k"], dev["v"], o, lse, q_descale=inp["q_descale"],
+                              k_descale=inp["k_descale"], v_descale=inp["v_descale"],
+                              scale=w.scale, causal=w.causal, window=window, doc_offsets=docs,
+                              options=opts, stream=stream)
         else:
             attn.attn_fwd(dev["q"], dev["k"], dev["v"], o, lse, scale=w.scale, causal=w.causal,
                           window=window, doc_offsets=docs, options=opts, stream=stream)
@@ -380,22 +394,31 @@ def run_ours(args):
 
     peaks, peak_kind = read_peaks()
     achieved = flops / (launch_avg_ms / 1e3) / 1e12
-    peak = float(peaks["bf16_tflops"])
-    metric = METRIC if not w.backward else \
-        f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()})"
+    # fp8 contractions: the measured bf16 peak times the nominal dense
+    # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s).
+    peak_mult = 2.0 if fp8 else 1.0
+    peak = float(peaks["bf16_tflops"]) * peak_mult
+    if w.backward:
+        metric = f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()})"
+    elif fp8:
+        metric = f"attention fwd TFLOP/s and % of B200 FP8 tensor peak ({w.describe()})"
+    else:
+        metric = METRIC
     result = {
         "metric": metric, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8e4m3" if fp8 else "bf16",
         "data": "synthetic", "config": cfg,
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(w.name),
-                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
-                     if peak_kind == "measured" else "fallback 1590 TFLOP/s",
-                     "frac_of_sustained": round(achieved / float(
-                         peaks.get("bf16_tflops_sustained", peak)), 4),
+                     "peak_source": (f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
+                                     if peak_kind == "measured" else "fallback 1590 TFLOP/s")
+                     + (" x 2 (nominal fp8/bf16 dense ratio)" if fp8 else ""),
+                     "frac_of_sustained": round(achieved / (peak_mult * float(
+                         peaks.get("bf16_tflops_sustained", peak))), 4),
                      "flops_per_launch": flops, "launch_ms": round(launch_avg_ms, 4),
                      "kernel": "attn_bwd (preprocess, dK/dV, dQ kernels per step)"
                      if w.backward else "attn_fwd_kernel"},

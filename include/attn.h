@@ -142,6 +142,27 @@ ATTN_API attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, 
                           const attn_fwd_options_t *opts, void *stream);
 
 /*
+ * Low-precision forward ("Hardware-Aware FP4 FlashAttention-4", "Precisión":
+ * the FP8 path that Direct-P is measured against).  q, k, v hold fp8 e4m3
+ * codes (1 byte each, same [B,S,H,D] layouts, 16-byte aligned); the values
+ * they stand for are q_descale * q, k_descale * k, v_descale * v (each factor
+ * > 0 and finite).  Both products QK^T and PV run on the tensor cores in
+ * e4m3 with fp32 accumulation; the probabilities P are rounded to e4m3
+ * after scaling by 2^(8 - rescale_threshold), which keeps them inside e4m3's
+ * range (the row sum l is taken from the unrounded values, as in attn_fwd).
+ * O is bf16 and LSE fp32 as in attn_fwd, for the dequantized inputs.
+ * D must be 128; rescale_threshold must be <= 8 (smaller values keep more
+ * precision for small probabilities at the cost of more rescales); score
+ * modifiers are not supported (ATTN_ERR_UNSUPPORTED).  opts may be NULL.
+ */
+ATTN_API attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v,
+                                    float q_descale, float k_descale, float v_descale,
+                                    void *o, float *lse, int B, int Hq, int Hkv, int Sq,
+                                    int Sk, int D, float scale, int causal, int window_left,
+                                    int window_right, const int *doc_offsets, int num_docs,
+                                    const attn_fwd_options_t *opts, void *stream);
+
+/*
  * Backward ("Hardware-Aware FP4 FlashAttention-4", "Causal Backward
  * Cuantizado": gradients from the saved LSE, probabilities rebuilt rather
  * than stored).  For L with dO = dL/dO:

@@ -197,3 +197,37 @@ def test_binding_refuses_cpu_tensors(L):
     lse = torch.zeros(1, 1, 4)
     with pytest.raises(TypeError):
         attn.attn_fwd(q, q, q, q, lse, scale=0.1)
+
+
+def call_fp8(L, **kw):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, qd=0.01, kd=0.02, vd=0.03, B=1, Hq=2, Hkv=2, Sq=16,
+             Sk=16, D=128, scale=0.1, causal=0, wl=-1, wr=-1, docs=None, nd=0, opts=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return L.attn_fwd_fp8(vp(a["q"]), vp(a["k"]), vp(a["v"]), a["qd"], a["kd"], a["vd"],
+                          vp(a["o"]), vp(a["lse"]), a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Sk"],
+                          a["D"], a["scale"], a["causal"], a["wl"], a["wr"],
+                          vp(a["docs"]) if a["docs"] else None, a["nd"],
+                          None if a["opts"] is None else ctypes.byref(a["opts"]), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=64), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(qd=0.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(kd=-1.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(vd=float("inf")), attn.ATTN_ERR_INVALID_ARG),
+    (dict(vd=float("nan")), attn.ATTN_ERR_INVALID_ARG),
+    (dict(q=P + 4), attn.ATTN_ERR_MISALIGNED),
+    (dict(q=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), attn.ATTN_ERR_INVALID_ARG),
+    (dict(opts=attn.default_options(softcap=5.0)), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(opts=attn.default_options(alibi_slopes=P)), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(opts=attn.default_options(rescale_threshold=9.0)), attn.ATTN_ERR_INVALID_ARG),
+])
+def test_fp8_invalid_arguments_rejected_before_launch(L, kw, status):
+    assert call_fp8(L, **kw) == status
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
+def test_valid_fp8_call_without_gpu_reports_cuda_error(L):
+    assert call_fp8(L) == attn.ATTN_ERR_CUDA

@@ -25,7 +25,7 @@ ATTN_ERR_LAUNCH = 4
 ATTN_ERR_DEVICE_TIMEOUT = 5
 ATTN_ERR_CUDA = 6
 
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_default_options", "attn_bwd",
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_fp8", "attn_fwd_default_options", "attn_bwd",
             "attn_bwd_ex", "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_status",
             "attn_status_string", "attn_last_error_detail", "attn_abi_version")
 
@@ -71,6 +71,11 @@ def lib():
             L.attn_fwd.argtypes = _FWD_ARGS + [ctypes.c_void_p]
             L.attn_fwd_ex.restype = ctypes.c_int
             L.attn_fwd_ex.argtypes = _FWD_ARGS + [ctypes.POINTER(FwdOptions), ctypes.c_void_p]
+            L.attn_fwd_fp8.restype = ctypes.c_int
+            L.attn_fwd_fp8.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_float] * 3 + \
+                [ctypes.c_void_p] * 2 + [ctypes.c_int] * 6 + [ctypes.c_float] + \
+                [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(FwdOptions),
+                                      ctypes.c_void_p]
             L.attn_fwd_default_options.restype = None
             L.attn_fwd_default_options.argtypes = [ctypes.POINTER(FwdOptions)]
             L.attn_get_device_status.restype = ctypes.c_int
@@ -196,6 +201,53 @@ def attention(q, k, v, *, scale=None, causal=False, window=None, doc_offsets=Non
     attn_fwd(q, k, v, o, lse, scale=scale, causal=causal, window=window,
              doc_offsets=doc_offsets, options=options, stream=stream, softcap=softcap,
              alibi_slopes=alibi_slopes)
+    return o, lse
+
+
+def attn_fwd_fp8(q, k, v, o, lse, *, q_descale, k_descale, v_descale, scale, causal=False,
+                 window=None, doc_offsets=None, options=None, stream=None):
+    """Enqueue the fp8 forward: q, k, v contiguous CUDA tensors of e4m3 codes
+    (torch.float8_e4m3fn or uint8) standing for descale * code; o bf16, lse
+    fp32 as in attn_fwd."""
+    fp8_types = (torch.float8_e4m3fn, torch.uint8)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype not in fp8_types or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA float8_e4m3fn tensor")
+    for name, t, dt in (("o", o, torch.bfloat16), ("lse", lse, torch.float32)):
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA {dt} tensor")
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    if doc_offsets is not None:
+        if doc_offsets.dtype != torch.int32 or not doc_offsets.is_cuda:
+            raise TypeError("doc_offsets must be a CUDA int32 tensor")
+        docs_ptr, nd = _ptr(doc_offsets), doc_offsets.numel() - 1
+    else:
+        docs_ptr, nd = None, 0
+    st = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), float(q_descale), float(k_descale),
+                            float(v_descale), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
+                            float(scale), int(bool(causal)), wl, wr, docs_ptr, nd,
+                            None if options is None else ctypes.byref(options),
+                            _stream_handle(stream))
+    _check(st, "attn_fwd_fp8")
+
+
+def attention_fp8(q, k, v, *, q_descale, k_descale, v_descale, scale=None, causal=False,
+                  window=None, doc_offsets=None, options=None, stream=None):
+    """Allocate O (bf16) and LSE with torch and run the fp8 forward."""
+    B, Sq, Hq, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o = torch.empty((B, Sq, Hq, D), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if doc_offsets is not None and not torch.is_tensor(doc_offsets):
+        doc_offsets = torch.as_tensor(doc_offsets, dtype=torch.int32)
+    if doc_offsets is not None and not doc_offsets.is_cuda:
+        doc_offsets = doc_offsets.to(q.device)
+    attn_fwd_fp8(q, k, v, o, lse, q_descale=q_descale, k_descale=k_descale,
+                 v_descale=v_descale, scale=scale, causal=causal, window=window,
+                 doc_offsets=doc_offsets, options=options, stream=stream)
     return o, lse
 
 

@@ -86,15 +86,20 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor [B][S][H][D] as a 4-D map (D, S, H, B), box (64, 128, 1, 1),
 // 128-byte swizzle, zero fill out of bounds.
-attn_status_t make_map(CUtensorMap *map, const void *base, int B, int S, int H, int D) {
+// 4-D map of a [B][S][H][D] tensor with `eb`-byte elements; the box is one
+// 128-byte row chunk (128 / eb elements) by kBlockM positions.
+attn_status_t make_map(CUtensorMap *map, const void *base, int B, int S, int H, int D,
+                       int eb = 2) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)H * D * 2, (cuuint64_t)D * 2,
-                                   (cuuint64_t)S * H * D * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)tab::kBlockM, 1, 1};
+    const cuuint64_t strides[3] = {(cuuint64_t)H * D * eb, (cuuint64_t)D * eb,
+                                   (cuuint64_t)S * H * D * eb};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / eb), (cuuint32_t)tab::kBlockM, 1, 1};
     const cuuint32_t estride[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+    const CUtensorMapDataType dtype =
+        eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = fn(map, dtype, 4, const_cast<void *>(base), dims,
                     strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -104,12 +109,12 @@ attn_status_t make_map(CUtensorMap *map, const void *base, int B, int S, int H, 
 
 // --------------------------------------------------------------- launching
 
-template <int D, int NS, int EXP, int MOD = 0>
+template <int D, int NS, int EXP, int MOD = 0, int FP8 = 0>
 attn_status_t launch_fwd(const tab::FwdParams &p, int grid, cudaStream_t stream) {
-    using Smem = tab::FwdSmem<D, NS>;
+    using Smem = tab::FwdSmem<D, NS, FP8 ? 1 : 2>;
     constexpr size_t smem = sizeof(Smem) + 1024;
     static_assert(smem <= 232448, "shared memory budget");
-    auto kernel = tab::attn_fwd_kernel<D, NS, EXP, MOD>;
+    auto kernel = tab::attn_fwd_kernel<D, NS, EXP, MOD, FP8>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     int dev = 0;
@@ -146,6 +151,7 @@ constexpr int kStagesD128 = 4;
 // key/value head the group covers 32 query heads.
 constexpr int kFwdHeadGroup = 8;
 constexpr int kStagesD64 = 8;
+constexpr int kStagesFp8 = 8;  // fp8 K/V tiles are 16 KB at D = 128
 
 template <int D, int NS>
 attn_status_t dispatch_exp(const tab::FwdParams &p, int grid, int exp_mode, int mod,
@@ -161,6 +167,14 @@ attn_status_t dispatch_exp(const tab::FwdParams &p, int grid, int exp_mode, int 
         case 0: return launch_fwd<D, NS, 0>(p, grid, s);
         case 1: return launch_fwd<D, NS, 1>(p, grid, s);
         default: return launch_fwd<D, NS, 2>(p, grid, s);
+    }
+}
+
+attn_status_t dispatch_fp8(const tab::FwdParams &p, int grid, int exp_mode, cudaStream_t s) {
+    switch (exp_mode) {
+        case 0: return launch_fwd<128, kStagesFp8, 0, 0, 1>(p, grid, s);
+        case 1: return launch_fwd<128, kStagesFp8, 1, 0, 1>(p, grid, s);
+        default: return launch_fwd<128, kStagesFp8, 2, 0, 1>(p, grid, s);
     }
 }
 
@@ -291,11 +305,13 @@ void attn_fwd_default_options(attn_fwd_options_t *opts) {
     opts->exp2_mode = 1;
 }
 
-attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
-                          int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
-                          int causal, int window_left, int window_right,
-                          const int *doc_offsets, int num_docs,
-                          const attn_fwd_options_t *opts, void *stream) {
+// The forward of both entry points.  fp8: Q, K, V are e4m3 codes with the
+// given dequantisation factors (ignored for bf16).
+static attn_status_t fwd_impl(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                       int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                       int window_left, int window_right, const int *doc_offsets,
+                       int num_docs, const attn_fwd_options_t *opts, bool fp8,
+                       float q_descale, float k_descale, float v_descale, void *stream) {
     attn_fwd_options_t op;
     attn_fwd_default_options(&op);
     if (opts) op = *opts;
@@ -324,6 +340,16 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
         attn_status_t c = check_modifiers(op.softcap, op.reserved0, op.alibi_slopes, op.reserved, 4);
         if (c != ATTN_OK) return c;
     }
+    if (fp8) {
+        if (D != 128) return fail(ATTN_ERR_UNSUPPORTED, "the fp8 forward supports D = 128 only");
+        for (float d : {q_descale, k_descale, v_descale})
+            if (!(d > 0.0f) || !std::isfinite(d))
+                return fail(ATTN_ERR_INVALID_ARG, "descale factors must be > 0 and finite");
+        if (op.softcap != 0.0f || op.alibi_slopes)
+            return fail(ATTN_ERR_UNSUPPORTED, "the fp8 forward has no score modifiers");
+        if (op.rescale_threshold > 8.0f)
+            return fail(ATTN_ERR_INVALID_ARG, "the fp8 forward needs rescale_threshold <= 8");
+    }
     const long long num_qblocks = (Sq + 2LL * tab::kBlockM - 1) / (2LL * tab::kBlockM);
     const long long grid = num_qblocks * Hq * B;
     if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
@@ -335,9 +361,10 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
 
     tab::FwdParams p;
     memset(&p, 0, sizeof p);
-    if ((s = make_map(&p.tm_q, q, B, Sq, Hq, D)) != ATTN_OK) return s;
-    if ((s = make_map(&p.tm_k, k, B, Sk, Hkv, D)) != ATTN_OK) return s;
-    if ((s = make_map(&p.tm_v, v, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    const int eb = fp8 ? 1 : 2;
+    if ((s = make_map(&p.tm_q, q, B, Sq, Hq, D, eb)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_k, k, B, Sk, Hkv, D, eb)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_v, v, B, Sk, Hkv, D, eb)) != ATTN_OK) return s;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     p.doc_offsets = doc_offsets;
@@ -355,6 +382,13 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
     p.num_qblocks = (int)num_qblocks;
     p.head_group = std::min(B * Hq, kFwdHeadGroup * (Hq / Hkv));
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    if (fp8) {
+        p.scale_log2 = (float)((double)scale * q_descale * k_descale * 1.4426950408889634);
+        p.v_descale = v_descale;
+        // P = 2^(x - m + 8 - tau) <= 2^8: e4m3 reaches 448, and the small
+        // probabilities keep as many normal-range bits as tau allows.
+        p.p_offset = 8.0f - op.rescale_threshold;
+    }
     p.rescale_threshold = op.rescale_threshold;
     p.timeout_ns = op.wait_timeout_us > 0 ? 1000ull * (unsigned long long)op.wait_timeout_us
                                           : tab::kWaitTimeoutNs;
@@ -371,8 +405,28 @@ attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, 
 #endif
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (fp8) return dispatch_fp8(p, (int)grid, op.exp2_mode, cs);
     if (D == 128) return dispatch_exp<128, kStagesD128>(p, (int)grid, op.exp2_mode, mod, cs);
     return dispatch_exp<64, kStagesD64>(p, (int)grid, op.exp2_mode, mod, cs);
+}
+
+attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
+                          int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                          int causal, int window_left, int window_right,
+                          const int *doc_offsets, int num_docs,
+                          const attn_fwd_options_t *opts, void *stream) {
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, window_left,
+                    window_right, doc_offsets, num_docs, opts, false, 1.0f, 1.0f, 1.0f, stream);
+}
+
+attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v, float q_descale,
+                           float k_descale, float v_descale, void *o, float *lse, int B,
+                           int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                           int window_left, int window_right, const int *doc_offsets,
+                           int num_docs, const attn_fwd_options_t *opts, void *stream) {
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, window_left,
+                    window_right, doc_offsets, num_docs, opts, true, q_descale, k_descale,
+                    v_descale, stream);
 }
 
 attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse,

@@ -87,6 +87,10 @@ struct FwdParams {
     float softcap_in;   // scale / cap
     float softcap_out;  // cap * log2(e)
     const float *alibi_slopes;
+    // fp8 kernels: V's dequantisation factor (Q's and K's are folded into
+    // scale_log2) and the exponent offset that puts P into (0, 2^8].
+    float v_descale;
+    float p_offset;
 };
 
 // Opt-in event trace (compile with -DATTN_TRACE): lane 0 of warps 0 and 4
@@ -107,12 +111,15 @@ constexpr int kTraceEvents = 8;
     } while (0)
 #endif
 
-template <int D, int NS>
+// EB: bytes per element of Q, K, V (2 = bf16, 1 = fp8 e4m3).  A tile row of
+// D elements is D*EB bytes, stored as chunks of 128-byte rows.
+template <int D, int NS, int EB = 2>
 struct FwdSmem {
-    static constexpr int kChunks = D / 64;
-    static constexpr int kChunkElems = kBlockM * 64;  // 16 KB
-    __nv_bfloat16 q[2][kChunks][kChunkElems];
-    __nv_bfloat16 kv[NS][kChunks][kChunkElems];
+    static constexpr int kChunkBytes = kBlockM * 128;  // 16 KB: 128 rows x 128 bytes
+    static constexpr int kChunks = D * EB / 128;
+    static constexpr int kChunkElems = 128 / EB;       // elements per 128-byte row
+    uint8_t q[2][kChunks][kChunkBytes];
+    uint8_t kv[NS][kChunks][kChunkBytes];
     uint64_t q_full;
     uint64_t kv_full[NS];
     uint64_t kv_empty[NS];
@@ -163,6 +170,35 @@ __device__ __forceinline__ float exp_pack_half(const float *s, float c, float ne
     return (sum0 + sum1) + (sum2 + sum3);
 }
 
+// The same for 8-bit P: 64 probabilities of a row to e4m3, four per word.
+template <int EXP_MODE>
+__device__ __forceinline__ float exp_pack_half_fp8(const float *s, float c, float neg_m,
+                                                   uint32_t *pk) {
+    float sum0 = 0.0f, sum1 = 0.0f, sum2 = 0.0f, sum3 = 0.0f;
+#pragma unroll
+    for (int e = 0; e < kBlockN / 2; e += 4) {
+        float x0, x1, x2, x3, p0, p1, p2, p3;
+        fma2(x0, x1, s[e], s[e + 1], c, c, neg_m, neg_m);
+        fma2(x2, x3, s[e + 2], s[e + 3], c, c, neg_m, neg_m);
+        if (use_poly<EXP_MODE>(e)) {
+            ex2_poly2(p0, p1, x0, x1);
+        } else {
+            p0 = ex2_mufu(x0);
+            p1 = ex2_mufu(x1);
+        }
+        if (use_poly<EXP_MODE>(e + 2)) {
+            ex2_poly2(p2, p3, x2, x3);
+        } else {
+            p2 = ex2_mufu(x2);
+            p3 = ex2_mufu(x3);
+        }
+        add2(sum0, sum1, sum0, sum1, p0, p1);
+        add2(sum2, sum3, sum2, sum3, p2, p3);
+        pk[e >> 2] = pack_e4m3x4(p0, p1, p2, p3);
+    }
+    return (sum0 + sum1) + (sum2 + sum3);
+}
+
 // Score modifier, in log2 units: MOD bit 0 soft-cap, bit 1 ALiBi.  `raw` is
 // <q_i, k_j>; `dist` is i + (Sk - Sq) - j as a float.
 template <int MOD>
@@ -175,10 +211,12 @@ __device__ __forceinline__ float modified_score(float raw, float c, float softca
     return x;
 }
 
-template <int D, int NS, int EXP_MODE, int MOD = 0>
+template <int D, int NS, int EXP_MODE, int MOD = 0, int FP8 = 0>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ FwdParams p) {
-    using Smem = FwdSmem<D, NS>;
+    static_assert(!(FP8 && MOD), "the fp8 path has no score modifiers");
+    constexpr int EB = FP8 ? 1 : 2;
+    using Smem = FwdSmem<D, NS, EB>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_off = smem_u32(smem_raw);
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (raw_off & 1023u)) & 1023u));
@@ -273,7 +311,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
     const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : lo1;
     const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : hi1;
     const int n_blocks = (has0 || has1) ? (uhi - ulo + 1) : 0;
-    constexpr uint32_t kTileBytes = kBlockM * D * 2;
+    constexpr uint32_t kTileBytes = kBlockM * D * EB;
 
     // Registers: the softmax warpgroups hold a 128-column score row per
     // thread; the MMA / TMA warpgroup needs few.  384 x 168 at launch =
@@ -291,7 +329,8 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
                 for (int i = 0; i < 2; ++i)
                     for (int c = 0; c < Smem::kChunks; ++c)
-                        tma_load_4d(sm.q[i][c], &p.tm_q, &sm.q_full, c * 64, q0 + i * kBlockM, hq, b);
+                        tma_load_4d(sm.q[i][c], &p.tm_q, &sm.q_full, c * Smem::kChunkElems,
+                                    q0 + i * kBlockM, hq, b);
                 uint32_t it = 0;
                 bool ok = true;
                 for (int t = 0; t < n_blocks && ok; ++t) {
@@ -307,7 +346,8 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                         mbar_arrive_expect_tx(&sm.kv_full[slot], kTileBytes);
                         const CUtensorMap *map = which ? &p.tm_v : &p.tm_k;
                         for (int c = 0; c < Smem::kChunks; ++c)
-                            tma_load_4d(sm.kv[slot][c], map, &sm.kv_full[slot], c * 64, key0, hkv, b);
+                            tma_load_4d(sm.kv[slot][c], map, &sm.kv_full[slot], c * Smem::kChunkElems,
+                                        key0, hkv, b);
                     }
                 }
                 // Every copy still in flight lands before the CTA can exit (only
@@ -326,10 +366,18 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             // tcgen05 instructions (and the commits that track them).
             if (n_blocks > 0) {
                 const bool leader = elect_one();
-                constexpr uint32_t kIdescQK = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
-                constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlockM, D, 0, 1);
-                constexpr uint32_t kQTileBytes = Smem::kChunks * Smem::kChunkElems * 2;
-                constexpr uint32_t kChunkBytes = Smem::kChunkElems * 2;
+                constexpr uint32_t kIdescQK = FP8 ? idesc_e4m3_f32(kBlockM, kBlockN, 0, 0)
+                                                  : idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+                constexpr uint32_t kIdescPV = FP8 ? idesc_e4m3_f32(kBlockM, D, 0, 1)
+                                                  : idesc_bf16_f32(kBlockM, D, 0, 1);
+                constexpr uint32_t kQTileBytes = Smem::kChunks * Smem::kChunkBytes;
+                constexpr uint32_t kChunkBytes = Smem::kChunkBytes;
+                // One MMA consumes 32 bytes of each operand row: 16 bf16 or
+                // 32 fp8 elements.  PV takes kPvK keys per instruction from
+                // 8 TMEM columns of P; a 64-key half of P is kPvSteps of them.
+                constexpr int kKSteps = D * EB / 32;
+                constexpr int kPvK = 32 / EB;
+                constexpr int kPvSteps = (kBlockN / 2) / kPvK;
                 // Base descriptors; a K-step or a ring slot only moves the start
                 // address (bits 0-13, in 16-byte units), a constant add.
                 const uint64_t q_desc = smem_desc_sw128(smem_u32(&sm.q[0][0][0]), 16, 1024);
@@ -359,10 +407,10 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                     const uint64_t b0 = k_desc + (((ring_pos(j, 0) % NS) * kQTileBytes) >> 4);
                     if (leader) {
 #pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
+                        for (int ks = 0; ks < kKSteps; ++ks) {
                             const uint32_t off = ((ks >> 2) * kChunkBytes + (ks & 3) * 32) >> 4;
-                            mma_ss(tmem + i * kBlockN, a0 + off, b0 + off, kIdescQK,
-                                   ks > 0 ? 1u : 0u);
+                            mma_ss_k<FP8>(tmem + i * kBlockN, a0 + off, b0 + off, kIdescQK,
+                                          ks > 0 ? 1u : 0u);
                         }
                         tc_commit(&sm.s_full[i]);
                     }
@@ -407,9 +455,10 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                             tc_fence_after();
                             if (leader) {
 #pragma unroll
-                                for (int ks = 0; ks < kBlockN / 32; ++ks)
-                                    mma_ts(o_tmem, p_tmem + ks * 8, vb + ((ks * 16 * 128) >> 4),
-                                           kIdescPV, ks > 0 ? 1u : first);
+                                for (int ks = 0; ks < kPvSteps; ++ks)
+                                    mma_ts_k<FP8>(o_tmem, p_tmem + ks * 8,
+                                                  vb + ((ks * kPvK * 128) >> 4), kIdescPV,
+                                                  ks > 0 ? 1u : first);
                             }
                             __syncwarp();
                             ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_full[i], par,
@@ -419,9 +468,9 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                             tc_fence_after();
                             if (leader) {
 #pragma unroll
-                                for (int ks = kBlockN / 32; ks < kBlockN / 16; ++ks)
-                                    mma_ts(o_tmem, p_tmem + ks * 8, vb + ((ks * 16 * 128) >> 4),
-                                           kIdescPV, 1u);
+                                for (int ks = kPvSteps; ks < 2 * kPvSteps; ++ks)
+                                    mma_ts_k<FP8>(o_tmem, p_tmem + ks * 8,
+                                                  vb + ((ks * kPvK * 128) >> 4), kIdescPV, 1u);
                                 if (j == hi_i) tc_commit(&sm.o_final[i]);
                             }
                             __syncwarp();
@@ -546,7 +595,10 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 alpha = ex2_mufu(m_run - m_cand);
                 m_run = m_cand;
             }
-            const float neg_m = m_run == -INFINITY ? 0.0f : -m_run;
+            // fp8: P = 2^(x - m + p_offset) <= 2^8 keeps e4m3's range for the
+            // small probabilities (the same factor scales l, so O and LSE are
+            // unchanged).
+            const float neg_m = m_run == -INFINITY ? 0.0f : (FP8 ? p.p_offset - m_run : -m_run);
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 3);
 
             l_run *= alpha;
@@ -580,16 +632,30 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             // use MUFU only: ex2(-inf) = 0 exactly.
             uint32_t pk[kBlockN / 2];
             if (MOD) __syncwarp();  // converged before the warp-collective TMEM store
-            l_run += masked ? exp_pack_half<0>(s, c_exp, neg_m, pk)
-                            : exp_pack_half<EXP_MODE>(s, c_exp, neg_m, pk);
-            tmem_st32(s_tmem + 0, pk + 0);
+            if constexpr (FP8) {
+                // 64 e4m3 probabilities per 16 columns.
+                l_run += masked ? exp_pack_half_fp8<0>(s, c_exp, neg_m, pk)
+                                : exp_pack_half_fp8<EXP_MODE>(s, c_exp, neg_m, pk);
+                tmem_st16(s_tmem + 0, pk + 0);
+            } else {
+                l_run += masked ? exp_pack_half<0>(s, c_exp, neg_m, pk)
+                                : exp_pack_half<EXP_MODE>(s, c_exp, neg_m, pk);
+                tmem_st32(s_tmem + 0, pk + 0);
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_half[i]);
-            l_run += masked ? exp_pack_half<0>(s + 64, c_exp, neg_m, pk + 32)
-                            : exp_pack_half<EXP_MODE>(s + 64, c_exp, neg_m, pk + 32);
-            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
-            tmem_st32(s_tmem + 32, pk + 32);
+            if constexpr (FP8) {
+                l_run += masked ? exp_pack_half_fp8<0>(s + 64, c_exp, neg_m, pk + 16)
+                                : exp_pack_half_fp8<EXP_MODE>(s + 64, c_exp, neg_m, pk + 16);
+                if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
+                tmem_st16(s_tmem + 16, pk + 16);
+            } else {
+                l_run += masked ? exp_pack_half<0>(s + 64, c_exp, neg_m, pk + 32)
+                                : exp_pack_half<EXP_MODE>(s + 64, c_exp, neg_m, pk + 32);
+                if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
+                tmem_st32(s_tmem + 32, pk + 32);
+            }
             tmem_wait_st();
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 5);
             tc_fence_before();
@@ -605,7 +671,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         }
         if (ok) {
             const bool row_ok = row < p.Sq;
-            const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+            const float inv_l = l_run > 0.0f ? (FP8 ? p.v_descale : 1.0f) / l_run : 0.0f;
             __nv_bfloat16 *o_row =
                 p.o + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)D;
 #pragma unroll
@@ -632,7 +698,8 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 }
             }
             if (row_ok) {
-                const float lse = l_run > 0.0f ? (m_run + log2f(l_run)) * 0.69314718055994531f
+                const float m_lse = FP8 ? m_run - p.p_offset : m_run;
+                const float lse = l_run > 0.0f ? (m_lse + log2f(l_run)) * 0.69314718055994531f
                                                : -INFINITY;
                 p.lse[((size_t)b * p.Hq + hq) * p.Sq + row] = lse;
             }

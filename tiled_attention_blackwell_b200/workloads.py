@@ -13,7 +13,10 @@ Recipe (all on the CPU, deterministic):
     before rounding, which forces running-max jumps;
   * document lengths are drawn with ``numpy.random.default_rng(seed)`` as
     integers uniform in [512, 4096] (inclusive) until they cover the
-    sequence; the last document is clipped to what is left.
+    sequence; the last document is clipped to what is left;
+  * fp8 workloads draw the same fp32 tensors and quantise each one to e4m3
+    with one per-tensor factor, descale = max|x| / 448 (torch's
+    round-to-nearest conversion of x / descale).
 No public dataset or benchmark suite stands behind these shapes; the pages
 measure on none that could be used here, so synthetic inputs of the named
 shapes stand in.
@@ -44,6 +47,7 @@ class Workload:
     doc_lengths: Optional[tuple] = None  # (lo, hi) inclusive, or None
     backward: bool = False
     window: tuple = (-1, -1)
+    dtype: str = "bf16"  # "bf16" or "fp8" (e4m3 Q, K, V with per-tensor factors)
 
     @property
     def scale(self) -> float:
@@ -54,7 +58,7 @@ class Workload:
         if self.doc_lengths:
             mask = f"document-causal, docs U[{self.doc_lengths[0]},{self.doc_lengths[1]}]"
         return (f"B={self.B} Hq={self.Hq} Hkv={self.Hkv} Sq=Sk={self.S} D={self.D} "
-                f"{mask} bf16" + (" backward" if self.backward else " forward"))
+                f"{mask} {self.dtype}" + (" backward" if self.backward else " forward"))
 
 
 # The five workloads: tiny oracle case, outlier-K non-causal, the causal
@@ -68,6 +72,9 @@ WORKLOADS = {
                                doc_lengths=(512, 4096)),
     "causal_bwd_s4096": Workload("causal_bwd_s4096", 2, 16, 16, 4096, 128, True, seed=5,
                                  backward=True),
+    # The headline shape with e4m3 inputs (the low-precision forward).
+    "causal_s8192_fp8": Workload("causal_s8192_fp8", 2, 16, 16, 8192, 128, True, seed=3,
+                                 dtype="fp8"),
 }
 
 HEADLINE = "causal_s8192"
@@ -103,11 +110,35 @@ def make_tensors(B, Hq, Hkv, Sq, Sk, D, seed, *, qk_std=1.0, k_outlier_frac=0.0,
     return out
 
 
+def quantize_e4m3(x: torch.Tensor):
+    """Per-tensor e4m3 codes (torch.float8_e4m3fn) and the descale factor
+    with x ~= descale * codes."""
+    amax = float(x.abs().max())
+    descale = amax / 448.0 if amax > 0 else 1.0
+    return (x.float() / descale).to(torch.float8_e4m3fn), descale
+
+
+def make_tensors_fp8(B, Hq, Hkv, Sq, Sk, D, seed, *, qk_std=1.0, v_std=1.0):
+    """e4m3 CPU tensors q8/k8/v8 and their descale factors (fp32 draws in
+    the order Q, K, V, as make_tensors)."""
+    g = torch.Generator().manual_seed(int(seed))
+    out = {}
+    for name, shape, std in (("q", (B, Sq, Hq, D), qk_std), ("k", (B, Sk, Hkv, D), qk_std),
+                             ("v", (B, Sk, Hkv, D), v_std)):
+        codes, descale = quantize_e4m3(torch.randn(shape, generator=g, dtype=torch.float32) * std)
+        out[name] = codes
+        out[name + "_descale"] = descale
+    return out
+
+
 def make_inputs(w: Workload):
     """All inputs of a named workload (CPU tensors) plus its mask arguments."""
-    t = make_tensors(w.B, w.Hq, w.Hkv, w.S, w.S, w.D, w.seed, qk_std=w.qk_std,
-                     k_outlier_frac=w.k_outlier_frac, k_outlier_mult=w.k_outlier_mult,
-                     with_dout=w.backward)
+    if w.dtype == "fp8":
+        t = make_tensors_fp8(w.B, w.Hq, w.Hkv, w.S, w.S, w.D, w.seed, qk_std=w.qk_std)
+    else:
+        t = make_tensors(w.B, w.Hq, w.Hkv, w.S, w.S, w.D, w.seed, qk_std=w.qk_std,
+                         k_outlier_frac=w.k_outlier_frac, k_outlier_mult=w.k_outlier_mult,
+                         with_dout=w.backward)
     t["doc_offsets"] = (draw_doc_offsets(w.S, w.seed, *w.doc_lengths)
                         if w.doc_lengths else None)
     t["causal"] = w.causal
