@@ -34,7 +34,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from tiled_attention_blackwell_b200.workloads import (HEADLINE, WORKLOADS,  # noqa: E402
-                                                      make_inputs, useful_flops)
+                                                      make_inputs, useful_flops,
+                                                      window_keys_per_row)
 
 METRIC = "attention fwd TFLOP/s and % of B200 BF16 tensor peak (S=8192 causal, D=128)"
 UNIT = "TFLOP/s"
@@ -60,6 +61,10 @@ def parse_args(argv=None):
                     help="skip the oracle timing leg (faster local iteration)")
     ap.add_argument("--exp2-mode", type=int, default=None)
     ap.add_argument("--rescale-threshold", type=float, default=None)
+    ap.add_argument("--softcap", type=float, default=None,
+                    help="forward with the soft-capping score modifier (cap value)")
+    ap.add_argument("--alibi", action="store_true",
+                    help="forward with ALiBi slopes 2^(-8(h+1)/Hq)")
     return ap.parse_args(argv)
 
 
@@ -104,7 +109,10 @@ def profiled_traffic(config: str):
 
 def allowed_keys_per_row(w, doc_offsets):
     """Number of keys each query row may see (for FLOP accounting of a row
-    sample): causal -> i + 1, document-causal -> i - doc_start + 1."""
+    sample): causal -> i + 1, document-causal -> i - doc_start + 1, sliding
+    window -> the window's width clipped at the sequence ends."""
+    if tuple(w.window) != (-1, -1):
+        return window_keys_per_row(w.S, w.S, w.window, w.causal)
     i = np.arange(w.S, dtype=np.int64)
     if doc_offsets is not None:
         starts = np.repeat(doc_offsets[:-1], np.diff(doc_offsets)).astype(np.int64)
@@ -260,6 +268,9 @@ def workload_config(w, doc_offsets):
            "scale": w.scale}
     if doc_offsets is not None:
         cfg["num_docs"] = int(len(doc_offsets) - 1)
+    if tuple(w.window) != (-1, -1):
+        cfg["mask"] = "causal sliding window" if w.causal else "sliding window"
+        cfg["window"] = list(w.window)
     eb = 1 if w.dtype == "fp8" else 2  # bytes per Q/K/V element; O is bf16
     io_bytes = (eb * (w.B * w.S * w.Hq * w.D + 2 * w.B * w.S * w.Hkv * w.D)
                 + 2 * w.B * w.S * w.Hq * w.D + 4 * w.B * w.Hq * w.S)
@@ -281,7 +292,8 @@ def run_ours(args):
     w = WORKLOADS[args.config]
     inp = make_inputs(w)
     docs_np = inp["doc_offsets"]
-    flops = useful_flops(w.B, w.Hq, w.S, w.S, w.D, causal=w.causal, doc_offsets=docs_np)
+    flops = useful_flops(w.B, w.Hq, w.S, w.S, w.D, causal=w.causal, doc_offsets=docs_np,
+                         window=w.window)
     cfg = workload_config(w, docs_np)
     cfg["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
 
@@ -312,12 +324,24 @@ def run_ours(args):
     flush = None if cfg["io_bytes"] > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8,
                                                                  device=device)
     opts = None
-    if args.exp2_mode is not None or args.rescale_threshold is not None:
+    slopes = None
+    if args.alibi:
+        slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / w.Hq) for h in range(w.Hq)],
+                              dtype=torch.float32, device=device)
+        cfg["alibi"] = "slopes 2^(-8(h+1)/Hq)"
+    if args.softcap is not None:
+        cfg["softcap"] = args.softcap
+    if (args.exp2_mode is not None or args.rescale_threshold is not None
+            or slopes is not None or args.softcap is not None):
         kw = {}
         if args.exp2_mode is not None:
             kw["exp2_mode"] = args.exp2_mode
         if args.rescale_threshold is not None:
             kw["rescale_threshold"] = args.rescale_threshold
+        if args.softcap is not None:
+            kw["softcap"] = args.softcap
+        if slopes is not None:
+            kw["alibi_slopes"] = slopes.data_ptr()
         opts = attn.default_options(**kw)
     stream = torch.cuda.current_stream(device)
 
@@ -402,6 +426,10 @@ def run_ours(args):
         metric = f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()})"
     elif fp8:
         metric = f"attention fwd TFLOP/s and % of B200 FP8 tensor peak ({w.describe()})"
+    elif w.name != HEADLINE or slopes is not None or args.softcap is not None:
+        mods = "".join([f", softcap {args.softcap:g}" if args.softcap is not None else "",
+                        ", ALiBi" if slopes is not None else ""])
+        metric = f"attention fwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()}{mods})"
     else:
         metric = METRIC
     result = {
@@ -427,7 +455,8 @@ def run_ours(args):
         "gpu_launches": args.steps * (3 if w.backward else 1),
         "clocks": sampler.summary(),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not w.backward:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and not w.backward
+            and slopes is None and args.softcap is None):
         n_rows = rows_for_seconds(w, inp, 15.0)
         dt, fl, cores = oracle_sample(w, inp, n_rows)
         result["cpu_baseline"] = {

@@ -53,13 +53,15 @@ def test_single_rank_reductions_are_identity():
 
 
 @pytest.mark.parametrize("name", ["causal_s8192", "gqa_doc_s16384", "outlier_s4096",
-                                  "tiny_d64"])
+                                  "tiny_d64", "window_s16384"])
 def test_row_key_counts_match_dense_mask(name):
     """The per-row key counts used for the CPU sample's FLOPs equal the
     allowed-set sizes of the mask, on a shrunken copy of the workload."""
     w0 = WORKLOADS[name]
     S = 1000
-    w = Workload(name, 1, 1, 1, S, w0.D, w0.causal, w0.seed, doc_lengths=w0.doc_lengths)
+    window = (255, 0) if tuple(w0.window) != (-1, -1) else (-1, -1)
+    w = Workload(name, 1, 1, 1, S, w0.D, w0.causal, w0.seed, doc_lengths=w0.doc_lengths,
+                 window=window)
     docs = None
     if w.doc_lengths:
         docs = np.array([0, 130, 131, 600, 1000], dtype=np.int32)
@@ -72,9 +74,14 @@ def test_row_key_counts_match_dense_mask(name):
     if docs is not None:
         ids = np.repeat(np.arange(len(docs) - 1), np.diff(docs))
         allowed &= ids[:, None] == ids[None, :]
+    if window != (-1, -1):
+        allowed &= j >= i - window[0]
     np.testing.assert_array_equal(keys, allowed.sum(axis=1))
+    if window != (-1, -1):
+        assert useful_flops(1, 1, S, S, w.D, causal=True, window=window) == \
+            4.0 * w.D * allowed.sum()
     # and the whole-workload convention: causal = half of the square
-    if docs is None:
+    elif docs is None:
         full = useful_flops(1, 1, S, S, w.D, causal=w.causal)
         expect = 4.0 * w.D * (S * S / 2 if w.causal else S * S)
         assert full == expect

@@ -238,18 +238,20 @@ def sample_rows(B, H, S, n_random, seed):
 
 
 @pytest.mark.parametrize("name", ["outlier_s4096", "causal_s8192", "gqa_doc_s16384",
-                                  "causal_bwd_s4096"])
+                                  "causal_bwd_s4096", "window_s16384"])
 def test_full_size_workload_sampled(name):
     """The benchmark's workloads at full size, in the benchmark's launch
     configuration: sampled rows against the oracle, plus properties of every
     row (finite O, finite LSE: every row here has at least one key)."""
     w = WORKLOADS[name]
     t = make_inputs(w)
-    o, lse = run_gpu(t, causal=w.causal, doc_offsets=t["doc_offsets"], scale=w.scale)
+    window = None if tuple(w.window) == (-1, -1) else w.window
+    o, lse = run_gpu(t, causal=w.causal, window=window, doc_offsets=t["doc_offsets"],
+                     scale=w.scale)
     assert np.isfinite(o).all() and np.isfinite(lse).all()
     rows = sample_rows(w.B, w.Hq, w.S, 200, seed=w.seed)
     o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=w.scale, causal=w.causal,
-                                     doc_offsets=t["doc_offsets"], rows=rows)
+                                     window=window, doc_offsets=t["doc_offsets"], rows=rows)
     o_s = o[rows[:, 0], rows[:, 2], rows[:, 1]]
     lse_s = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
     err = np.abs(o_s - o_ref)

@@ -72,6 +72,9 @@ WORKLOADS = {
                                doc_lengths=(512, 4096)),
     "causal_bwd_s4096": Workload("causal_bwd_s4096", 2, 16, 16, 4096, 128, True, seed=5,
                                  backward=True),
+    # Causal sliding window of 4096 keys (window_left 4095) over S = 16384.
+    "window_s16384": Workload("window_s16384", 1, 16, 16, 16384, 128, True, seed=6,
+                              window=(4095, 0)),
     # The headline shape with e4m3 inputs (the low-precision forward).
     "causal_s8192_fp8": Workload("causal_s8192_fp8", 2, 16, 16, 8192, 128, True, seed=3,
                                  dtype="fp8"),
@@ -147,10 +150,26 @@ def make_inputs(w: Workload):
     return t
 
 
-def useful_flops(B, Hq, Sq, Sk, D, *, causal=False, doc_offsets=None):
+def window_keys_per_row(Sq, Sk, window, causal):
+    """Keys each query row may see under a sliding window (bottom-right
+    aligned, as the masks): int64 [Sq]."""
+    i = np.arange(Sq, dtype=np.int64) + (Sk - Sq)
+    wl, wr = window
+    lo = np.maximum(i - wl, 0) if wl >= 0 else np.zeros_like(i)
+    hi = i if causal else np.full_like(i, Sk - 1)
+    if wr >= 0:
+        hi = np.minimum(hi, i + wr)
+    hi = np.minimum(hi, Sk - 1)
+    return np.maximum(hi - lo + 1, 0)
+
+
+def useful_flops(B, Hq, Sq, Sk, D, *, causal=False, doc_offsets=None, window=None):
     """Forward FLOPs by the useful-work convention: 4*D per (row, key) pair,
     counting a causal mask as half of the square (per document when a
-    document mask is given).  Used only for reporting throughput."""
+    document mask is given); a sliding window counts its allowed pairs
+    exactly.  Used only for reporting throughput."""
+    if window is not None and tuple(window) != (-1, -1):
+        return 4.0 * B * Hq * D * float(window_keys_per_row(Sq, Sk, window, causal).sum())
     if doc_offsets is not None:
         lengths = np.diff(np.asarray(doc_offsets, dtype=np.int64))
         pairs = float(np.sum(lengths.astype(np.float64) ** 2)) / 2.0
