@@ -86,25 +86,32 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(config: str):
-    """DRAM bytes per launch from the committed ncu summary of this workload,
-    if it was taken on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", f"fwd_{config}_ncu.md")
+def _profile_fields(name: str):
     try:
-        text = open(path).read()
+        text = open(os.path.join(ROOT, "profiles", name)).read()
     except OSError:
-        return None
+        return {}
     fields = {}
     for line in text.splitlines():
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             fields[k.strip()] = v.strip().strip("`")
-    if fields.get("kernel_sources_sha256") != kernel_source_hash():
-        return None
-    try:
-        return int(fields["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    return fields
+
+
+def profiled_traffic(config: str):
+    """DRAM bytes per launch from the committed ncu summaries of this
+    workload, if they were taken on the current kernel sources; else None."""
+    for name, key in ((f"fwd_{config}_ncu.md", "dram_bytes_per_launch"),
+                      ("fwd_all_workloads_ncu.md", f"dram_bytes_per_launch[{config}]")):
+        fields = _profile_fields(name)
+        if fields.get("kernel_sources_sha256") != kernel_source_hash() or key not in fields:
+            continue
+        try:
+            return int(fields[key])
+        except ValueError:
+            return None
+    return None
 
 
 def allowed_keys_per_row(w, doc_offsets):

@@ -107,3 +107,15 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["higher_is_better"] is True
+
+
+def test_profiled_traffic_is_tied_to_the_kernel_sources(monkeypatch):
+    """The roofline's traffic comes from the committed ncu summary only while
+    the kernel sources hash to the value recorded there."""
+    real = bench.kernel_source_hash()
+    fields = bench._profile_fields("fwd_causal_s8192_ncu.md")
+    if fields.get("kernel_sources_sha256") == real:
+        assert bench.profiled_traffic("causal_s8192") == int(fields["dram_bytes_per_launch"])
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0000000000000000")
+    assert bench.profiled_traffic("causal_s8192") is None
+    assert bench.profiled_traffic("causal_s8192_fp8") is None
