@@ -223,18 +223,20 @@ attn_status_t prepare_kernel(Kernel kernel, size_t smem, int threads, int min_re
 }
 
 constexpr int kBwdStagesQ = 2;
-constexpr int kBwdStagesKV = 4;
+// dQ kernel: K and V ring depths (224 KB of SMEM with Q and dO at D = 128).
+constexpr int bwd_k_stages(int D) { return D == 128 ? 3 : 6; }
+constexpr int bwd_v_stages(int D) { return D == 128 ? 2 : 4; }
 
 template <int D, int MOD>
 attn_status_t launch_bwd(const tab::BwdParams &p, cudaStream_t stream) {
     using DkdvS = tab::DkdvSmem<D, kBwdStagesQ>;
-    using DqS = tab::DqSmem<D, kBwdStagesKV>;
+    using DqS = tab::DqSmem<D, bwd_k_stages(D), bwd_v_stages(D)>;
     constexpr size_t smem_dkdv = sizeof(DkdvS) + 1024;
     constexpr size_t smem_dq = sizeof(DqS) + 1024;
     static_assert(smem_dkdv <= 232448 && smem_dq <= 232448, "shared memory budget");
     auto k_pre = tab::attn_bwd_preprocess_kernel<D>;
     auto k_dkdv = tab::attn_bwd_dkdv_kernel<D, kBwdStagesQ, MOD>;
-    auto k_dq = tab::attn_bwd_dq_kernel<D, kBwdStagesKV, MOD>;
+    auto k_dq = tab::attn_bwd_dq_kernel<D, bwd_k_stages(D), bwd_v_stages(D), MOD>;
     static std::once_flag once[kMaxDevices];
     static attn_status_t prep[kMaxDevices];
     int dev = 0;

@@ -611,26 +611,30 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
 
 // --------------------------------------------------------------------- dQ
 
-template <int D, int NS>
+// K and V have rings of their own: K of a block is read twice (by S and,
+// after the block's dS, by dQ) while V is read once (by dP), so in one shared
+// ring the next K would wait for the dQ of the block before last.
+template <int D, int NK, int NV>
 struct DqSmem {
     static constexpr int kChunks = D / 64;
     static constexpr int kChunkElems = 128 * 64;
     __nv_bfloat16 q[kChunks][kChunkElems];
     __nv_bfloat16 dout[kChunks][kChunkElems];
-    __nv_bfloat16 kv[NS][kChunks][kChunkElems];
+    __nv_bfloat16 k[NK][kChunks][kChunkElems];
+    __nv_bfloat16 v[NV][kChunks][kChunkElems];
     uint64_t q_full;
-    uint64_t kv_full[NS];
-    uint64_t kv_empty[NS];
+    uint64_t k_full[NK], k_empty[NK];
+    uint64_t v_full[NV], v_empty[NV];
     uint64_t s_full, dp_free, ds_ready, final_bar, drain;
     uint32_t tmem_base;
     int abort_flag;
     int range[2];
 };
 
-template <int D, int NS, int MOD = 0>
+template <int D, int NK, int NV, int MOD = 0>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
-    using Smem = DqSmem<D, NS>;
+    using Smem = DqSmem<D, NK, NV>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_off = smem_u32(smem_raw);
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (raw_off & 1023u)) & 1023u));
@@ -649,9 +653,13 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
 
     if (threadIdx.x == 0) {
         mbar_init(&sm.q_full, 1);
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+        for (int s = 0; s < NK; ++s) {
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.k_empty[s], 1);
+        }
+        for (int s = 0; s < NV; ++s) {
+            mbar_init(&sm.v_full[s], 1);
+            mbar_init(&sm.v_empty[s], 1);
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.dp_free, 256);
@@ -710,25 +718,31 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                 tma_load_4d(sm.q[c], &p.tm_q, &sm.q_full, c * 64, q0, hq, b);
                 tma_load_4d(sm.dout[c], &p.tm_do, &sm.q_full, c * 64, q0, hq, b);
             }
-            uint32_t it = 0;
+            int nk = 0, nv = 0;  // K and V copies issued
             bool ok = true;
             for (int t = 0; t < n_blocks && ok; ++t) {
                 const int key0 = (lo_b + t) * 128;
-                for (int which = 0; which < 2 && ok; ++which, ++it) {
-                    const uint32_t slot = it % NS;
-                    ok = wait_bounded(&sm.kv_empty[slot], ((it / NS) & 1u) ^ 1u, abort_flag,
-                                      p.status);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&sm.kv_full[slot], kTileBytes);
-                    const CUtensorMap *map = which ? &p.tm_v : &p.tm_k;
-                    for (int c = 0; c < Smem::kChunks; ++c)
-                        tma_load_4d(sm.kv[slot][c], map, &sm.kv_full[slot], c * 64, key0, hkv, b);
-                }
+                ok = wait_bounded(&sm.k_empty[t % NK], ((uint32_t)(t / NK) & 1u) ^ 1u,
+                                  abort_flag, p.status);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&sm.k_full[t % NK], kTileBytes);
+                for (int c = 0; c < Smem::kChunks; ++c)
+                    tma_load_4d(sm.k[t % NK][c], &p.tm_k, &sm.k_full[t % NK], c * 64, key0, hkv, b);
+                ++nk;
+                ok = wait_bounded(&sm.v_empty[t % NV], ((uint32_t)(t / NV) & 1u) ^ 1u,
+                                  abort_flag, p.status);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&sm.v_full[t % NV], kTileBytes);
+                for (int c = 0; c < Smem::kChunks; ++c)
+                    tma_load_4d(sm.v[t % NV][c], &p.tm_v, &sm.v_full[t % NV], c * 64, key0, hkv, b);
+                ++nv;
             }
+            // Copies still in flight land before the CTA can exit.
             wait_bounded(&sm.q_full, 0, abort_flag, p.status, false);
-            const uint32_t first = it > NS ? it - NS : 0;
-            for (uint32_t L = first; L < it; ++L)
-                wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status, false);
+            for (int t = nk > NK ? nk - NK : 0; t < nk; ++t)
+                wait_bounded(&sm.k_full[t % NK], (uint32_t)(t / NK) & 1u, abort_flag, p.status, false);
+            for (int t = nv > NV ? nv - NV : 0; t < nv; ++t)
+                wait_bounded(&sm.v_full[t % NV], (uint32_t)(t / NV) & 1u, abort_flag, p.status, false);
         }
         __syncwarp();
     } else if (warp == kBwdMmaWarp) {
@@ -740,24 +754,22 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
             constexpr uint32_t kChunkBytes = Smem::kChunkElems * 2;
             const uint64_t q_desc = smem_desc_sw128(smem_u32(&sm.q[0][0]), 16, 1024);
             const uint64_t do_desc = smem_desc_sw128(smem_u32(&sm.dout[0][0]), 16, 1024);
-            const uint64_t kv_kdesc = smem_desc_sw128(smem_u32(&sm.kv[0][0][0]), 16, 1024);
-            const uint64_t kv_mdesc =
-                smem_desc_sw128(smem_u32(&sm.kv[0][0][0]), kChunkBytes, 1024);
+            const uint64_t k_kdesc = smem_desc_sw128(smem_u32(&sm.k[0][0][0]), 16, 1024);
+            const uint64_t k_mdesc = smem_desc_sw128(smem_u32(&sm.k[0][0][0]), kChunkBytes, 1024);
+            const uint64_t v_kdesc = smem_desc_sw128(smem_u32(&sm.v[0][0][0]), 16, 1024);
             bool ok = __all_sync(0xffffffffu, wait_bounded(&sm.q_full, 0, abort_flag, p.status));
             tc_fence_after();
-            auto wait_slot = [&](uint32_t L) {
+            auto wait_full = [&](uint64_t *bar, uint32_t parity) {
                 if (ok)
-                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u,
-                                                              abort_flag, p.status));
+                    ok = __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, p.status));
                 tc_fence_after();
             };
             // S of block t into its buffer (needs K), then dP (needs V); one
             // commit signals both.
             auto issue_s = [&](int t) {
-                const uint32_t Lk = 2u * t;
-                wait_slot(Lk);
+                wait_full(&sm.k_full[t % NK], (uint32_t)(t / NK) & 1u);
                 if (!ok) return;
-                const uint64_t kb_k = kv_kdesc + (((Lk % NS) * kTile) >> 4);
+                const uint64_t kb_k = k_kdesc + (((uint32_t)(t % NK) * kTile) >> 4);
                 const uint32_t col = (t & 1) ? kColS1 : kColS;
                 if (leader) {
 #pragma unroll
@@ -769,10 +781,9 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                 __syncwarp();
             };
             auto issue_dp = [&](int t) {
-                const uint32_t Lv = 2u * t + 1;
-                wait_slot(Lv);
+                wait_full(&sm.v_full[t % NV], (uint32_t)(t / NV) & 1u);
                 if (!ok) return;
-                const uint64_t vb_k = kv_kdesc + (((Lv % NS) * kTile) >> 4);
+                const uint64_t vb_k = v_kdesc + (((uint32_t)(t % NV) * kTile) >> 4);
                 if (leader) {
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
@@ -781,7 +792,7 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                                ks > 0 ? 1u : 0u);
                     }
                     tc_commit(&sm.s_full);
-                    tc_commit(&sm.kv_empty[Lv % NS]);  // V of this block is consumed
+                    tc_commit(&sm.v_empty[t % NV]);  // V of this block is consumed
                 }
                 __syncwarp();
             };
@@ -802,8 +813,7 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                                                           abort_flag, p.status));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t Lk = 2u * t;
-                const uint64_t kb_m = kv_mdesc + (((Lk % NS) * kTile) >> 4);
+                const uint64_t kb_m = k_mdesc + (((uint32_t)(t % NK) * kTile) >> 4);
                 const uint32_t col = (t & 1) ? kColS1 : kColS;
                 if (leader) {
 #pragma unroll
@@ -811,7 +821,7 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                         mma_ts(tmem + kColDQ, tmem + half_operand_col(col, ks),
                                kb_m + ((ks * 16 * 128) >> 4), kIdescQ,
                                (t > 0 || ks > 0) ? 1u : 0u);
-                    tc_commit(&sm.kv_empty[Lk % NS]);  // K of this block is consumed
+                    tc_commit(&sm.k_empty[t % NK]);  // K of this block is consumed
                 }
                 __syncwarp();
             }
