@@ -52,6 +52,16 @@ __device__ __forceinline__ float bwd_ex2(float x, int e) {
     const int pair = (e >> 1) % 5;
     return (pair == 1 || pair == 3) ? ex2_poly(x) : ex2_mufu(x);
 }
+// The same split for the pair (e, e+1), e even, in packed f32x2 arithmetic.
+__device__ __forceinline__ void bwd_ex2_pair(float &y0, float &y1, float x0, float x1, int e) {
+    const int pair = (e >> 1) % 5;
+    if (pair == 1 || pair == 3) {
+        ex2_poly2(y0, y1, x0, x1);
+    } else {
+        y0 = ex2_mufu(x0);
+        y1 = ex2_mufu(x1);
+    }
+}
 
 struct BwdParams {
     CUtensorMap tm_q;   // bf16 [B][Sq][Hq][D], box (64, 128, 1, 1)
@@ -502,10 +512,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
 #pragma unroll
                 for (int e = 0; e < 64; e += 4) {
                     const float4 l = l4[e >> 2];
-                    pv[e + 0] = bwd_ex2(fmaf(pv[e + 0], c, -l.x), e + 0);
-                    pv[e + 1] = bwd_ex2(fmaf(pv[e + 1], c, -l.y), e + 1);
-                    pv[e + 2] = bwd_ex2(fmaf(pv[e + 2], c, -l.z), e + 2);
-                    pv[e + 3] = bwd_ex2(fmaf(pv[e + 3], c, -l.w), e + 3);
+                    float x0, x1, x2, x3;
+                    fma2(x0, x1, pv[e + 0], pv[e + 1], c, c, -l.x, -l.y);
+                    fma2(x2, x3, pv[e + 2], pv[e + 3], c, c, -l.z, -l.w);
+                    bwd_ex2_pair(pv[e + 0], pv[e + 1], x0, x1, e + 0);
+                    bwd_ex2_pair(pv[e + 2], pv[e + 3], x2, x3, e + 2);
                     pk[(e >> 1) + 0] = pack_bf16x2(pv[e + 0], pv[e + 1]);
                     pk[(e >> 1) + 1] = pack_bf16x2(pv[e + 2], pv[e + 3]);
                 }
@@ -547,10 +558,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
 #pragma unroll
             for (int e = 0; e < 64; e += 4) {
                 const float4 dd = d4[e >> 2];
-                const float g0 = pv[e + 0] * (__uint_as_float(dr[e + 0]) - dd.x);
-                const float g1 = pv[e + 1] * (__uint_as_float(dr[e + 1]) - dd.y);
-                const float g2 = pv[e + 2] * (__uint_as_float(dr[e + 2]) - dd.z);
-                const float g3 = pv[e + 3] * (__uint_as_float(dr[e + 3]) - dd.w);
+                float a0, a1, a2, a3, g0, g1, g2, g3;
+                add2(a0, a1, __uint_as_float(dr[e + 0]), __uint_as_float(dr[e + 1]), -dd.x, -dd.y);
+                add2(a2, a3, __uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3]), -dd.z, -dd.w);
+                mul2(g0, g1, pv[e + 0], pv[e + 1], a0, a1);
+                mul2(g2, g3, pv[e + 2], pv[e + 3], a2, a3);
                 pk[(e >> 1) + 0] = pack_bf16x2(g0, g1);
                 pk[(e >> 1) + 1] = pack_bf16x2(g2, g3);
             }
@@ -892,13 +904,18 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                 }
             } else {
 #pragma unroll
-                for (int e = 0; e < 64; ++e) pv[e] = bwd_ex2(fmaf(pv[e], c, -l2), e);
+                for (int e = 0; e < 64; e += 2) {
+                    float x0, x1;
+                    fma2(x0, x1, pv[e], pv[e + 1], c, c, -l2, -l2);
+                    bwd_ex2_pair(pv[e], pv[e + 1], x0, x1, e);
+                }
             }
             uint32_t pk[32];
 #pragma unroll
             for (int e = 0; e < 64; e += 2) {
-                const float g0 = pv[e] * (__uint_as_float(dr[e]) - dval);
-                const float g1 = pv[e + 1] * (__uint_as_float(dr[e + 1]) - dval);
+                float a0, a1, g0, g1;
+                add2(a0, a1, __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), -dval, -dval);
+                mul2(g0, g1, pv[e], pv[e + 1], a0, a1);
                 pk[e / 2] = pack_bf16x2(g0, g1);
             }
             __syncwarp();
