@@ -276,3 +276,39 @@ def test_device_wait_timeout_is_reported_and_recoverable():
     o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=1 / math.sqrt(128),
                                      causal=True)
     check(o, lse, o_ref, lse_ref, "after a timeout")
+
+
+# ------------------------------------------------------------ maximum sizes
+
+def test_large_tensors_need_64bit_offsets():
+    """O with 2^31 elements (B=1, S=65536, Hq=256, Hkv=4, D=128, causal): every
+    row's output and LSE offsets past 2^31 must land where they belong.
+    Inputs are seeded normals drawn on the device (the host copy for the
+    oracle is taken from the same tensors); rows sampled near the end of the
+    sequence and the last heads are checked against the oracle."""
+    B, S, Hq, Hkv, D = 1, 65536, 256, 4, 128
+    need = (2 * B * S * Hq * D + 2 * B * S * Hkv * D) * 2 + B * Hq * S * 4
+    free, _ = torch.cuda.mem_get_info()
+    if free < need + (4 << 30):
+        pytest.skip("not enough device memory for the 2^31-element case")
+    g = torch.Generator(device=DEV).manual_seed(91)
+    q = torch.randn((B, S, Hq, D), generator=g, device=DEV, dtype=torch.bfloat16)
+    k = torch.randn((B, S, Hkv, D), generator=g, device=DEV, dtype=torch.bfloat16)
+    v = torch.randn((B, S, Hkv, D), generator=g, device=DEV, dtype=torch.bfloat16)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = attn.attention(q, k, v, scale=scale, causal=True)
+    torch.cuda.synchronize()
+    assert attn.device_status() == attn.ATTN_OK
+    rows = np.array([(0, h, i) for h in (0, 1, Hq - 2, Hq - 1)
+                     for i in (0, 1, 127, 128, S // 2, S - 129, S - 2, S - 1)], dtype=np.int64)
+    # the element offset of the last row's output is beyond 2^31
+    assert ((S - 1) * Hq + Hq - 1) * D >= 2 ** 31 - D
+    o_ref, lse_ref = oracle.attn_fwd(q.cpu(), k.cpu(), v.cpu(), scale=scale, causal=True,
+                                     rows=rows)
+    o_s = o[rows[:, 0], rows[:, 2], rows[:, 1]].float().cpu().numpy().astype(np.float64)
+    lse_s = lse[rows[:, 0], rows[:, 1], rows[:, 2]].cpu().numpy().astype(np.float64)
+    err = np.abs(o_s - o_ref)
+    assert err.max() <= O_MAX and err.mean() <= O_MEAN, (err.max(), err.mean())
+    assert np.abs(lse_s - lse_ref).max() <= LSE_TOL
+    # and the whole output is finite (nothing left unwritten or NaN)
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
