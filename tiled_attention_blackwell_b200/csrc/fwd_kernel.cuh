@@ -529,16 +529,19 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             tc_fence_after();
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 1);
 
-            // Scores of this row: two halves, the max of the first half overlaps
-            // the load of the second.
+            // Scores of this row: all four loads in flight together, one wait
+            // (measured slightly faster than overlapping the second half's
+            // load with the first half's max).
             uint32_t sr[kBlockN];
             tmem_ld32(s_tmem + 0, sr + 0);
             tmem_ld32(s_tmem + 32, sr + 32);
+            tmem_ld32(s_tmem + 64, sr + 64);
+            tmem_ld32(s_tmem + 96, sr + 96);
             tmem_wait_ld();
             reg_fence32(sr + 0);
             reg_fence32(sr + 32);
-            tmem_ld32(s_tmem + 64, sr + 64);
-            tmem_ld32(s_tmem + 96, sr + 96);
+            reg_fence32(sr + 64);
+            reg_fence32(sr + 96);
             float *s = reinterpret_cast<float *>(sr);
 
             const int key0 = j * kBlockN;
@@ -567,9 +570,6 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], s[e + u], s[e + 4 + u]);
 #pragma unroll
             for (int u = 0; u < 4; ++u) mx[u] = fmaxf(mx[u], s[kBlockN / 2 - 4 + u]);
-            tmem_wait_ld();
-            reg_fence32(sr + 64);
-            reg_fence32(sr + 96);
             if (MOD) {
 #pragma unroll
                 for (int e = kBlockN / 2; e < kBlockN; ++e)
