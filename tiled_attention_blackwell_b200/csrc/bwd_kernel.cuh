@@ -682,23 +682,10 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
         fence_mbar_init();
     }
     if (warp == kBwdLoadWarp) {
-        int lo = 0x7fffffff, hi = -1;
-        for (int t = lane; t < 128; t += 32) {
-            const int row = q0 + t;
-            if (row >= p.Sq) break;
-            const KeyRange r = row_key_range(p, row);
-            if (r.lo <= r.hi) {
-                lo = min(lo, r.lo);
-                hi = max(hi, r.hi);
-            }
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        }
+        const KeyRange kr = tile_key_range(p, q0, min(q0 + 127, p.Sq - 1), lane);
         if (lane == 0) {
-            sm.range[0] = hi < 0 ? 1 : lo / 128;
-            sm.range[1] = hi < 0 ? 0 : hi / 128;
+            sm.range[0] = kr.lo > kr.hi ? 1 : kr.lo / 128;
+            sm.range[1] = kr.lo > kr.hi ? 0 : kr.hi / 128;
         }
     }
     if (warp == kBwdMmaWarp) {

@@ -41,6 +41,33 @@ __device__ __forceinline__ KeyRange row_key_range(const Params &p, int row) {
     return {(int)lo, (int)hi};
 }
 
+// Union of the key intervals of rows [r0, r1] (r0 <= r1 < Sq), computed by
+// one whole warp; {1, 0} when no row has a key.  Every mask here is monotone
+// -- a row's interval never moves left as the row index grows, and the rows
+// with a key form one contiguous run -- so when the first and the last row
+// both have keys they bound the union; otherwise (a tile at the edge of the
+// rows that see any key) every row is visited.
+template <class Params>
+__device__ __forceinline__ KeyRange tile_key_range(const Params &p, int r0, int r1, int lane) {
+    const KeyRange a = row_key_range(p, r0);
+    const KeyRange z = row_key_range(p, r1);
+    if (a.lo <= a.hi && z.lo <= z.hi) return {a.lo, z.hi};
+    int lo = 0x7fffffff, hi = -1;
+    for (int row = r0 + lane; row <= r1; row += 32) {
+        const KeyRange r = row_key_range(p, row);
+        if (r.lo <= r.hi) {
+            lo = min(lo, r.lo);
+            hi = max(hi, r.hi);
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    if (hi < 0) return {1, 0};
+    return {lo, hi};
+}
+
 // Bounded wait.  Returns false when the CTA is aborting (own timeout or
 // another role's); `honor_abort` = false keeps waiting until the timeout only.
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,

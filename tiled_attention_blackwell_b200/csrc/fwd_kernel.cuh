@@ -270,27 +270,16 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
     if (warp == 9) {
         // Key-block range of each query tile: union of its rows' key ranges.
         for (int i = 0; i < 2; ++i) {
-            int lo = 0x7fffffff, hi = -1;
-            for (int t = lane; t < kBlockM; t += 32) {
-                const int row = q0 + i * kBlockM + t;
-                if (row >= p.Sq) break;
-                const KeyRange r = row_key_range(p, row);
-                if (r.lo <= r.hi) {
-                    lo = min(lo, r.lo);
-                    hi = max(hi, r.hi);
-                }
-            }
-            for (int o = 16; o > 0; o >>= 1) {
-                lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-                hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-            }
+            const int r0 = q0 + i * kBlockM;
+            KeyRange kr{1, 0};
+            if (r0 < p.Sq) kr = tile_key_range(p, r0, min(r0 + kBlockM - 1, p.Sq - 1), lane);
             if (lane == 0) {
-                if (hi < 0) {
+                if (kr.lo > kr.hi) {
                     sm.range[i][0] = 1;
                     sm.range[i][1] = 0;
                 } else {
-                    sm.range[i][0] = lo / kBlockN;
-                    sm.range[i][1] = hi / kBlockN;
+                    sm.range[i][0] = kr.lo / kBlockN;
+                    sm.range[i][1] = kr.hi / kBlockN;
                 }
             }
         }
