@@ -107,6 +107,28 @@ attn_status_t make_map(CUtensorMap *map, const void *base, int B, int S, int H, 
     return ATTN_OK;
 }
 
+// 5-D map of a bf16 [B][S][H][D] tensor whose box is a whole 128-row tile:
+// dims (64 columns, S, D/64 column chunks, H, B), box (64, 128, D/64, 1, 1),
+// so one copy fills the tile's D/64 chunks of [128 rows][128 bytes] (the
+// chunk dimension's stride, 128 bytes, is smaller than the row stride; the
+// copy is still one affine box).
+attn_status_t make_map_tile(CUtensorMap *map, const void *base, int B, int S, int H, int D) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[5] = {64, (cuuint64_t)S, (cuuint64_t)(D / 64), (cuuint64_t)H,
+                                (cuuint64_t)B};
+    const cuuint64_t strides[4] = {(cuuint64_t)H * D * 2, 128, (cuuint64_t)D * 2,
+                                   (cuuint64_t)S * H * D * 2};
+    const cuuint32_t box[5] = {64, (cuuint32_t)tab::kBlockM, (cuuint32_t)(D / 64), 1, 1};
+    const cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims,
+                    strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled (tile) failed (%d)", (int)r);
+    return ATTN_OK;
+}
+
 // --------------------------------------------------------------- launching
 
 template <int D, int NS, int EXP, int MOD = 0, int FP8 = 0>
@@ -491,10 +513,10 @@ attn_status_t attn_bwd_ex(const void *q, const void *k, const void *v, const voi
     if ((s = device_state(&st)) != ATTN_OK) return s;
     tab::BwdParams p;
     memset(&p, 0, sizeof p);
-    if ((s = make_map(&p.tm_q, q, B, Sq, Hq, D)) != ATTN_OK) return s;
-    if ((s = make_map(&p.tm_do, dout, B, Sq, Hq, D)) != ATTN_OK) return s;
-    if ((s = make_map(&p.tm_k, k, B, Sk, Hkv, D)) != ATTN_OK) return s;
-    if ((s = make_map(&p.tm_v, v, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    if ((s = make_map_tile(&p.tm_q, q, B, Sq, Hq, D)) != ATTN_OK) return s;
+    if ((s = make_map_tile(&p.tm_do, dout, B, Sq, Hq, D)) != ATTN_OK) return s;
+    if ((s = make_map_tile(&p.tm_k, k, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    if ((s = make_map_tile(&p.tm_v, v, B, Sk, Hkv, D)) != ATTN_OK) return s;
     p.o = static_cast<const __nv_bfloat16 *>(o);
     p.dout = static_cast<const __nv_bfloat16 *>(dout);
     p.lse = lse;

@@ -64,7 +64,7 @@ __device__ __forceinline__ void bwd_ex2_pair(float &y0, float &y1, float x0, flo
 }
 
 struct BwdParams {
-    CUtensorMap tm_q;   // bf16 [B][Sq][Hq][D], box (64, 128, 1, 1)
+    CUtensorMap tm_q;   // bf16 [B][Sq][Hq][D] as (64, Sq, D/64, Hq, B), box = one tile
     CUtensorMap tm_do;  // bf16 [B][Sq][Hq][D]
     CUtensorMap tm_k;   // bf16 [B][Sk][Hkv][D]
     CUtensorMap tm_v;
@@ -273,10 +273,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
             prefetch_tensormap(&p.tm_k);
             prefetch_tensormap(&p.tm_v);
             mbar_arrive_expect_tx(&sm.kv_full, 2 * kTileBytes);
-            for (int c = 0; c < Smem::kChunks; ++c) {
-                tma_load_4d(sm.k[c], &p.tm_k, &sm.kv_full, c * 64, k0, hkv, b);
-                tma_load_4d(sm.v[c], &p.tm_v, &sm.kv_full, c * 64, k0, hkv, b);
-            }
+            tma_load_5d(sm.k[0], &p.tm_k, &sm.kv_full, 0, k0, 0, hkv, b);
+            tma_load_5d(sm.v[0], &p.tm_v, &sm.kv_full, 0, k0, 0, hkv, b);
         }
         __syncwarp();
         bool ok = true;
@@ -336,13 +334,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
             if (lane < 2) {
                 // lane 0 copies the Q tile, lane 1 the dO tile, side by side
                 mbar_expect_tx(&sm.st_full[s], kTileBytes);
-                for (int c = 0; c < Smem::kChunks; ++c) {
-                    if (lane == 0)
-                        tma_load_4d(sm.q[s][c], &p.tm_q, &sm.st_full[s], c * 64, qb * 128, hq, b);
-                    else
-                        tma_load_4d(sm.dout[s][c], &p.tm_do, &sm.st_full[s], c * 64, qb * 128,
-                                    hq, b);
-                }
+                if (lane == 0)
+                    tma_load_5d(sm.q[s][0], &p.tm_q, &sm.st_full[s], 0, qb * 128, 0, hq, b);
+                else
+                    tma_load_5d(sm.dout[s][0], &p.tm_do, &sm.st_full[s], 0, qb * 128, 0, hq, b);
             }
             BWD_TRACE(1, it, 3);
 #pragma unroll
@@ -713,10 +708,8 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
             prefetch_tensormap(&p.tm_k);
             prefetch_tensormap(&p.tm_v);
             mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
-            for (int c = 0; c < Smem::kChunks; ++c) {
-                tma_load_4d(sm.q[c], &p.tm_q, &sm.q_full, c * 64, q0, hq, b);
-                tma_load_4d(sm.dout[c], &p.tm_do, &sm.q_full, c * 64, q0, hq, b);
-            }
+            tma_load_5d(sm.q[0], &p.tm_q, &sm.q_full, 0, q0, 0, hq, b);
+            tma_load_5d(sm.dout[0], &p.tm_do, &sm.q_full, 0, q0, 0, hq, b);
             int nk = 0, nv = 0;  // K and V copies issued
             bool ok = true;
             for (int t = 0; t < n_blocks && ok; ++t) {
@@ -725,15 +718,13 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
                                   abort_flag, p.status);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&sm.k_full[t % NK], kTileBytes);
-                for (int c = 0; c < Smem::kChunks; ++c)
-                    tma_load_4d(sm.k[t % NK][c], &p.tm_k, &sm.k_full[t % NK], c * 64, key0, hkv, b);
+                tma_load_5d(sm.k[t % NK][0], &p.tm_k, &sm.k_full[t % NK], 0, key0, 0, hkv, b);
                 ++nk;
                 ok = wait_bounded(&sm.v_empty[t % NV], ((uint32_t)(t / NV) & 1u) ^ 1u,
                                   abort_flag, p.status);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&sm.v_full[t % NV], kTileBytes);
-                for (int c = 0; c < Smem::kChunks; ++c)
-                    tma_load_4d(sm.v[t % NV][c], &p.tm_v, &sm.v_full[t % NV], c * 64, key0, hkv, b);
+                tma_load_5d(sm.v[t % NV][0], &p.tm_v, &sm.v_full[t % NV], 0, key0, 0, hkv, b);
                 ++nv;
             }
             // Copies still in flight land before the CTA can exit.
