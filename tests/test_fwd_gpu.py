@@ -312,3 +312,41 @@ def test_large_tensors_need_64bit_offsets():
     assert np.abs(lse_s - lse_ref).max() <= LSE_TOL
     # and the whole output is finite (nothing left unwritten or NaN)
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+def test_forward_and_backward_replay_in_a_cuda_graph():
+    """The entry points only enqueue work on the given stream, so a CUDA graph
+    captured around them replays the same results as eager calls."""
+    t = make_tensors(1, 4, 2, 700, 700, 128, seed=95, with_dout=True)
+    q, k, v, do = (t[n].to(DEV) for n in ("q", "k", "v", "dout"))
+    o = torch.empty_like(q)
+    lse = torch.empty((1, 4, 700), dtype=torch.float32, device=DEV)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=DEV)
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn.bwd_workspace_size(1, 4, 2, 700, 700, 128), dtype=torch.uint8,
+                     device=DEV)
+
+    def run(stream):
+        attn.attn_fwd(q, k, v, o, lse, scale=0.1, causal=True, stream=stream)
+        attn.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, scale=0.1, causal=True,
+                      stream=stream)
+
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        run(s)                      # eager: reference results
+    s.synchronize()
+    ref = [x.clone() for x in (o, lse, dq, dk, dv)]
+    for x in (o, lse, dq, dk, dv):
+        x.zero_()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run(s)
+    for x in (o, lse, dq, dk, dv):
+        x.zero_()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    for got, want in zip((o, lse, dq, dk, dv), ref):
+        assert torch.equal(got, want)
+    assert attn.device_status() == attn.ATTN_OK
