@@ -256,6 +256,44 @@ def oracle_sample(w, inputs, n_rows: int, seed: int = 0):
     return time.perf_counter() - t0, flops, oracle.num_threads()
 
 
+def oracle_bwd_sample(w, inputs, n_kv: int):
+    """Time the oracle backward on batch 0's first n_kv key/value heads (and
+    their query heads): a smaller problem of the same shape per head.
+    Returns (seconds, useful FLOPs by the 2.5x-forward convention, threads)."""
+    import oracle  # test infrastructure: only this leg of the benchmark loads it
+    g = w.Hq // w.Hkv
+    q = inputs["q"][:1, :, :n_kv * g].contiguous()
+    dout = inputs["dout"][:1, :, :n_kv * g].contiguous()
+    k = inputs["k"][:1, :, :n_kv].contiguous()
+    v = inputs["v"][:1, :, :n_kv].contiguous()
+    window = None if w.window == (-1, -1) else w.window
+    flops = 2.5 * useful_flops(1, n_kv * g, w.S, w.S, w.D, causal=w.causal,
+                               doc_offsets=inputs["doc_offsets"], window=w.window)
+    t0 = time.perf_counter()
+    oracle.attn_bwd(q, k, v, dout, scale=w.scale, causal=w.causal, window=window,
+                    doc_offsets=inputs["doc_offsets"])
+    return time.perf_counter() - t0, flops, oracle.num_threads()
+
+
+def kv_heads_for_seconds(w, inputs, seconds: float) -> int:
+    """Number of key/value heads of batch 0 the oracle backward covers in
+    about `seconds` (at least one, at most all of batch 0's)."""
+    t1, _, _ = oracle_bwd_sample(w, inputs, 1)
+    return int(min(max(1, seconds // max(t1, 1e-3)), w.Hkv))
+
+
+def metric_for(w, softcap=None, alibi=False) -> str:
+    if w.backward:
+        return f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()})"
+    if w.dtype == "fp8":
+        return f"attention fwd TFLOP/s and % of B200 FP8 tensor peak ({w.describe()})"
+    if w.name != HEADLINE or alibi or softcap is not None:
+        mods = "".join([f", softcap {softcap:g}" if softcap is not None else "",
+                        ", ALiBi" if alibi else ""])
+        return f"attention fwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()}{mods})"
+    return METRIC
+
+
 def rows_for_seconds(w, inputs, seconds: float) -> int:
     """Calibrate the row count so the oracle runs for about `seconds`.  Each
     call has a fixed cost (converting the inputs) besides the per-row work, so
@@ -459,16 +497,7 @@ def run_ours(args):
     # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s).
     peak_mult = 2.0 if fp8 else 1.0
     peak = float(peaks["bf16_tflops"]) * peak_mult
-    if w.backward:
-        metric = f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()})"
-    elif fp8:
-        metric = f"attention fwd TFLOP/s and % of B200 FP8 tensor peak ({w.describe()})"
-    elif w.name != HEADLINE or slopes is not None or args.softcap is not None:
-        mods = "".join([f", softcap {args.softcap:g}" if args.softcap is not None else "",
-                        ", ALiBi" if slopes is not None else ""])
-        metric = f"attention fwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()}{mods})"
-    else:
-        metric = METRIC
+    metric = metric_for(w, args.softcap, slopes is not None)
     result = {
         "metric": metric, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -493,13 +522,19 @@ def run_ours(args):
         "gpu_launches": args.steps * (3 if w.backward else 1),
         "clocks": sampler.summary(),
     }
-    if (rank == 0 and world == 1 and not args.no_cpu_baseline and not w.backward
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline
             and slopes is None and args.softcap is None):
-        n_rows = rows_for_seconds(w, inp, 15.0)
-        dt, fl, cores = oracle_sample(w, inp, n_rows)
-        result["cpu_baseline"] = {
-            "value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{n_rows} random (b, head, row) rows of {w.name}, fp64, {dt:.1f} s"}
+        if w.backward:
+            n_kv = kv_heads_for_seconds(w, inp, 15.0)
+            dt, fl, cores = oracle_bwd_sample(w, inp, n_kv)
+            sample = (f"backward of batch 0's first {n_kv} key/value heads of {w.name}, "
+                      f"fp64, {dt:.1f} s")
+        else:
+            n_rows = rows_for_seconds(w, inp, 15.0)
+            dt, fl, cores = oracle_sample(w, inp, n_rows)
+            sample = f"{n_rows} random (b, head, row) rows of {w.name}, fp64, {dt:.1f} s"
+        result["cpu_baseline"] = {"value": round(fl / dt / 1e12, 6), "unit": UNIT,
+                                  "cores": cores, "kind": "oracle", "sample": sample}
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -518,25 +553,32 @@ def run_reference(args):
     cfg = workload_config(w, inp["doc_offsets"])
     cfg["parallelism"] = "CPU oracle, rank 0 only"
     # each step: ~2 s of oracle work, so steps + warmup end within minutes
-    n_rows = rows_for_seconds(w, inp, 2.0)
+    if w.backward:
+        n_kv = kv_heads_for_seconds(w, inp, 2.0)
+        sample_fn = lambda i: oracle_bwd_sample(w, inp, n_kv)  # noqa: E731
+        sample = f"backward of batch 0's first {n_kv} key/value heads of {w.name} per step, fp64"
+    else:
+        n_rows = rows_for_seconds(w, inp, 2.0)
+        sample_fn = lambda i: oracle_sample(w, inp, n_rows, seed=i)  # noqa: E731
+        sample = f"{n_rows} random (b, head, row) rows of {w.name} per step, fp64"
     for i in range(args.warmup):
-        oracle_sample(w, inp, n_rows, seed=1000 + i)
+        sample_fn(1000 + i)
     times, fl_total, cores = [], 0.0, 1
     for i in range(args.steps):
-        dt, fl, cores = oracle_sample(w, inp, n_rows, seed=i)
+        dt, fl, cores = sample_fn(i)
         times.append(dt)
         fl_total += fl
     total = sum(times)
     value = fl_total / total / 1e12
     result = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "impl": "reference", "metric": metric_for(w), "value": round(value, 6), "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": cfg,
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
                          "kind": "oracle",
-                         "sample": f"{n_rows} random (b, head, row) rows of {w.name} per step, fp64"},
+                         "sample": sample},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
