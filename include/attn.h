@@ -74,7 +74,7 @@ typedef enum {
  * changes the mathematical result, only rounding. */
 typedef struct {
     /* Online-softmax rescale threshold in log2 units ("La ventaja técnica" of
-     * the ainvest.com FlashAttention-4 page: rescale only when the running
+     * "FlashAttention-4 de NVIDIA": rescale only when the running
      * maximum moves significantly).  The running max of a row, and with it
      * the output accumulator, is updated only when a new block raises the
      * row maximum by more than this amount; in between, unnormalised

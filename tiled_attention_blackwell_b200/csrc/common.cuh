@@ -102,7 +102,7 @@ __device__ __forceinline__ float tanh_full(float y) {
     return 1.0f - __fdividef(2.0f, e + 1.0f);
 }
 
-// Software 2^x for the FMA pipe ("La ventaja técnica", ainvest.com page:
+// Software 2^x for the FMA pipe ("FlashAttention-4 de NVIDIA", "La ventaja técnica":
 // part of the exponentials as a cubic on the CUDA cores): our minimax cubic
 // (exp2_poly.cuh, fitted by fit_exp2.py) with 2^round(x) applied through the
 // exponent field.

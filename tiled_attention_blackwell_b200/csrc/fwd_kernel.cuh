@@ -15,7 +15,7 @@
 //   warp  9     TMA producer (one thread)
 //   warps 10-11 idle
 // The pipeline stages load -> MMA -> softmax -> correction -> epilogue of the
-// FA4 design ("La ventaja técnica", ainvest.com page) map onto these roles;
+// FA4 design ("FlashAttention-4 de NVIDIA", "La ventaja técnica") map onto these roles;
 // the correction (rescaling the output accumulator in TMEM) runs inside the
 // softmax warps because threshold gating makes it rare.
 //
