@@ -119,3 +119,25 @@ def test_profiled_traffic_is_tied_to_the_kernel_sources(monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0000000000000000")
     assert bench.profiled_traffic("causal_s8192") is None
     assert bench.profiled_traffic("causal_s8192_fp8") is None
+
+
+def test_metric_names_per_workload():
+    assert bench.metric_for(WORKLOADS["causal_s8192"]) == bench.METRIC
+    assert "bwd" in bench.metric_for(WORKLOADS["causal_bwd_s4096"])
+    assert "FP8" in bench.metric_for(WORKLOADS["causal_s8192_fp8"])
+    assert "softcap 30" in bench.metric_for(WORKLOADS["causal_s8192"], softcap=30.0)
+    assert "ALiBi" in bench.metric_for(WORKLOADS["causal_s8192"], alibi=True)
+
+
+def test_oracle_backward_sample_counts_the_sliced_problem():
+    """The CPU backward sample runs batch 0's first n key/value heads; its
+    FLOPs are the 2.5x-forward count of exactly that slice."""
+    from tiled_attention_blackwell_b200.workloads import make_inputs
+    w = Workload("bwd_small", 2, 4, 2, 160, 64, True, seed=7, backward=True)
+    inp = make_inputs(w)
+    dt, fl, cores = bench.oracle_bwd_sample(w, inp, 1)
+    assert dt > 0 and cores >= 1
+    assert fl == 2.5 * useful_flops(1, 2, 160, 160, 64, causal=True)
+    n = bench.kv_heads_for_seconds(w, inp, 1e-9)
+    assert n == 1
+    assert bench.kv_heads_for_seconds(w, inp, 1e9) == w.Hkv
