@@ -29,6 +29,14 @@
 // bf16 tile stored as D/64 column chunks of [128 rows][128 bytes] with the
 // 128-byte swizzle that both TMA and the tcgen05 descriptors use.
 //
+// Template variants: EXP_MODE picks the MUFU / polynomial split of the
+// exponentials; MOD (bit 0 soft-cap, bit 1 ALiBi, "El FlexAttention de
+// PyTorch con FlashAttention-4", intro) transforms the scores into log2
+// units before the mask and the max; FP8 takes e4m3 Q, K, V (one 128-byte
+// chunk per row at D = 128, kind::f8f6f4 MMAs) and writes P as four e4m3
+// values per TMEM column ("Hardware-Aware FP4 FlashAttention-4",
+// "Precisión": the FP8 path).
+//
 // Online softmax in log2 units: x = s * scale * log2(e).  Each row keeps a
 // running max m and sum l; a new block changes m (and rescales O and l) only
 // when it raises the row max by more than `rescale_threshold` ("La ventaja
