@@ -150,3 +150,11 @@ def test_full_size_causal_backward_workload():
     dq, dk, dv, _, _ = oracle.attn_bwd(t["q"], t["k"], t["v"], t["dout"], scale=w.scale,
                                        causal=w.causal)
     check_grads(got, (dq, dk, dv), w.name)
+
+
+@pytest.mark.parametrize("case_kw", [dict(window=(64, 16)), dict(docs=[0, 1, 100, 333, 400]),
+                                     dict(causal=True, window=(200, 0))])
+def test_head_dim_64_masks(case_kw):
+    kw = dict(case_kw)
+    case(1, 4, 2, 400, 400, 64, seed=311, causal=kw.pop("causal", kw.get("docs") is not None),
+         **kw)

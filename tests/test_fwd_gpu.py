@@ -350,3 +350,11 @@ def test_forward_and_backward_replay_in_a_cuda_graph():
     for got, want in zip((o, lse, dq, dk, dv), ref):
         assert torch.equal(got, want)
     assert attn.device_status() == attn.ATTN_OK
+
+
+@pytest.mark.parametrize("Sq,Sk,window", [(1, 65536, None), (3, 70001, (4000, -1)),
+                                          (130, 65536, (1000, 0))])
+def test_decode_like_rows_against_long_key_sequences(Sq, Sk, window):
+    """Few query rows (bottom-right aligned) against tens of thousands of keys:
+    hundreds of key blocks per tile, ragged key tail."""
+    full_case(1, 4, 2, Sq, Sk, 128, seed=97, causal=True, window=window)
