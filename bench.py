@@ -63,9 +63,9 @@ def parse_args(argv=None):
     ap.add_argument("--exp2-mode", type=int, default=None)
     ap.add_argument("--rescale-threshold", type=float, default=None)
     ap.add_argument("--softcap", type=float, default=None,
-                    help="forward with the soft-capping score modifier (cap value)")
+                    help="time with the soft-capping score modifier (cap value)")
     ap.add_argument("--alibi", action="store_true",
-                    help="forward with ALiBi slopes 2^(-8(h+1)/Hq)")
+                    help="time with ALiBi slopes 2^(-8(h+1)/Hq)")
     return ap.parse_args(argv)
 
 
@@ -292,13 +292,13 @@ def kv_heads_for_seconds(w, inputs, seconds: float) -> int:
 
 
 def metric_for(w, softcap=None, alibi=False) -> str:
+    mods = "".join([f", softcap {softcap:g}" if softcap is not None else "",
+                    ", ALiBi" if alibi else ""])
     if w.backward:
-        return f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()})"
+        return f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()}{mods})"
     if w.dtype == "fp8":
         return f"attention fwd TFLOP/s and % of B200 FP8 tensor peak ({w.describe()})"
     if w.name != HEADLINE or alibi or softcap is not None:
-        mods = "".join([f", softcap {softcap:g}" if softcap is not None else "",
-                        ", ALiBi" if alibi else ""])
         return f"attention fwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()}{mods})"
     return METRIC
 
@@ -358,12 +358,19 @@ def run_ours(args):
     o = torch.empty(dev["q"].shape, dtype=torch.bfloat16, device=device)
     lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=device)
     window = None if w.window == (-1, -1) else w.window
+    slopes = None
+    if args.alibi:
+        slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / w.Hq) for h in range(w.Hq)],
+                              dtype=torch.float32, device=device)
+        cfg["alibi"] = "slopes 2^(-8(h+1)/Hq)"
     if w.backward:
-        # Backward workload: O and LSE come from one forward before timing;
-        # a step is one attn_bwd (preprocess, dK/dV and dQ kernels).
+        # Backward workload: O and LSE come from one forward (with the same
+        # score modifiers) before timing; a step is one attn_bwd (preprocess,
+        # dK/dV and dQ kernels).
         flops *= 2.5
         attn.attn_fwd(dev["q"], dev["k"], dev["v"], o, lse, scale=w.scale, causal=w.causal,
-                      window=window, doc_offsets=docs)
+                      window=window, doc_offsets=docs, softcap=args.softcap,
+                      alibi_slopes=slopes)
         host.update(o=o.cpu().pin_memory(), lse=lse.cpu().pin_memory(),
                     dout=inp["dout"].pin_memory())
         dev.update(o=o, lse=lse, dout=host["dout"].to(device))
@@ -378,11 +385,6 @@ def run_ours(args):
     flush = None if cfg["io_bytes"] > L2_BYTES else torch.empty(2 * L2_BYTES, dtype=torch.uint8,
                                                                  device=device)
     opts = None
-    slopes = None
-    if args.alibi:
-        slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / w.Hq) for h in range(w.Hq)],
-                              dtype=torch.float32, device=device)
-        cfg["alibi"] = "slopes 2^(-8(h+1)/Hq)"
     if args.softcap is not None:
         cfg["softcap"] = args.softcap
     if (args.exp2_mode is not None or args.rescale_threshold is not None
@@ -404,7 +406,7 @@ def run_ours(args):
         if w.backward:
             attn.attn_bwd(d["q"], d["k"], d["v"], d["o"], d["lse"], d["dout"], outs[0], outs[1],
                           outs[2], ws, scale=w.scale, causal=w.causal, window=window,
-                          doc_offsets=docs, stream=s)
+                          doc_offsets=docs, stream=s, softcap=args.softcap, alibi_slopes=slopes)
         elif fp8:
             attn.attn_fwd_fp8(d["q"], d["k"], d["v"], outs[0], outs[1],
                               q_descale=inp["q_descale"], k_descale=inp["k_descale"],
