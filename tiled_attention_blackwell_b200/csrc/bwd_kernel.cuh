@@ -93,25 +93,24 @@ struct BwdParams {
     const float *alibi_slopes;
 };
 
-// Modified score of one element in log2 units (MOD bit 0 soft-cap, bit 1
-// ALiBi at distance `dist` = i + (Sk - Sq) - j) and, in *dfac, its
-// derivative with respect to the scaled score scale * raw: 1 - tanh^2 under
-// the cap, else 1 (the ALiBi bias is constant).
+// Modified scores of a pair in log2 units (MOD bit 0 soft-cap, bit 1 ALiBi
+// at distances d0, d1 = i + (Sk - Sq) - j) and their derivatives with
+// respect to the scaled score scale * raw: 1 - tanh^2 = 4 r (1 - r) under
+// the cap (see softcap_pair), else 1 (the ALiBi bias is constant).
 template <int MOD>
-__device__ __forceinline__ float bwd_modified(float raw, float c, float softcap_in,
-                                              float softcap_out, float slope2, float dist,
-                                              float *dfac) {
-    float x;
+__device__ __forceinline__ void bwd_modified_pair(float &x0, float &x1, float &f0, float &f1,
+                                                  float raw0, float raw1, float c, float k1,
+                                                  float so, float slope2, float d0, float d1) {
     if (MOD & 1) {
-        const float t = tanh_full(raw * softcap_in);
-        x = softcap_out * t;
-        *dfac = fmaf(-t, t, 1.0f);
+        float r0, r1, m0, m1;
+        softcap_pair(x0, x1, r0, r1, raw0, raw1, k1, so);
+        mul2(m0, m1, r0, r1, 4.0f, 4.0f);
+        fma2(f0, f1, -m0, -m1, r0, r1, m0, m1);
     } else {
-        x = raw * c;
-        *dfac = 1.0f;
+        mul2(x0, x1, raw0, raw1, c, c);
+        f0 = f1 = 1.0f;
     }
-    if (MOD & 2) x = fmaf(-slope2, fabsf(dist), x);
-    return x;
+    if (MOD & 2) fma2(x0, x1, -slope2, -slope2, fabsf(d0), fabsf(d1), x0, x1);
 }
 
 // Opt-in event trace of the dK/dV kernel (compile with -DATTN_TRACE), same
@@ -487,21 +486,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
                 const int *rlo = sm.rlo[s] + h * 64;
                 const int *rhi = sm.rhi[s] + h * 64;
                 const float *l2 = sm.lse2[s] + h * 64;
+                const float k1 = p.softcap_in * (2.0f * kLog2e);
 #pragma unroll
                 for (int e = 0; e < 64; e += 2) {
-                    float pr[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int r = e + u;
-                        float dfac;
-                        const float x = bwd_modified<MOD>(pv[r], c, p.softcap_in, p.softcap_out,
-                                                          slope2, dist0 + (float)r, &dfac);
-                        const bool in = full || (rlo[r] <= key && key <= rhi[r]);
-                        const float pe = ex2_mufu(x - l2[r]);
-                        pr[u] = in ? pe : 0.0f;
-                        pv[r] = pr[u] * dfac;
-                    }
-                    pk[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+                    float x0, x1, f0, f1;
+                    bwd_modified_pair<MOD>(x0, x1, f0, f1, pv[e], pv[e + 1], c, k1,
+                                           p.softcap_out, slope2, dist0 + (float)e,
+                                           dist0 + (float)(e + 1));
+                    add2(x0, x1, x0, x1, -l2[e], -l2[e + 1]);
+                    const float p0 = ex2_mufu(x0), p1 = ex2_mufu(x1);
+                    const float pr0 = (full || (rlo[e] <= key && key <= rhi[e])) ? p0 : 0.0f;
+                    const float pr1 = (full || (rlo[e + 1] <= key && key <= rhi[e + 1])) ? p1 : 0.0f;
+                    mul2(pv[e], pv[e + 1], pr0, pr1, f0, f1);
+                    pk[e >> 1] = pack_bf16x2(pr0, pr1);
                 }
             } else if (full) {
 #pragma unroll
@@ -864,15 +861,19 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
             if (MOD) {
                 // pv becomes P * d(modified)/d(scaled), all dS needs.
                 const float dist0 = (float)(row + p.Sk - p.Sq - key0);
+                const float k1 = p.softcap_in * (2.0f * kLog2e);
 #pragma unroll
-                for (int e = 0; e < 64; ++e) {
+                for (int e = 0; e < 64; e += 2) {
+                    float x0, x1, f0, f1;
+                    bwd_modified_pair<MOD>(x0, x1, f0, f1, pv[e], pv[e + 1], c, k1,
+                                           p.softcap_out, slope2, dist0 - (float)e,
+                                           dist0 - (float)(e + 1));
+                    add2(x0, x1, x0, x1, -l2, -l2);
+                    float p0 = ex2_mufu(x0), p1 = ex2_mufu(x1);
+                    mul2(p0, p1, p0, p1, f0, f1);
                     const int key = key0 + e;
-                    float dfac;
-                    const float x = bwd_modified<MOD>(pv[e], c, p.softcap_in, p.softcap_out,
-                                                      slope2, dist0 - (float)e, &dfac);
-                    const bool in = !masked || (key >= kr.lo && key <= kr.hi);
-                    const float pe = ex2_mufu(x - l2) * dfac;
-                    pv[e] = in ? pe : 0.0f;
+                    pv[e] = (!masked || (key >= kr.lo && key <= kr.hi)) ? p0 : 0.0f;
+                    pv[e + 1] = (!masked || (key + 1 >= kr.lo && key + 1 <= kr.hi)) ? p1 : 0.0f;
                 }
             } else if (masked) {
 #pragma unroll

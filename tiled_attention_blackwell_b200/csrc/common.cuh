@@ -91,15 +91,22 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
 
 constexpr float kLog2eF = 1.4426950408889634f;
 
-// tanh to fp32 accuracy from the identity tanh(y) = 1 - 2 / (e^(2y) + 1):
-// one ex2 and one fast division (the MUFU tanh approximation is too coarse
-// for soft-capped logits: its error is multiplied by the cap).  |y| is
-// clamped to 20, where tanh is +-1 in fp32, so nothing overflows; a NaN
-// input stays NaN.
-__device__ __forceinline__ float tanh_full(float y) {
-    y = fminf(fmaxf(y, -20.0f), 20.0f);
-    const float e = ex2_mufu(y * 2.8853900817779268f);  // e^(2y), at most e^40
-    return 1.0f - __fdividef(2.0f, e + 1.0f);
+// Soft-capped scores of a pair, in log2 units: with u = e^(2y), y = raw *
+// scale / cap, tanh(y) = 1 - 2 / (u + 1), so cap * log2(e) * tanh(y) =
+// so - 2 so r with r = 1 / (u + 1).  k1 = 2 log2(e) scale / cap, so =
+// cap log2(e).  Two MUFU operations per score (ex2, rcp) and three packed
+// FMA-pipe operations per pair; u = inf gives r = 0 (tanh = 1), u = 0 gives
+// r = 1 (tanh = -1).  r is returned too: the backward's d tanh / dy =
+// 1 - tanh^2 = 4 r (1 - r).
+__device__ __forceinline__ void softcap_pair(float &x0, float &x1, float &r0, float &r1,
+                                             float raw0, float raw1, float k1, float so) {
+    float a0, a1;
+    mul2(a0, a1, raw0, raw1, k1, k1);
+    float u0 = ex2_mufu(a0), u1 = ex2_mufu(a1);
+    add2(u0, u1, u0, u1, 1.0f, 1.0f);
+    r0 = rcp_mufu(u0);
+    r1 = rcp_mufu(u1);
+    fma2(x0, x1, r0, r1, -2.0f * so, -2.0f * so, so, so);
 }
 
 // Software 2^x for the FMA pipe ("FlashAttention-4 de NVIDIA", "La ventaja técnica":

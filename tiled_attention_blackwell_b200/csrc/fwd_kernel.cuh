@@ -207,16 +207,27 @@ __device__ __forceinline__ float exp_pack_half_fp8(const float *s, float c, floa
     return (sum0 + sum1) + (sum2 + sum3);
 }
 
-// Score modifier, in log2 units: MOD bit 0 soft-cap, bit 1 ALiBi.  `raw` is
-// <q_i, k_j>; `dist` is i + (Sk - Sq) - j as a float.
-template <int MOD>
-__device__ __forceinline__ float modified_score(float raw, float c, float softcap_in,
-                                                float softcap_out, float slope2, float dist) {
-    float x;
-    if (MOD & 1) x = softcap_out * tanh_full(raw * softcap_in);
-    else x = raw * c;
-    if (MOD & 2) x = fmaf(-slope2, fabsf(dist), x);
-    return x;
+// Score modifiers of n consecutive scores (n even), in log2 units, in place:
+// MOD bit 0 soft-cap, bit 1 ALiBi.  v holds <q_i, k_j>; dist0 is
+// i + (Sk - Sq) - j of the first as a float.
+template <int MOD, int N>
+__device__ __forceinline__ void modify_scores(float *v, float c, float k1, float so,
+                                              float slope2, float dist0) {
+#pragma unroll
+    for (int e = 0; e < N; e += 2) {
+        float x0, x1;
+        if (MOD & 1) {
+            float r0, r1;
+            softcap_pair(x0, x1, r0, r1, v[e], v[e + 1], k1, so);
+        } else {
+            mul2(x0, x1, v[e], v[e + 1], c, c);
+        }
+        if (MOD & 2)
+            fma2(x0, x1, -slope2, -slope2, fabsf(dist0 - (float)e), fabsf(dist0 - (float)(e + 1)),
+                 x0, x1);
+        v[e] = x0;
+        v[e + 1] = x1;
+    }
 }
 
 template <int D, int NS, int EXP_MODE, int MOD = 0, int FP8 = 0>
@@ -512,6 +523,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         // the max, so the exponent step multiplies by 1 instead of c.
         const float c_exp = MOD ? 1.0f : c;
         const float slope2 = (MOD & 2) ? __ldg(p.alibi_slopes + hq) * kLog2eF : 0.0f;
+        const float k1 = p.softcap_in * (2.0f * kLog2eF);  // soft-cap: 2 log2(e) scale / cap
         const float diag_f = (float)(row + p.Sk - p.Sq);
         float m_run = -INFINITY;
         float l_run = 0.0f;
@@ -543,12 +555,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
 
             const int key0 = j * kBlockN;
             const float dist0 = diag_f - (float)key0;  // distance to key0 of this block
-            if (MOD) {
-#pragma unroll
-                for (int e = 0; e < kBlockN / 2; ++e)
-                    s[e] = modified_score<MOD>(s[e], c, p.softcap_in, p.softcap_out, slope2,
-                                               dist0 - (float)e);
-            }
+            if (MOD) modify_scores<MOD, kBlockN / 2>(s, c, k1, p.softcap_out, slope2, dist0);
             const bool need_mask = key0 < kr.lo || key0 + kBlockN - 1 > kr.hi;
             const bool masked = __any_sync(0xffffffffu, need_mask);
             if (masked) {
@@ -567,12 +574,9 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 for (int u = 0; u < 4; ++u) mx[u] = fmax3(mx[u], s[e + u], s[e + 4 + u]);
 #pragma unroll
             for (int u = 0; u < 4; ++u) mx[u] = fmaxf(mx[u], s[kBlockN / 2 - 4 + u]);
-            if (MOD) {
-#pragma unroll
-                for (int e = kBlockN / 2; e < kBlockN; ++e)
-                    s[e] = modified_score<MOD>(s[e], c, p.softcap_in, p.softcap_out, slope2,
-                                               dist0 - (float)e);
-            }
+            if (MOD)
+                modify_scores<MOD, kBlockN / 2>(s + kBlockN / 2, c, k1, p.softcap_out, slope2,
+                                                dist0 - (float)(kBlockN / 2));
             if (masked) {
 #pragma unroll
                 for (int e = kBlockN / 2; e < kBlockN; ++e) {

@@ -300,6 +300,13 @@ __device__ __forceinline__ float ex2_mufu(float x) {
     return y;
 }
 
+// Reciprocal on MUFU (rcp.approx: +inf -> +0).
+__device__ __forceinline__ float rcp_mufu(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Three-input max (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
