@@ -484,3 +484,35 @@ def test_fp8_row_subset_matches_full():
     for n, (b, h, i) in enumerate(rows):
         np.testing.assert_array_equal(o_r[n], o[b, i, h])
         assert lse_r[n] == lse[b, h, i]
+
+
+def test_fp8_path_equals_bf16_path_on_shared_values():
+    """e4m3 values are exact in bf16: with unit factors the fp8 oracle and the
+    bf16 oracle see identical numbers and must agree bit for bit."""
+    g = torch.Generator().manual_seed(24)
+    q8, _ = quantize_e4m3(torch.randn(1, 30, 2, 16, generator=g))
+    k8, _ = quantize_e4m3(torch.randn(1, 30, 2, 16, generator=g))
+    v8, _ = quantize_e4m3(torch.randn(1, 30, 2, 16, generator=g))
+    o8, l8 = oracle.attn_fwd_fp8(q8, k8, v8, q_descale=1.0, k_descale=1.0, v_descale=1.0,
+                                 scale=0.02, causal=True)
+    ob, lb = oracle.attn_fwd(q8.to(torch.bfloat16), k8.to(torch.bfloat16),
+                             v8.to(torch.bfloat16), scale=0.02, causal=True)
+    np.testing.assert_array_equal(o8, ob)
+    np.testing.assert_array_equal(l8, lb)
+
+
+def test_workload_fp8_quantization_is_within_e4m3_rounding():
+    """The fp8 workload generator: descale * code reproduces the fp32 draw to
+    e4m3's round-to-nearest precision (relative 2^-4 in the normal range,
+    absolute half a subnormal step below it), and the largest magnitude maps
+    to the largest code."""
+    from tiled_attention_blackwell_b200.workloads import quantize_e4m3 as wq
+    x = torch.randn(4096, generator=torch.Generator().manual_seed(25)) * 3
+    codes, descale = wq(x)
+    back = codes.to(torch.float64) * descale
+    xs = x.to(torch.float64) / descale
+    normal = xs.abs() >= 2.0 ** -6
+    rel = ((back / descale - xs).abs() / xs.abs())[normal]
+    assert float(rel.max()) <= 2.0 ** -4
+    assert float((back / descale - xs).abs()[~normal].max()) <= 2.0 ** -10
+    assert float(codes.to(torch.float32).abs().max()) == 448.0
