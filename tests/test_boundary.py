@@ -231,3 +231,35 @@ def test_fp8_invalid_arguments_rejected_before_launch(L, kw, status):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
 def test_valid_fp8_call_without_gpu_reports_cuda_error(L):
     assert call_fp8(L) == attn.ATTN_ERR_CUDA
+
+
+def test_option_structs_match_the_c_layout(tmp_path):
+    """The ctypes mirrors of attn_fwd_options_t / attn_bwd_options_t have the
+    C header's size and field offsets (compiled here with gcc)."""
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stddef.h>\n#include <stdio.h>\n#include "attn.h"\n'
+        "#define F(T, m) printf(#T \" \" #m \" %zu\\n\", offsetof(T, m))\n"
+        "int main(void) {\n"
+        '  printf("attn_fwd_options_t size %zu\\n", sizeof(attn_fwd_options_t));\n'
+        '  printf("attn_bwd_options_t size %zu\\n", sizeof(attn_bwd_options_t));\n'
+        "  F(attn_fwd_options_t, rescale_threshold); F(attn_fwd_options_t, exp2_mode);\n"
+        "  F(attn_fwd_options_t, wait_timeout_us); F(attn_fwd_options_t, debug_withhold_kv);\n"
+        "  F(attn_fwd_options_t, softcap); F(attn_fwd_options_t, reserved0);\n"
+        "  F(attn_fwd_options_t, alibi_slopes); F(attn_fwd_options_t, reserved);\n"
+        "  F(attn_bwd_options_t, softcap); F(attn_bwd_options_t, reserved0);\n"
+        "  F(attn_bwd_options_t, alibi_slopes); F(attn_bwd_options_t, reserved);\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)],
+                   check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    c = {}
+    for line in out.splitlines():
+        t, m, v = line.split()
+        c[(t, m)] = int(v)
+    for name, cls in (("attn_fwd_options_t", attn.FwdOptions), ("attn_bwd_options_t", attn.BwdOptions)):
+        assert c[(name, "size")] == ctypes.sizeof(cls), name
+        for field, _ in cls._fields_:
+            assert c[(name, field)] == getattr(cls, field).offset, (name, field)
