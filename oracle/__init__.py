@@ -57,6 +57,19 @@ def _load():
             lib.oracle_attn_fwd_e4m3.restype = ctypes.c_int
             lib.oracle_attn_fwd_e4m3.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_double] * 3 + \
                 [ctypes.c_void_p] * 2 + dims[:-2] + [ctypes.c_void_p, ctypes.c_int64]
+            lib.oracle_attn_fwd_fp4.restype = ctypes.c_int
+            lib.oracle_attn_fwd_fp4.argtypes = \
+                ([ctypes.c_void_p, ctypes.c_void_p, ctypes.c_double] * 3 + [ctypes.c_void_p] * 2
+                 + dims[:-2] + [ctypes.c_int, ctypes.c_void_p, ctypes.c_int64])
+            lib.oracle_direct_p_row.restype = ctypes.c_int
+            lib.oracle_direct_p_row.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                                ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_void_p, ctypes.c_void_p]
+            for name in ("oracle_e2m1_to_double", "oracle_ue8m0_to_double"):
+                getattr(lib, name).restype = ctypes.c_double
+                getattr(lib, name).argtypes = [ctypes.c_int]
+            lib.oracle_e2m1_round.restype = ctypes.c_double
+            lib.oracle_e2m1_round.argtypes = [ctypes.c_double]
             lib.oracle_e4m3_to_double.restype = ctypes.c_double
             lib.oracle_e4m3_to_double.argtypes = [ctypes.c_int]
             lib.oracle_num_threads.restype = ctypes.c_int
@@ -196,6 +209,86 @@ def attn_fwd_fp8(q, k, v, *, q_descale, k_descale, v_descale, scale, causal=Fals
                                   _ptr(offs), nd, _ptr(rows_a), n)
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd_e4m3 failed with code {rc}")
+    return o, lse
+
+
+_CLASSIFIERS = {"affine": 1, "exp2": 2}
+
+
+def e2m1_to_float(code: int) -> float:
+    """The value of one 4-bit E2M1 code (0..15, bit 3 = sign)."""
+    return float(_load().oracle_e2m1_to_double(int(code)))
+
+
+def ue8m0_to_float(u: int) -> float:
+    """The value of one UE8M0 scale byte: 2^(u - 127), NaN for 255."""
+    return float(_load().oracle_ue8m0_to_double(int(u)))
+
+
+def e2m1_round(x: float) -> float:
+    """x >= 0 rounded to the nearest E2M1 magnitude (ties to the even code),
+    saturating at 6."""
+    return float(_load().oracle_e2m1_round(float(x)))
+
+
+def direct_p_row(y, v, *, allow=None, classifier="affine"):
+    """Direct-P output and LSE of one row from its log2 scores y [n] and
+    value rows v [n, D] (allow: optional bool mask [n])."""
+    lib = _load()
+    y = np.ascontiguousarray(np.asarray(y, dtype=np.float64).reshape(-1))
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float64))
+    n, D = v.shape
+    if y.size != n:
+        raise ValueError("y and v disagree on the number of keys")
+    a = np.ones(n, dtype=np.uint8) if allow is None else \
+        np.ascontiguousarray(np.asarray(allow, dtype=bool).astype(np.uint8))
+    o = np.zeros(D)
+    lse = np.zeros(1)
+    rc = lib.oracle_direct_p_row(_ptr(y), _ptr(a), n, _ptr(v), D, _CLASSIFIERS[classifier],
+                                 _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise RuntimeError(f"oracle_direct_p_row failed with code {rc}")
+    return o, float(lse[0])
+
+
+def attn_fwd_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_codes,
+                 v_scales, v_global, *, scale, causal=False, window=None, doc_offsets=None,
+                 classifier="affine", rows=None):
+    """Direct-P forward in fp64 of NVFP4 Q/K and MXFP4 V.
+
+    q_codes [B,Sq,Hq,D/2], q_scales [B,Sq,Hq,D/16] (e4m3 bytes), likewise K;
+    v_codes [B,Sk,Hkv,D/2], v_scales [B,ceil(Sk/32),Hkv,D] (UE8M0 bytes); all
+    uint8.  classifier: "affine" or "exp2".  Shapes of the results as
+    attn_fwd."""
+    lib = _load()
+    qc, qs, kc, ks, vc, vs = (_as_codes(t) for t in (q_codes, q_scales, k_codes, k_scales,
+                                                     v_codes, v_scales))
+    B, Sq, Hq, Dh = qc.shape
+    Sk, Hkv = kc.shape[1], kc.shape[2]
+    D = 2 * Dh
+    if kc.shape != (B, Sk, Hkv, Dh) or vc.shape != kc.shape:
+        raise ValueError("code tensors disagree in shape")
+    if qs.shape != (B, Sq, Hq, D // 16) or ks.shape != (B, Sk, Hkv, D // 16):
+        raise ValueError("NVFP4 scales must be [B, S, H, D/16]")
+    if vs.shape != (B, (Sk + 31) // 32, Hkv, D):
+        raise ValueError("MXFP4 scales of V must be [B, ceil(Sk/32), Hkv, D]")
+    causal_i, wl, wr, offs, nd = _mask_args(causal, window, doc_offsets)
+    if rows is None:
+        o = np.zeros((B, Sq, Hq, D), dtype=np.float64)
+        lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+        rows_a, n = None, 0
+    else:
+        rows_a = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+        n = rows_a.shape[0]
+        o = np.zeros((n, D), dtype=np.float64)
+        lse = np.zeros((n,), dtype=np.float64)
+    rc = lib.oracle_attn_fwd_fp4(_ptr(qc), _ptr(qs), float(q_global), _ptr(kc), _ptr(ks),
+                                 float(k_global), _ptr(vc), _ptr(vs), float(v_global),
+                                 _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, float(scale),
+                                 causal_i, wl, wr, _ptr(offs), nd, _CLASSIFIERS[classifier],
+                                 _ptr(rows_a), n)
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_fp4 failed with code {rc}")
     return o, lse
 
 

@@ -40,8 +40,11 @@
  * one dominant logit -> that V row, constant V -> rows of P sum to one,
  * causal row 0), library softmax / logsumexp on dense masked scores, mask
  * and GQA invariants, finite differences for the backward; the e4m3 decoder
- * against torch's float8_e4m3fn conversion for all 256 codes.  Nothing here
- * is "parity unpinned".
+ * against torch's float8_e4m3fn conversion for all 256 codes; for the FP4
+ * Direct-P forward, the E2M1 table, brute-force nearest rounding, hand-worked
+ * constant-score rows, exact agreement with the softmax for scores on the
+ * E2M1 grid, integer-shift invariance, masking and the NVFP4 / MXFP4
+ * decoding.  Nothing here is "parity unpinned".
  *
  * Layouts (row-major, contiguous):
  *   q, o, dq, do : [B, Sq, Hq,  D]
@@ -67,6 +70,10 @@ typedef struct {
     int num_docs;
     double softcap;             /* > 0: scores pass through softcap * tanh(s / softcap) */
     const double *alibi_slopes; /* host double[Hq] or NULL */
+    /* 0: the exact softmax.  1, 2: Direct-P probabilities (affine or
+     * exponential classifier, see direct_p_row); `scale` then maps the dot
+     * product to log2 units. */
+    int direct_p;
 } oracle_shape_t;
 
 /* ------------------------------------------------------------------ input */
@@ -151,6 +158,10 @@ static double score_grad(const oracle_shape_t *s, double dot) {
     return s->scale;
 }
 
+static void direct_p_row(const double *y, const unsigned char *allow, long n,
+                         const double *vd, int D, int classifier, double *o_out,
+                         double *lse_out);
+
 static void forward_row(const oracle_shape_t *s, int hq, const double *qi,
                         const double *kd, const double *vd, long i,
                         double *srow, unsigned char *allow,
@@ -167,6 +178,10 @@ static void forward_row(const oracle_shape_t *s, int hq, const double *qi,
         srow[j] = modified_score(s, hq, i, j, dot);
         if (srow[j] > M) M = srow[j];
         ++n_allowed;
+    }
+    if (s->direct_p) {
+        direct_p_row(srow, allow, Sk, vd, D, s->direct_p, o_out, lse_out);
+        return;
     }
     for (int d = 0; d < D; ++d) o_out[d] = 0.0;
     if (n_allowed == 0) {
@@ -429,6 +444,198 @@ int oracle_attn_fwd_e4m3(const uint8_t *q, const uint8_t *k, const uint8_t *v,
     double *qd = decode_e4m3(q, nq, q_descale);
     double *kd = decode_e4m3(k, nkv, k_descale);
     double *vd = decode_e4m3(v, nkv, v_descale);
+    int status = -2;
+    if (qd && kd && vd) status = attn_fwd_core(&s, qd, kd, vd, 0, o, lse, rows, n_rows);
+    free(qd);
+    free(kd);
+    free(vd);
+    return status;
+}
+
+/* ------------------------------------------- FP4 inputs, Direct-P forward
+ * "Hardware-Aware FP4 FlashAttention-4", "Metodología", item 1 (Direct-P):
+ * Q and K arrive in NVFP4, V in MXFP4, and the probabilities P are built as
+ * MXFP4 values -- E2M1 codes with one power-of-two scale per 32 keys --
+ * straight from the normalised log2 scores; the softmax normaliser is the
+ * sum of exactly those represented values ("consistent normalisation"), so
+ * numerator and denominator describe the same approximate operator.
+ *
+ * Formats (from their definitions):
+ *   E2M1 (4 bits): bit 3 sign, bits 2-1 exponent with bias 1, bit 0
+ *     mantissa; exponent field 0 holds the subnormal m * 0.5.  The eight
+ *     magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ *   NVFP4: one e4m3 scale per 16 consecutive elements of a row (along D)
+ *     times a per-tensor fp32 factor: x = g * e4m3(scale) * e2m1(code).
+ *   MXFP4: one UE8M0 scale (2^(u - 127), u = 255 is NaN) per 32 elements:
+ *     here 32 consecutive keys of one (batch, head, d) column of V, the
+ *     contraction direction of PV, times a per-tensor factor.
+ *   Two codes per byte, element 2j in the low nibble.
+ *
+ * The Direct-P probabilities of one row (readings where the page is silent,
+ * listed in the design notes):
+ *   y_j        = log2-unit score of key j (the page's normalised log score;
+ *                the anchor it is measured from cancels out, see below);
+ *   block      = keys [32 g, 32 g + 32), aligned to the key index, the
+ *                32-key producer fragments the page pairs with MXFP4;
+ *   E_g        = floor(max_{j in block, allowed} y_j) - 2: the OCP MX rule
+ *                (shared exponent = floor(log2 amax) - 2 for E2M1), which
+ *                puts the block maximum at 2^(y - E) in [4, 8);
+ *   code_j     = the E2M1 magnitude chosen for r_j = y_j - E_g:
+ *                affine classifier (the page's fast path): index
+ *                clamp(rint(2 r + 2), 0, 7) -- the line through the
+ *                half-octave grid on which the magnitudes 1, 2, 4 sit at
+ *                indices 2, 4, 6 -- decoded as an E2M1 magnitude;
+ *                exponential classifier (the page's "native exponentials"):
+ *                2^r rounded to the nearest E2M1 magnitude, ties to the even
+ *                code, saturating at 6;
+ *   w_j        = code_j * 2^E_g (0 for masked keys);
+ *   l          = sum_j w_j;  O = sum_j w_j v_j / l;  LSE = ln(l) (natural
+ *                units: w_j approximates 2^y_j = e^s_j).
+ * Shifting every y of a row by an integer changes every E_g by the same
+ * integer and no code, so the result does not depend on which integer
+ * anchor the scores are measured from; the range guard of the page (an
+ * anchor that keeps the block scales in range) is therefore exact here and
+ * this function works with the row maximum's floor only to keep doubles in
+ * range. */
+static const double kE2m1Mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+static double e2m1_to_double(unsigned c) {
+    const unsigned e = (c >> 1) & 3u, m = c & 1u;
+    const double mag = e == 0 ? 0.5 * (double)m : ldexp(1.0 + 0.5 * (double)m, (int)e - 1);
+    return (c & 8u) ? -mag : mag;
+}
+
+static double ue8m0_to_double(uint8_t u) { return u == 255 ? NAN : ldexp(1.0, (int)u - 127); }
+
+/* Round x >= 0 to the nearest E2M1 magnitude (ties to the even code index),
+ * saturating at 6; returns the magnitude. */
+static double e2m1_round(double x) {
+    if (!(x < 6.0)) return 6.0;
+    int k = 0;
+    while (k < 7 && kE2m1Mag[k + 1] <= x) ++k; /* kE2m1Mag[k] <= x < kE2m1Mag[k+1] */
+    const double lo = kE2m1Mag[k], hi = kE2m1Mag[k + 1], mid = 0.5 * (lo + hi);
+    if (x < mid) return lo;
+    if (x > mid) return hi;
+    return (k & 1) ? hi : lo;
+}
+
+static double direct_p_code(double r, int classifier) {
+    if (classifier == 2) return e2m1_round(exp2(r));
+    double t = nearbyint(2.0 * r + 2.0);
+    if (!(t > 0.0)) t = 0.0; /* also r = -inf */
+    if (t > 7.0) t = 7.0;
+    return kE2m1Mag[(int)t];
+}
+
+static void direct_p_row(const double *y, const unsigned char *allow, long n,
+                         const double *vd, int D, int classifier, double *o_out,
+                         double *lse_out) {
+    double M = -INFINITY;
+    for (long j = 0; j < n; ++j)
+        if (allow[j] && y[j] > M) M = y[j];
+    for (int d = 0; d < D; ++d) o_out[d] = 0.0;
+    if (M == -INFINITY) {
+        *lse_out = -INFINITY;
+        return;
+    }
+    const double Mi = floor(M);
+    double l = 0.0;
+    for (long g0 = 0; g0 < n; g0 += 32) {
+        const long g1 = g0 + 32 < n ? g0 + 32 : n;
+        double bmax = -INFINITY;
+        for (long j = g0; j < g1; ++j)
+            if (allow[j] && y[j] > bmax) bmax = y[j];
+        if (bmax == -INFINITY) continue;
+        const double E = floor(bmax) - 2.0;
+        for (long j = g0; j < g1; ++j) {
+            if (!allow[j]) continue;
+            const double w = ldexp(direct_p_code(y[j] - E, classifier), (int)(E - Mi));
+            if (w == 0.0) continue;
+            l += w;
+            const double *vj = vd + (size_t)j * D;
+            for (int d = 0; d < D; ++d) o_out[d] += w * vj[d];
+        }
+    }
+    for (int d = 0; d < D; ++d) o_out[d] /= l;
+    *lse_out = log(2.0) * (Mi + log2(l));
+}
+
+double oracle_e2m1_to_double(int code) { return e2m1_to_double((unsigned)code & 15u); }
+double oracle_ue8m0_to_double(int u) { return ue8m0_to_double((uint8_t)u); }
+double oracle_e2m1_round(double x) { return e2m1_round(x); }
+
+/* One Direct-P row on given log2 scores y[n] (allow[n] != 0 marks the
+ * allowed keys) and value rows v[n][D]. */
+int oracle_direct_p_row(const double *y, const unsigned char *allow, int64_t n,
+                        const double *v, int D, int classifier, double *o, double *lse) {
+    if (n < 1 || D < 1 || (classifier != 1 && classifier != 2)) return -1;
+    direct_p_row(y, allow, (long)n, v, D, classifier, o, lse);
+    return 0;
+}
+
+/* NVFP4 tensor of n elements (rows of D, D a multiple of 16) to doubles,
+ * times `mul`. */
+static double *decode_nvfp4(const uint8_t *codes, const uint8_t *scales, size_t n,
+                            double mul) {
+    double *d = (double *)malloc((n ? n : 1) * sizeof(double));
+    if (!d) return NULL;
+    for (size_t t = 0; t < n; ++t) {
+        const unsigned c = (codes[t / 2] >> (4 * (t & 1))) & 15u;
+        d[t] = mul * e4m3_to_double(scales[t / 16]) * e2m1_to_double(c);
+    }
+    return d;
+}
+
+/* MXFP4 V [B][Sk][H][D] with scales [B][ceil(Sk/32)][H][D] to doubles. */
+static double *decode_mxfp4_v(const uint8_t *codes, const uint8_t *scales, int B, int Sk,
+                              int H, int D, double mul) {
+    const size_t n = (size_t)B * Sk * H * D;
+    const int nblk = (Sk + 31) / 32;
+    double *d = (double *)malloc((n ? n : 1) * sizeof(double));
+    if (!d) return NULL;
+    for (size_t t = 0; t < n; ++t) {
+        const size_t row = t / (size_t)D;
+        const int dd = (int)(t % (size_t)D);
+        const int h = (int)(row % (size_t)H);
+        const int j = (int)((row / (size_t)H) % (size_t)Sk);
+        const int b = (int)(row / ((size_t)H * Sk));
+        const uint8_t u = scales[(((size_t)b * nblk + j / 32) * H + h) * D + dd];
+        const unsigned c = (codes[t / 2] >> (4 * (t & 1))) & 15u;
+        d[t] = mul * ue8m0_to_double(u) * e2m1_to_double(c);
+    }
+    return d;
+}
+
+/*
+ * Direct-P forward of NVFP4 Q/K and MXFP4 V.  classifier 1 = affine,
+ * 2 = exponential.  The log2 score is <q', k'> * c with q', k' decoded
+ * without their per-tensor factors and c = fp32(scale * q_global *
+ * k_global * log2 e): the code decisions are taken on that value, the
+ * precision in which the kernel takes them.  O includes v_global; LSE is in
+ * natural units of the scores scale * <q, k>.  Layouts as the kernel's:
+ * codes [B][S][H][D/2], Q/K scales [B][S][H][D/16], V scales
+ * [B][ceil(Sk/32)][Hkv][D].
+ */
+int oracle_attn_fwd_fp4(const uint8_t *q_codes, const uint8_t *q_scales, double q_global,
+                        const uint8_t *k_codes, const uint8_t *k_scales, double k_global,
+                        const uint8_t *v_codes, const uint8_t *v_scales, double v_global,
+                        double *o, double *lse, int B, int Hq, int Hkv, int Sq, int Sk,
+                        int D, double scale, int causal, int window_left, int window_right,
+                        const int *doc_offsets, int num_docs, int classifier,
+                        const int64_t *rows, int64_t n_rows) {
+    if (classifier != 1 && classifier != 2) return -1;
+    if (D % 32 != 0) return -1;
+    const double softcap = 0.0;
+    const double *alibi_slopes = NULL;
+    const double c = (double)(float)(scale * q_global * k_global * 1.4426950408889634);
+    ORACLE_SHAPE;
+    s.scale = c;
+    s.direct_p = classifier;
+    if (!shape_ok(&s)) return -1;
+    const size_t nq = (size_t)B * Sq * Hq * D, nkv = (size_t)B * Sk * Hkv * D;
+    double *qd = decode_nvfp4(q_codes, q_scales, nq, 1.0);
+    double *kd = decode_nvfp4(k_codes, k_scales, nkv, 1.0);
+    double *vd = decode_mxfp4_v(v_codes, v_scales, B, Sk, Hkv, D, v_global);
     int status = -2;
     if (qd && kd && vd) status = attn_fwd_core(&s, qd, kd, vd, 0, o, lse, rows, n_rows);
     free(qd);

@@ -16,7 +16,19 @@ Recipe (all on the CPU, deterministic):
     sequence; the last document is clipped to what is left;
   * fp8 workloads draw the same fp32 tensors and quantise each one to e4m3
     with one per-tensor factor, descale = max|x| / 448 (torch's
-    round-to-nearest conversion of x / descale).
+    round-to-nearest conversion of x / descale);
+  * fp4 workloads draw the same fp32 tensors and encode Q and K as NVFP4
+    (E2M1 codes, one e4m3 scale per 16 elements of a row, one fp32 factor
+    per tensor) and V as MXFP4 (E2M1 codes, one power-of-two scale per 32
+    keys of each (batch, head, d) column, the OCP rule 2^(floor(log2 amax)
+    - 2)).  Codes are the nearest E2M1 magnitude (ties to the even code,
+    saturating at 6).  With ``pow2_scales`` the NVFP4 block scales are the
+    power of two 2^ceil(log2(amax / 6)) and K's per-tensor factor is chosen
+    so that scale * q_global * k_global * log2(e) is a power of two: every
+    score is then an exact dyadic number, so the fp32 dot products of the
+    kernel and the fp64 ones of the oracle agree bit for bit and the
+    quantised decisions on them can be compared exactly.  Otherwise the
+    NVFP4 scales are e4m3(amax / (6 g)) with g = max|x| / (6 * 448).
 No public dataset or benchmark suite stands behind these shapes; the pages
 measure on none that could be used here, so synthetic inputs of the named
 shapes stand in.
@@ -47,7 +59,7 @@ class Workload:
     doc_lengths: Optional[tuple] = None  # (lo, hi) inclusive, or None
     backward: bool = False
     window: tuple = (-1, -1)
-    dtype: str = "bf16"  # "bf16" or "fp8" (e4m3 Q, K, V with per-tensor factors)
+    dtype: str = "bf16"  # "bf16", "fp8" (e4m3 Q, K, V) or "fp4" (NVFP4 Q/K, MXFP4 V)
 
     @property
     def scale(self) -> float:
@@ -78,6 +90,10 @@ WORKLOADS = {
     # The headline shape with e4m3 inputs (the low-precision forward).
     "causal_s8192_fp8": Workload("causal_s8192_fp8", 2, 16, 16, 8192, 128, True, seed=3,
                                  dtype="fp8"),
+    # The headline shape in FP4 (NVFP4 Q/K with power-of-two block scales,
+    # MXFP4 V), for the Direct-P forward.
+    "causal_s8192_fp4": Workload("causal_s8192_fp4", 2, 16, 16, 8192, 128, True, seed=3,
+                                 dtype="fp4"),
 }
 
 HEADLINE = "causal_s8192"
@@ -134,10 +150,98 @@ def make_tensors_fp8(B, Hq, Hkv, Sq, Sk, D, seed, *, qk_std=1.0, v_std=1.0):
     return out
 
 
+_E2M1_MIDPOINTS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def e2m1_encode(x: np.ndarray) -> np.ndarray:
+    """4-bit E2M1 codes of x (bit 3 = sign): the nearest of the magnitudes
+    0, 0.5, 1, 1.5, 2, 3, 4, 6, ties to the even code, saturating at 6."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    idx = np.searchsorted(_E2M1_MIDPOINTS, a, side="left")
+    tie = (idx < 7) & (a == _E2M1_MIDPOINTS[np.minimum(idx, 6)])
+    idx = idx + (tie & (idx % 2 == 1))
+    return (idx | np.where(np.signbit(x) & (idx > 0), 8, 0)).astype(np.uint8)
+
+
+def _pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """[..., D] 4-bit codes -> [..., D/2] bytes, element 2j in the low nibble."""
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def quantize_nvfp4(x: torch.Tensor, *, pow2_scales: bool, global_scale=None):
+    """NVFP4 encoding of x [..., D] along its last dimension: (codes uint8
+    [..., D/2], e4m3 scale bytes uint8 [..., D/16], per-tensor factor g) with
+    x ~= g * scale * e2m1(code)."""
+    xf = x.double().numpy()
+    if global_scale is None:
+        amax = float(np.abs(xf).max())
+        global_scale = 1.0 if pow2_scales else (amax / (6.0 * 448.0) if amax > 0 else 1.0)
+    blocks = xf.reshape(*xf.shape[:-1], -1, 16) / global_scale
+    bmax = np.abs(blocks).max(axis=-1)
+    if pow2_scales:
+        e = np.ceil(np.log2(np.where(bmax > 0, bmax / 6.0, 1.0)))
+        scale = np.exp2(np.clip(e, -9, 8))
+    else:
+        scale = torch.from_numpy(np.where(bmax > 0, bmax / 6.0, 1.0)).float() \
+            .to(torch.float8_e4m3fn).float().double().numpy()
+    scale_bytes = torch.from_numpy(scale).float().to(torch.float8_e4m3fn).view(torch.uint8)
+    codes = e2m1_encode(blocks / scale[..., None]).reshape(xf.shape)
+    return (torch.from_numpy(_pack_nibbles(codes)), scale_bytes.reshape(*xf.shape[:-1], -1),
+            float(global_scale))
+
+
+def quantize_mxfp4_keys(x: torch.Tensor):
+    """MXFP4 encoding of V [B, S, H, D] with one UE8M0 scale per 32 keys of
+    each (b, h, d) column: (codes uint8 [B, S, H, D/2], scale bytes uint8
+    [B, ceil(S/32), H, D])."""
+    xf = x.double().numpy()
+    B, S, H, D = xf.shape
+    nblk = (S + 31) // 32
+    pad = np.zeros((B, nblk * 32, H, D))
+    pad[:, :S] = xf
+    blocks = pad.reshape(B, nblk, 32, H, D)
+    amax = np.abs(blocks).max(axis=2)
+    e = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2, 0)
+    e = np.clip(e, -127, 127)
+    codes = e2m1_encode(blocks / np.exp2(e)[:, :, None]).reshape(B, nblk * 32, H, D)[:, :S]
+    return (torch.from_numpy(_pack_nibbles(codes)),
+            torch.from_numpy((e + 127).astype(np.uint8)))
+
+
+def fp4_k_global(scale: float) -> float:
+    """K's per-tensor factor that makes scale * k_global * log2(e) (with
+    q_global = 1) the power of two just below scale * log2(e)."""
+    c = scale * 1.4426950408889634
+    return 2.0 ** math.floor(math.log2(c)) / c
+
+
+def make_tensors_fp4(B, Hq, Hkv, Sq, Sk, D, seed, *, scale=None, pow2_scales=True,
+                     qk_std=1.0, v_std=1.0):
+    """NVFP4 Q/K and MXFP4 V (CPU uint8 tensors and per-tensor factors) from
+    the fp32 draws of make_tensors (order Q, K, V)."""
+    g = torch.Generator().manual_seed(int(seed))
+    q = torch.randn((B, Sq, Hq, D), generator=g, dtype=torch.float32) * qk_std
+    k = torch.randn((B, Sk, Hkv, D), generator=g, dtype=torch.float32) * qk_std
+    v = torch.randn((B, Sk, Hkv, D), generator=g, dtype=torch.float32) * v_std
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out = {}
+    out["q_codes"], out["q_scales"], out["q_global"] = quantize_nvfp4(
+        q, pow2_scales=pow2_scales, global_scale=1.0 if pow2_scales else None)
+    kg = fp4_k_global(scale) if pow2_scales else None
+    out["k_codes"], out["k_scales"], out["k_global"] = quantize_nvfp4(
+        k, pow2_scales=pow2_scales, global_scale=kg)
+    out["v_codes"], out["v_scales"] = quantize_mxfp4_keys(v)
+    out["v_global"] = 1.0
+    return out
+
+
 def make_inputs(w: Workload):
     """All inputs of a named workload (CPU tensors) plus its mask arguments."""
     if w.dtype == "fp8":
         t = make_tensors_fp8(w.B, w.Hq, w.Hkv, w.S, w.S, w.D, w.seed, qk_std=w.qk_std)
+    elif w.dtype == "fp4":
+        t = make_tensors_fp4(w.B, w.Hq, w.Hkv, w.S, w.S, w.D, w.seed, qk_std=w.qk_std)
     else:
         t = make_tensors(w.B, w.Hq, w.Hkv, w.S, w.S, w.D, w.seed, qk_std=w.qk_std,
                          k_outlier_frac=w.k_outlier_frac, k_outlier_mult=w.k_outlier_mult,
