@@ -46,7 +46,9 @@ KERNEL_SOURCES = ["tiled_attention_blackwell_b200/csrc/fwd_kernel.cuh",
                   "tiled_attention_blackwell_b200/csrc/common.cuh",
                   "tiled_attention_blackwell_b200/csrc/ptx.cuh",
                   "tiled_attention_blackwell_b200/csrc/exp2_poly.cuh",
+                  "tiled_attention_blackwell_b200/csrc/fp4_dequant.cuh",
                   "tiled_attention_blackwell_b200/csrc/attn_api.cu"]
+FP4_INPUTS = ("q_codes", "q_scales", "k_codes", "k_scales", "v_codes", "v_scales")
 
 
 # ------------------------------------------------------------------ helpers
@@ -66,6 +68,8 @@ def parse_args(argv=None):
                     help="time with the soft-capping score modifier (cap value)")
     ap.add_argument("--alibi", action="store_true",
                     help="time with ALiBi slopes 2^(-8(h+1)/Hq)")
+    ap.add_argument("--classifier", default="affine", choices=["affine", "exp2"],
+                    help="Direct-P code classifier of the fp4 workloads")
     return ap.parse_args(argv)
 
 
@@ -259,6 +263,13 @@ def oracle_sample(w, inputs, n_rows: int, seed: int = 0):
                             q_descale=inputs["q_descale"], k_descale=inputs["k_descale"],
                             v_descale=inputs["v_descale"], scale=w.scale, causal=w.causal,
                             window=window, doc_offsets=inputs["doc_offsets"], rows=rows)
+    elif w.dtype == "fp4":
+        oracle.attn_fwd_fp4(*[inputs[n] for n in ("q_codes", "q_scales", "q_global", "k_codes",
+                                                  "k_scales", "k_global", "v_codes", "v_scales",
+                                                  "v_global")],
+                            scale=w.scale, causal=w.causal, window=window,
+                            doc_offsets=inputs["doc_offsets"], rows=rows,
+                            classifier=inputs.get("classifier", "affine"))
     else:
         oracle.attn_fwd(inputs["q"], inputs["k"], inputs["v"], scale=w.scale, causal=w.causal,
                         window=window, doc_offsets=inputs["doc_offsets"], rows=rows)
@@ -291,9 +302,13 @@ def kv_heads_for_seconds(w, inputs, seconds: float) -> int:
     return int(min(max(1, seconds // max(t1, 1e-3)), w.Hkv))
 
 
-def metric_for(w, softcap=None, alibi=False) -> str:
+def metric_for(w, softcap=None, alibi=False, classifier="affine") -> str:
     mods = "".join([f", softcap {softcap:g}" if softcap is not None else "",
                     ", ALiBi" if alibi else ""])
+    if w.dtype == "fp4":
+        # f16 operands on the tensor cores: the same dense peak as bf16
+        return (f"attention fwd TFLOP/s and % of B200 BF16/F16 tensor peak ({w.describe()}, "
+                f"Direct-P {classifier} classifier)")
     if w.backward:
         return f"attention bwd TFLOP/s and % of B200 BF16 tensor peak ({w.describe()}{mods})"
     if w.dtype == "fp8":
@@ -325,9 +340,14 @@ def workload_config(w, doc_offsets):
     if tuple(w.window) != (-1, -1):
         cfg["mask"] = "causal sliding window" if w.causal else "sliding window"
         cfg["window"] = list(w.window)
-    eb = 1 if w.dtype == "fp8" else 2  # bytes per Q/K/V element; O is bf16
-    io_bytes = (eb * (w.B * w.S * w.Hq * w.D + 2 * w.B * w.S * w.Hkv * w.D)
-                + 2 * w.B * w.S * w.Hq * w.D + 4 * w.B * w.Hq * w.S)
+    # bytes per Q/K/V element (fp4: half a byte of code plus the block
+    # scales, 1/16 byte for NVFP4 Q/K and 1/32 for MXFP4 V); O is bf16
+    nq, nkv = w.B * w.S * w.Hq * w.D, w.B * w.S * w.Hkv * w.D
+    if w.dtype == "fp4":
+        in_bytes = nq * (0.5 + 1 / 16) + nkv * (0.5 + 1 / 16) + nkv * (0.5 + 1 / 32)
+    else:
+        in_bytes = (1 if w.dtype == "fp8" else 2) * (nq + 2 * nkv)
+    io_bytes = int(in_bytes + 2 * nq + 4 * w.B * w.Hq * w.S)
     cfg["io_bytes"] = io_bytes
     cfg["l2"] = (f"inputs+outputs {io_bytes / 2**20:.0f} MiB > L2 126 MiB; no flush"
                  if io_bytes > L2_BYTES else "L2 flushed between steps")
@@ -351,11 +371,17 @@ def run_ours(args):
     cfg = workload_config(w, docs_np)
     cfg["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
 
-    host = {n: inp[n].pin_memory() for n in ("q", "k", "v")}
+    fp8, fp4 = w.dtype == "fp8", w.dtype == "fp4"
+    host = {n: inp[n].pin_memory() for n in (FP4_INPUTS if fp4 else ("q", "k", "v"))}
     dev = {n: host[n].to(device) for n in host}
     docs = None if docs_np is None else torch.as_tensor(docs_np, dtype=torch.int32, device=device)
-    fp8 = w.dtype == "fp8"
-    o = torch.empty(dev["q"].shape, dtype=torch.bfloat16, device=device)
+    o = torch.empty((w.B, w.S, w.Hq, w.D), dtype=torch.bfloat16, device=device)
+    ws4 = None
+    if fp4:
+        ws4 = torch.empty(attn.fp4_workspace_size(w.B, w.Hq, w.Hkv, w.S, w.S, w.D),
+                          dtype=torch.uint8, device=device)
+        cfg["classifier"] = args.classifier
+        cfg["formats"] = "NVFP4 Q/K (power-of-two e4m3 block scales), MXFP4 V and P"
     lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=device)
     window = None if w.window == (-1, -1) else w.window
     slopes = None
@@ -374,7 +400,7 @@ def run_ours(args):
         host.update(o=o.cpu().pin_memory(), lse=lse.cpu().pin_memory(),
                     dout=inp["dout"].pin_memory())
         dev.update(o=o, lse=lse, dout=host["dout"].to(device))
-        g_dq = torch.empty(dev["q"].shape, dtype=torch.float32, device=device)
+        g_dq = torch.empty(o.shape, dtype=torch.float32, device=device)
         g_dk = torch.empty_like(dev["k"])
         g_dv = torch.empty_like(dev["v"])
         ws = torch.empty(attn.bwd_workspace_size(w.B, w.Hq, w.Hkv, w.S, w.S, w.D),
@@ -407,6 +433,12 @@ def run_ours(args):
             attn.attn_bwd(d["q"], d["k"], d["v"], d["o"], d["lse"], d["dout"], outs[0], outs[1],
                           outs[2], ws, scale=w.scale, causal=w.causal, window=window,
                           doc_offsets=docs, stream=s, softcap=args.softcap, alibi_slopes=slopes)
+        elif fp4:
+            attn.attn_fwd_fp4(d["q_codes"], d["q_scales"], inp["q_global"], d["k_codes"],
+                              d["k_scales"], inp["k_global"], d["v_codes"], d["v_scales"],
+                              inp["v_global"], outs[0], outs[1], ws4, scale=w.scale,
+                              causal=w.causal, window=window, doc_offsets=docs,
+                              classifier=args.classifier, stream=s)
         elif fp8:
             attn.attn_fwd_fp8(d["q"], d["k"], d["v"], outs[0], outs[1],
                               q_descale=inp["q_descale"], k_descale=inp["k_descale"],
@@ -446,6 +478,11 @@ def run_ours(args):
     attn.check_device_status(stream)
     total_ms = t_begin.elapsed_time(t_end)
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    if flush is not None:
+        # The L2 flush between steps is not part of the work: time the K
+        # steps as the sum of their own event intervals.
+        total_ms = float(sum(launch_ms))
+        cfg["timed"] = "sum of the per-step event intervals (L2 flush excluded)"
     total_ms_max = max_over_ranks(total_ms, world, device)
     ms_per_step = total_ms_max / args.steps
     value = flops * args.steps * world / (total_ms_max / 1e3) / 1e12
@@ -508,12 +545,13 @@ def run_ours(args):
     # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s).
     peak_mult = 2.0 if fp8 else 1.0
     peak = float(peaks["bf16_tflops"]) * peak_mult
-    metric = metric_for(w, args.softcap, slopes is not None)
+    metric = metric_for(w, args.softcap, slopes is not None, args.classifier)
     result = {
         "metric": metric, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8e4m3" if fp8 else "bf16",
+        "dtype": ("fp8e4m3" if fp8 else "fp4e2m1 (NVFP4/MXFP4) on f16 tensor operands"
+                  if fp4 else "bf16"),
         "data": "synthetic", "config": cfg,
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
@@ -526,13 +564,16 @@ def run_ours(args):
                          peaks.get("bf16_tflops_sustained", peak))), 4),
                      "flops_per_launch": flops, "launch_ms": round(launch_avg_ms, 4),
                      "kernel": "attn_bwd (preprocess, dK/dV, dQ kernels per step)"
-                     if w.backward else "attn_fwd_kernel"},
+                     if w.backward else
+                     ("attn_fwd_fp4 (fp4_dequant_kernel + attn_fwd_kernel, timed together)"
+                      if fp4 else "attn_fwd_kernel")},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "pipelining": "two buffer sets, copy-in / compute / copy-out streams"},
-        "gpu_launches": args.steps * (3 if w.backward else 1),
+        "gpu_launches": args.steps * (3 if w.backward else 2 if fp4 else 1),
         "clocks": sampler.summary(),
     }
+    inp["classifier"] = args.classifier
     if (rank == 0 and world == 1 and not args.no_cpu_baseline
             and slopes is None and args.softcap is None):
         if w.backward:
@@ -561,8 +602,11 @@ def run_reference(args):
         return
     w = WORKLOADS[args.config]
     inp = make_inputs(w)
+    inp["classifier"] = args.classifier
     cfg = workload_config(w, inp["doc_offsets"])
     cfg["parallelism"] = "CPU oracle, rank 0 only"
+    if w.dtype == "fp4":
+        cfg["classifier"] = args.classifier
     # each step: ~2 s of oracle work, so steps + warmup end within minutes
     if w.backward:
         n_kv = kv_heads_for_seconds(w, inp, 2.0)
@@ -582,7 +626,8 @@ def run_reference(args):
     total = sum(times)
     value = fl_total / total / 1e12
     result = {
-        "impl": "reference", "metric": metric_for(w), "value": round(value, 6), "unit": UNIT,
+        "impl": "reference", "metric": metric_for(w, classifier=args.classifier),
+        "value": round(value, 6), "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define ATTN_ABI_VERSION 1
+#define ATTN_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define ATTN_API __attribute__((visibility("default")))
@@ -67,7 +67,9 @@ typedef enum {
     ATTN_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned */
     ATTN_ERR_LAUNCH = 4,         /* the CUDA launch itself failed */
     ATTN_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait expired */
-    ATTN_ERR_CUDA = 6            /* another CUDA runtime error (see detail) */
+    ATTN_ERR_CUDA = 6,           /* another CUDA runtime error (see detail) */
+    ATTN_ERR_RANGE = 7           /* an input value outside the range the path
+                                    represents (FP4 scales; see attn_fwd_fp4) */
 } attn_status_t;
 
 /* Tuning knobs of the forward.  Pass NULL for the defaults.  None of them
@@ -163,6 +165,82 @@ ATTN_API attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v,
                                     const attn_fwd_options_t *opts, void *stream);
 
 /*
+ * FP4 Direct-P forward ("Hardware-Aware FP4 FlashAttention-4",
+ * "Metodología", item 1).  Q and K arrive in NVFP4, V in MXFP4; the
+ * probabilities are built directly as MXFP4 values and the softmax
+ * normaliser is the sum of exactly those values, so the output is the
+ * weighted mean of V under the quantised weights:
+ *
+ *   per row i and 32-key block g (keys [32g, 32g+32), allowed keys only):
+ *     y_j   = log2-unit score  scale * q_global * k_global * <q'_i, k'_j> / ln 2
+ *             (q', k': the NVFP4 values without their per-tensor factors)
+ *     E_g   = floor(max_j y_j) - 2                 (the OCP MX exponent rule)
+ *     r_j   = y_j - E_g                            (< 3)
+ *     c_j   = E2M1 magnitude (0, 0.5, 1, 1.5, 2, 3, 4, 6) chosen by
+ *             ATTN_DIRECT_P_AFFINE: index clamp(rint(2 r_j + 2), 0, 7)
+ *             ATTN_DIRECT_P_EXP2:   2^r_j rounded to nearest (ties even), max 6
+ *     w_j   = c_j * 2^E_g
+ *   O_i   = v_global * sum_j w_j v'_j / sum_j w_j       (bf16)
+ *   LSE_i = ln(sum_j w_j)                              (fp32, natural log)
+ *
+ * The scores are measured from an integer anchor that follows the running
+ * row maximum (rescaled only when the maximum rises by more than
+ * rescale_threshold, always by an exact power of two); shifting a row's
+ * log2 scores by an integer changes no code, so the result does not depend
+ * on the anchor.  A block whose maximum lies more than
+ * 26 - ceil(rescale_threshold) octaves below the anchor contributes nothing
+ * (its values would leave the normal range of the f16 container).
+ *
+ * Inputs (device memory, 16-byte aligned, caller-owned):
+ *   q_codes  uint8 [B, Sq, Hq,  D/2]  two E2M1 codes per byte, element 2j
+ *   k_codes  uint8 [B, Sk, Hkv, D/2]  in the low nibble (bit 3 = sign)
+ *   q_scales uint8 [B, Sq, Hq,  D/16] e4m3 scale per 16 elements of a row
+ *   k_scales uint8 [B, Sk, Hkv, D/16]
+ *   v_codes  uint8 [B, Sk, Hkv, D/2]
+ *   v_scales uint8 [B, ceil(Sk/32), Hkv, D]  UE8M0 scale (2^(u - 127)) per
+ *            32 keys of each (batch, head, d) column of V
+ *   q_global, k_global, v_global: per-tensor fp32 factors, > 0 and finite.
+ * A nonzero code whose scale is NaN, or (V) whose u - 127 lies outside
+ * [-13, 13], reads as 0 and makes attn_get_device_status() report
+ * ATTN_ERR_RANGE.
+ * Outputs: o bf16 [B, Sq, Hq, D], lse fp32 [B, Hq, Sq].
+ * workspace: at least attn_fwd_fp4_workspace_size() bytes, 16-byte aligned
+ * (Q, K, V widened to f16, exactly; contents on entry ignored).
+ * D must be 64 or 128; masks, GQA and shape rules as attn_fwd; no score
+ * modifiers.  Both products run on the tensor cores with f16 operands that
+ * hold the FP4 values exactly and fp32 accumulation.  opts may be NULL.
+ */
+#define ATTN_DIRECT_P_AFFINE 0
+#define ATTN_DIRECT_P_EXP2 1
+
+typedef struct {
+    /* Online rescale threshold of the integer anchor, in log2 units,
+     * [0, 8].  Default 8. */
+    float rescale_threshold;
+    /* ATTN_DIRECT_P_AFFINE (default) or ATTN_DIRECT_P_EXP2. */
+    int classifier;
+    /* Bound of every device-side wait, microseconds (0 = 1 s); as in
+     * attn_fwd_options_t.  Valid range [0, 60000000]. */
+    int wait_timeout_us;
+    int reserved[5]; /* must be zero */
+} attn_fp4_options_t;
+
+/* Fills *opts with the defaults. */
+ATTN_API void attn_fp4_default_options(attn_fp4_options_t *opts);
+
+/* Workspace bytes attn_fwd_fp4 needs for these sizes (0 for invalid ones). */
+ATTN_API size_t attn_fwd_fp4_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D);
+
+ATTN_API attn_status_t attn_fwd_fp4(const void *q_codes, const void *q_scales, float q_global,
+                                    const void *k_codes, const void *k_scales, float k_global,
+                                    const void *v_codes, const void *v_scales, float v_global,
+                                    void *o, float *lse, int B, int Hq, int Hkv, int Sq, int Sk,
+                                    int D, float scale, int causal, int window_left,
+                                    int window_right, const int *doc_offsets, int num_docs,
+                                    void *workspace, size_t workspace_bytes,
+                                    const attn_fp4_options_t *opts, void *stream);
+
+/*
  * Backward ("Hardware-Aware FP4 FlashAttention-4", "Causal Backward
  * Cuantizado": gradients from the saved LSE, probabilities rebuilt rather
  * than stored).  For L with dO = dL/dO:
@@ -234,8 +312,8 @@ ATTN_API attn_status_t attn_bwd_noalloc(const void *q, const void *k, const void
                                         const int *doc_offsets, int num_docs, void *stream);
 
 /* Synchronises `stream`, then reads and clears the device status word of
- * the current device.  Returns ATTN_OK or ATTN_ERR_DEVICE_TIMEOUT (or
- * ATTN_ERR_CUDA if the synchronisation itself failed). */
+ * the current device.  Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT or
+ * ATTN_ERR_RANGE (or ATTN_ERR_CUDA if the synchronisation itself failed). */
 ATTN_API attn_status_t attn_get_device_status(void *stream);
 
 /* Static description of a status code. */

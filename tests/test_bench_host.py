@@ -127,6 +127,28 @@ def test_metric_names_per_workload():
     assert "FP8" in bench.metric_for(WORKLOADS["causal_s8192_fp8"])
     assert "softcap 30" in bench.metric_for(WORKLOADS["causal_s8192"], softcap=30.0)
     assert "ALiBi" in bench.metric_for(WORKLOADS["causal_s8192"], alibi=True)
+    m = bench.metric_for(WORKLOADS["causal_s8192_fp4"], classifier="exp2")
+    assert "Direct-P exp2" in m and "fp4" in m
+
+
+def test_fp4_io_bytes_count_codes_and_scales():
+    w = WORKLOADS["causal_s8192_fp4"]
+    cfg = bench.workload_config(w, None)
+    n = w.B * w.S * w.Hq * w.D
+    # Q, K: half a byte of code + one e4m3 byte per 16; V: + one UE8M0 byte
+    # per 32; O bf16; LSE fp32
+    assert cfg["io_bytes"] == int(2 * n * (0.5 + 1 / 16) + n * (0.5 + 1 / 32) + 2 * n
+                                  + 4 * w.B * w.Hq * w.S)
+
+
+def test_fp4_oracle_sample_runs():
+    from tiled_attention_blackwell_b200.workloads import make_inputs
+    w = Workload("fp4_small", 1, 2, 2, 96, 64, True, seed=9, dtype="fp4")
+    inp = make_inputs(w)
+    for classifier in ("affine", "exp2"):
+        inp["classifier"] = classifier
+        dt, fl, cores = bench.oracle_sample(w, inp, 20)
+        assert dt > 0 and fl > 0 and cores >= 1
 
 
 def test_oracle_backward_sample_counts_the_sliced_problem():

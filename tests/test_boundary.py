@@ -42,8 +42,8 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.attn_abi_version() == 1
-    for code in range(7):
+    assert L.attn_abi_version() == 2
+    for code in range(8):
         s = L.attn_status_string(code).decode()
         assert s and s != "unknown status"
     assert L.attn_status_string(99).decode() == "unknown status"
@@ -243,12 +243,15 @@ def test_option_structs_match_the_c_layout(tmp_path):
         "int main(void) {\n"
         '  printf("attn_fwd_options_t size %zu\\n", sizeof(attn_fwd_options_t));\n'
         '  printf("attn_bwd_options_t size %zu\\n", sizeof(attn_bwd_options_t));\n'
+        '  printf("attn_fp4_options_t size %zu\\n", sizeof(attn_fp4_options_t));\n'
         "  F(attn_fwd_options_t, rescale_threshold); F(attn_fwd_options_t, exp2_mode);\n"
         "  F(attn_fwd_options_t, wait_timeout_us); F(attn_fwd_options_t, debug_withhold_kv);\n"
         "  F(attn_fwd_options_t, softcap); F(attn_fwd_options_t, reserved0);\n"
         "  F(attn_fwd_options_t, alibi_slopes); F(attn_fwd_options_t, reserved);\n"
         "  F(attn_bwd_options_t, softcap); F(attn_bwd_options_t, reserved0);\n"
         "  F(attn_bwd_options_t, alibi_slopes); F(attn_bwd_options_t, reserved);\n"
+        "  F(attn_fp4_options_t, rescale_threshold); F(attn_fp4_options_t, classifier);\n"
+        "  F(attn_fp4_options_t, wait_timeout_us); F(attn_fp4_options_t, reserved);\n"
         "  return 0;\n}\n")
     exe = tmp_path / "layout"
     import subprocess
@@ -259,7 +262,74 @@ def test_option_structs_match_the_c_layout(tmp_path):
     for line in out.splitlines():
         t, m, v = line.split()
         c[(t, m)] = int(v)
-    for name, cls in (("attn_fwd_options_t", attn.FwdOptions), ("attn_bwd_options_t", attn.BwdOptions)):
+    for name, cls in (("attn_fwd_options_t", attn.FwdOptions), ("attn_bwd_options_t", attn.BwdOptions),
+                      ("attn_fp4_options_t", attn.Fp4Options)):
         assert c[(name, "size")] == ctypes.sizeof(cls), name
         for field, _ in cls._fields_:
             assert c[(name, field)] == getattr(cls, field).offset, (name, field)
+
+
+# ------------------------------------------------------------ FP4 Direct-P
+
+def test_fp4_defaults_and_workspace(L):
+    o = attn.fp4_options()
+    assert o.rescale_threshold == 8.0 and o.classifier == attn.ATTN_DIRECT_P_AFFINE
+    assert o.wait_timeout_us == 0 and list(o.reserved) == [0] * 5
+    # Q, K, V widened to f16, each rounded up to 256 bytes
+    assert attn.fp4_workspace_size(2, 16, 16, 8192, 8192, 128) == 3 * 2 * 2 * 8192 * 16 * 128
+    assert attn.fp4_workspace_size(1, 2, 1, 3, 5, 64) == 768 + 2 * 768  # 768 B, 640 B -> 768
+    assert attn.fp4_workspace_size(0, 2, 1, 3, 5, 64) == 0
+
+
+def call_fp4(L, **kw):
+    a = dict(qc=P, qs=P, qg=1.0, kc=P, ks=P, kg=0.5, vc=P, vs=P, vg=1.0, o=P, lse=P, B=1, Hq=2,
+             Hkv=2, Sq=16, Sk=16, D=128, scale=0.1, causal=0, wl=-1, wr=-1, docs=None, nd=0,
+             ws=P, wsb=1 << 20, opts=None)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    return L.attn_fwd_fp4(vp(a["qc"]), vp(a["qs"]), a["qg"], vp(a["kc"]), vp(a["ks"]), a["kg"],
+                          vp(a["vc"]), vp(a["vs"]), a["vg"], vp(a["o"]), vp(a["lse"]), a["B"],
+                          a["Hq"], a["Hkv"], a["Sq"], a["Sk"], a["D"], a["scale"], a["causal"],
+                          a["wl"], a["wr"], vp(a["docs"]) if a["docs"] else None, a["nd"],
+                          vp(a["ws"]), a["wsb"],
+                          None if a["opts"] is None else ctypes.byref(a["opts"]), None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(qg=0.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(kg=float("nan")), attn.ATTN_ERR_INVALID_ARG),
+    (dict(vg=-1.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(vs=P + 8), attn.ATTN_ERR_MISALIGNED),
+    (dict(ws=P + 4), attn.ATTN_ERR_MISALIGNED),
+    (dict(lse=P + 2), attn.ATTN_ERR_MISALIGNED),
+    (dict(kc=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(ws=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(wsb=1000), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Sq=8, docs=P, nd=1), attn.ATTN_ERR_INVALID_ARG),
+    (dict(opts=attn.fp4_options(classifier=2)), attn.ATTN_ERR_INVALID_ARG),
+    (dict(opts=attn.fp4_options(rescale_threshold=8.5)), attn.ATTN_ERR_INVALID_ARG),
+    (dict(opts=attn.fp4_options(rescale_threshold=-1.0)), attn.ATTN_ERR_INVALID_ARG),
+    (dict(opts=attn.fp4_options(wait_timeout_us=-5)), attn.ATTN_ERR_INVALID_ARG),
+])
+def test_fp4_invalid_arguments_rejected_before_launch(L, kw, status):
+    assert call_fp4(L, **kw) == status
+
+
+def test_fp4_reserved_options_must_be_zero(L):
+    o = attn.fp4_options()
+    o.reserved[4] = 1
+    assert call_fp4(L, opts=o) == attn.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
+def test_valid_fp4_call_without_gpu_reports_cuda_error(L):
+    for classifier in (0, 1):
+        assert call_fp4(L, opts=attn.fp4_options(classifier=classifier)) == attn.ATTN_ERR_CUDA
+
+
+def test_fp4_binding_checks_shapes(L):
+    q = torch.zeros(1, 4, 1, 32, dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        attn.attn_fwd_fp4(q, q, 1.0, q, q, 1.0, q, q, 1.0, None, None, None, scale=0.1)

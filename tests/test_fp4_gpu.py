@@ -1,0 +1,228 @@
+"""GPU parity of the FP4 Direct-P forward against the oracle (B200).
+
+Inputs with power-of-two NVFP4 block scales and a power-of-two score factor
+make every log2 score an exact dyadic number in both fp32 (kernel) and fp64
+(oracle), so the quantised decisions -- block exponents and E2M1 codes --
+are the same on both sides and the comparison is element by element at the
+output's own rounding: |O - O_ref| <= 2^-8 |O_ref| + 2^-20 max|V| (bf16
+output, fp32 accumulation of exact products), |LSE - LSE_ref| <= 2e-5 +
+1e-6 |LSE_ref|.  General NVFP4 inputs (e4m3 block scales) round the scores
+in fp32 first, so a code may differ from the oracle's where a score sits
+within rounding of a decision boundary; those cases are held to the
+attention tolerance (O max-abs 2e-2, mean-abs 2e-3; LSE 1e-3).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tiled_attention_blackwell_b200 import attn
+from tiled_attention_blackwell_b200.workloads import (WORKLOADS, draw_doc_offsets,
+                                                      make_inputs, make_tensors_fp4)
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("q_codes", "q_scales", "q_global", "k_codes", "k_scales", "k_global", "v_codes",
+         "v_scales", "v_global")
+
+
+def _dev(t):
+    return [t[n].cuda() if torch.is_tensor(t[n]) else t[n] for n in NAMES]
+
+
+def _vmax(t):
+    c = t["v_codes"].numpy()
+    mag = np.maximum(np.abs(c & 7), np.abs((c >> 4) & 7)).max()
+    return [0, 0.5, 1, 1.5, 2, 3, 4, 6][mag] * 2.0 ** (int(t["v_scales"].numpy().max()) - 127)
+
+
+def _run(t, classifier, **kw):
+    o, lse = attn.attention_fp4(*_dev(t), classifier=classifier, **kw)
+    attn.check_device_status()
+    return o.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _ref(t, classifier, **kw):
+    return oracle.attn_fwd_fp4(*[t[n] for n in NAMES], classifier=classifier, **kw)
+
+
+def _tight(o, lse, o_ref, lse_ref, vmax):
+    err = np.abs(o - o_ref)
+    bound = 2.0 ** -8 * np.abs(o_ref) + 2.0 ** -20 * vmax
+    bad = err > bound
+    assert not bad.any(), (int(bad.sum()), float(err.max()), np.argwhere(bad)[:5])
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse), fin)
+    lerr = np.abs(lse[fin] - lse_ref[fin])
+    assert (lerr <= 2e-5 + 1e-6 * np.abs(lse_ref[fin])).all(), float(lerr.max())
+
+
+CASES = [
+    # B, Hq, Hkv, Sq, Sk, D, mask kwargs
+    (1, 2, 2, 300, 300, 128, dict(causal=True)),
+    (1, 2, 2, 300, 300, 64, dict(causal=False)),
+    (2, 4, 2, 257, 383, 128, dict(causal=True)),
+    (1, 2, 1, 600, 600, 128, dict(causal=True, window=(64, 0))),
+    (1, 2, 2, 333, 333, 64, dict(causal=False, window=(40, 17))),
+    (1, 2, 2, 1, 1000, 128, dict(causal=True)),
+    (1, 1, 1, 1, 1, 64, dict(causal=False)),
+    (1, 3, 3, 129, 129, 128, dict(causal=False)),
+]
+
+
+@pytest.mark.parametrize("classifier", ["affine", "exp2"])
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[:6]}-{sorted(c[6].items())}")
+def test_fp4_parity_exact_decisions(case, classifier):
+    B, Hq, Hkv, Sq, Sk, D, mask = case
+    scale = 1.0 / math.sqrt(D)
+    t = make_tensors_fp4(B, Hq, Hkv, Sq, Sk, D, seed=11 + Sq + D, scale=scale)
+    o, lse = _run(t, classifier, scale=scale, **mask)
+    o_ref, lse_ref = _ref(t, classifier, scale=scale, **mask)
+    _tight(o, lse, o_ref, lse_ref, _vmax(t))
+
+
+@pytest.mark.parametrize("classifier", ["affine", "exp2"])
+def test_fp4_parity_document_mask(classifier):
+    S, D = 700, 64
+    scale = 1.0 / math.sqrt(D)
+    t = make_tensors_fp4(1, 4, 2, S, S, D, seed=21, scale=scale)
+    docs = np.array([0, 100, 450, 451, 700], dtype=np.int32)
+    o, lse = _run(t, classifier, scale=scale, causal=True,
+                  doc_offsets=torch.from_numpy(docs).cuda())
+    o_ref, lse_ref = _ref(t, classifier, scale=scale, causal=True, doc_offsets=docs)
+    _tight(o, lse, o_ref, lse_ref, _vmax(t))
+
+
+@pytest.mark.parametrize("tau", [0.0, 3.0, 8.0])
+def test_fp4_rescale_threshold_does_not_change_the_result(tau):
+    # The anchor is an integer and every rescale an exact power of two: the
+    # result for any threshold matches the oracle, which has no anchor.
+    S, D = 520, 128
+    scale = 1.0 / math.sqrt(D)
+    t = make_tensors_fp4(1, 2, 2, S, S, D, seed=31, scale=scale)
+    o, lse = _run(t, "affine", scale=scale, causal=True,
+                  options=attn.fp4_options(rescale_threshold=tau))
+    o_ref, lse_ref = _ref(t, "affine", scale=scale, causal=True)
+    _tight(o, lse, o_ref, lse_ref, _vmax(t))
+
+
+@pytest.mark.parametrize("classifier", ["affine", "exp2"])
+def test_fp4_wide_logits(classifier):
+    # Score factor 2^3 instead of ~2^-3: log2 scores spread over hundreds of
+    # units, so the anchor moves by large steps and most blocks sit far below
+    # it (the range guard).  The kernel drops a block whose maximum lies more
+    # than 26 - ceil(threshold) octaves below the anchor; with threshold 0
+    # each dropped key weighs under 2^-24 of the row maximum's weight (the
+    # anchor is at most one octave above the maximum), so the output may
+    # differ from the oracle's by at most Sk * 2^-24 * 2 max|V| beyond the
+    # rounding bound.
+    S, D = 400, 128
+    t = make_tensors_fp4(1, 2, 2, S, S, D, seed=41, scale=8.0)
+    o, lse = _run(t, classifier, scale=8.0, causal=True,
+                  options=attn.fp4_options(rescale_threshold=0.0))
+    o_ref, lse_ref = _ref(t, classifier, scale=8.0, causal=True)
+    assert np.abs(lse_ref).max() > 100
+    vmax = _vmax(t)
+    err = np.abs(o - o_ref)
+    assert (err <= 2.0 ** -8 * np.abs(o_ref) + S * 2.0 ** -23 * vmax).all(), float(err.max())
+    assert np.abs(lse - lse_ref).max() <= 1e-4 * np.abs(lse_ref).max()
+
+
+@pytest.mark.parametrize("classifier", ["affine", "exp2"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp4_general_nvfp4_scales(classifier, D):
+    S = 300
+    scale = 1.0 / math.sqrt(D)
+    t = make_tensors_fp4(1, 2, 2, S, S, D, seed=51, scale=scale, pow2_scales=False)
+    o, lse = _run(t, classifier, scale=scale, causal=True)
+    o_ref, lse_ref = _ref(t, classifier, scale=scale, causal=True)
+    err = np.abs(o - o_ref)
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
+    assert np.abs(lse - lse_ref).max() <= 1e-3
+
+
+def test_fp4_full_size_sampled_rows():
+    # The benchmark's workload and launch (B2 H16 S8192 D128 causal), checked
+    # on sampled rows the oracle computes one by one.
+    w = WORKLOADS["causal_s8192_fp4"]
+    t = make_inputs(w)
+    o, lse = _run(t, "affine", scale=w.scale, causal=True)
+    rng = np.random.default_rng(5)
+    rows = np.stack([rng.integers(0, w.B, 48), rng.integers(0, w.Hq, 48),
+                     rng.integers(0, w.S, 48)], 1)
+    rows = np.concatenate([rows, [[0, 0, 0], [1, 15, w.S - 1], [0, 3, 127], [1, 8, 128]]])
+    for classifier in ("affine", "exp2"):
+        if classifier == "exp2":
+            o, lse = _run(t, classifier, scale=w.scale, causal=True)
+        o_ref, lse_ref = _ref(t, classifier, scale=w.scale, causal=True, rows=rows)
+        got = o[rows[:, 0], rows[:, 2], rows[:, 1]]
+        got_lse = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
+        _tight(got, got_lse, o_ref, lse_ref, _vmax(t))
+
+
+def test_fp4_range_error_reported():
+    S, D = 64, 64
+    t = make_tensors_fp4(1, 1, 1, S, S, D, seed=61)
+    # an out-of-range V scale under nonzero codes: reported, read as zero
+    t["v_scales"] = t["v_scales"].clone()
+    t["v_scales"][0, 0, 0, 0] = 200
+    t["v_codes"] = t["v_codes"].clone()
+    t["v_codes"][0, 0, 0, 0] = 0x11
+    attn.attention_fp4(*_dev(t), causal=True)
+    assert attn.device_status() == attn.ATTN_ERR_RANGE
+    assert attn.device_status() == attn.ATTN_OK  # reading clears it
+    # the same scale under zero codes is harmless
+    t["v_codes"][:, :32, 0, 0] = 0
+    attn.attention_fp4(*_dev(t), causal=True)
+    assert attn.device_status() == attn.ATTN_OK
+    # a NaN NVFP4 scale under nonzero codes
+    t2 = make_tensors_fp4(1, 1, 1, S, S, D, seed=62)
+    t2["q_scales"] = t2["q_scales"].clone()
+    t2["q_scales"][0, 3, 0, 1] = 0x7F
+    t2["q_codes"] = t2["q_codes"].clone()
+    t2["q_codes"][0, 3, 0, 8] = 0x22
+    attn.attention_fp4(*_dev(t2), causal=True)
+    assert attn.device_status() == attn.ATTN_ERR_RANGE
+
+
+def test_fp4_cosine_against_bf16_exact():
+    # Accuracy record (not parity): mean cosine similarity of the Direct-P
+    # output against exact attention of the decoded inputs, on Gaussian
+    # inputs with general NVFP4 scales; the page reports about 0.944 for its
+    # fast path against BF16.
+    S, D = 1024, 128
+    scale = 1.0 / math.sqrt(D)
+    t = make_tensors_fp4(1, 4, 4, S, S, D, seed=71, scale=scale, pow2_scales=False)
+    q = torch.from_numpy(_decode(t, "q")).to(torch.float64)
+    k = torch.from_numpy(_decode(t, "k")).to(torch.float64)
+    v = torch.from_numpy(_decode_v(t)).to(torch.float64)
+    ref, _ = oracle.attn_fwd(q.numpy(), k.numpy(), v.numpy(), scale=scale)
+    for classifier, floor in (("affine", 0.9), ("exp2", 0.95)):
+        o, _ = _run(t, classifier, scale=scale)
+        a, b = o.reshape(-1, D), ref.reshape(-1, D)
+        cos = (a * b).sum(1) / np.linalg.norm(a, axis=1) / np.linalg.norm(b, axis=1)
+        print(f"{classifier}: mean cosine {cos.mean():.4f}")
+        assert cos.mean() >= floor
+
+
+def _nibbles(c):
+    c = c.numpy()
+    return np.stack([c & 15, c >> 4], -1).reshape(*c.shape[:-1], -1)
+
+
+_E2M1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6])
+
+
+def _decode(t, name):
+    mag = _E2M1[_nibbles(t[name + "_codes"])]
+    sc = t[name + "_scales"].view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    return t[name + "_global"] * mag * np.repeat(sc, 16, axis=-1)
+
+
+def _decode_v(t):
+    mag = _E2M1[_nibbles(t["v_codes"])]
+    S = mag.shape[1]
+    sc = np.exp2(t["v_scales"].numpy().astype(np.float64) - 127)
+    return t["v_global"] * mag * np.repeat(sc, 32, axis=1)[:, :S]

@@ -24,8 +24,14 @@ ATTN_ERR_MISALIGNED = 3
 ATTN_ERR_LAUNCH = 4
 ATTN_ERR_DEVICE_TIMEOUT = 5
 ATTN_ERR_CUDA = 6
+ATTN_ERR_RANGE = 7
 
-EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_fp8", "attn_fwd_default_options", "attn_bwd",
+ATTN_DIRECT_P_AFFINE = 0
+ATTN_DIRECT_P_EXP2 = 1
+CLASSIFIERS = {"affine": ATTN_DIRECT_P_AFFINE, "exp2": ATTN_DIRECT_P_EXP2}
+
+EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_fp8", "attn_fwd_default_options",
+            "attn_fp4_default_options", "attn_fwd_fp4_workspace_size", "attn_fwd_fp4", "attn_bwd",
             "attn_bwd_ex", "attn_bwd_workspace_size", "attn_bwd_noalloc", "attn_get_device_status",
             "attn_status_string", "attn_last_error_detail", "attn_abi_version")
 
@@ -48,6 +54,12 @@ class BwdOptions(ctypes.Structure):
     """Mirror of attn_bwd_options_t."""
     _fields_ = [("softcap", ctypes.c_float), ("reserved0", ctypes.c_int),
                 ("alibi_slopes", ctypes.c_void_p), ("reserved", ctypes.c_int * 4)]
+
+
+class Fp4Options(ctypes.Structure):
+    """Mirror of attn_fp4_options_t."""
+    _fields_ = [("rescale_threshold", ctypes.c_float), ("classifier", ctypes.c_int),
+                ("wait_timeout_us", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
 
 
 _FWD_ARGS = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [ctypes.c_float] + \
@@ -75,6 +87,16 @@ def lib():
             L.attn_fwd_fp8.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_float] * 3 + \
                 [ctypes.c_void_p] * 2 + [ctypes.c_int] * 6 + [ctypes.c_float] + \
                 [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(FwdOptions),
+                                      ctypes.c_void_p]
+            L.attn_fp4_default_options.restype = None
+            L.attn_fp4_default_options.argtypes = [ctypes.POINTER(Fp4Options)]
+            L.attn_fwd_fp4_workspace_size.restype = ctypes.c_size_t
+            L.attn_fwd_fp4_workspace_size.argtypes = [ctypes.c_int] * 6
+            L.attn_fwd_fp4.restype = ctypes.c_int
+            L.attn_fwd_fp4.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float] * 3 + \
+                [ctypes.c_void_p] * 2 + [ctypes.c_int] * 6 + [ctypes.c_float] + \
+                [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                      ctypes.c_size_t, ctypes.POINTER(Fp4Options),
                                       ctypes.c_void_p]
             L.attn_fwd_default_options.restype = None
             L.attn_fwd_default_options.argtypes = [ctypes.POINTER(FwdOptions)]
@@ -248,6 +270,89 @@ def attention_fp8(q, k, v, *, q_descale, k_descale, v_descale, scale=None, causa
     attn_fwd_fp8(q, k, v, o, lse, q_descale=q_descale, k_descale=k_descale,
                  v_descale=v_descale, scale=scale, causal=causal, window=window,
                  doc_offsets=doc_offsets, options=options, stream=stream)
+    return o, lse
+
+
+def fp4_options(**overrides) -> Fp4Options:
+    opts = Fp4Options()
+    lib().attn_fp4_default_options(ctypes.byref(opts))
+    for k, v in overrides.items():
+        setattr(opts, k, v)
+    return opts
+
+
+def fp4_workspace_size(B, Hq, Hkv, Sq, Sk, D) -> int:
+    """Bytes of device workspace attn_fwd_fp4 needs."""
+    return int(lib().attn_fwd_fp4_workspace_size(B, Hq, Hkv, Sq, Sk, D))
+
+
+def attn_fwd_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_codes, v_scales,
+                 v_global, o, lse, workspace, *, scale, causal=False, window=None,
+                 doc_offsets=None, classifier="affine", options=None, stream=None):
+    """Enqueue the FP4 Direct-P forward.
+
+    q_codes uint8 CUDA [B,Sq,Hq,D/2], q_scales uint8 [B,Sq,Hq,D/16] (e4m3
+    bytes), likewise k_*; v_codes [B,Sk,Hkv,D/2], v_scales uint8
+    [B,ceil(Sk/32),Hkv,D] (UE8M0 bytes); o bf16 [B,Sq,Hq,D]; lse fp32
+    [B,Hq,Sq]; workspace uint8 CUDA of fp4_workspace_size() bytes.  All
+    contiguous.  classifier: "affine" or "exp2" (overrides `options`).
+    """
+    B, Sq, Hq, Dh = q_codes.shape
+    _, Sk, Hkv, _ = k_codes.shape
+    D = 2 * Dh
+    shapes = (("q_codes", q_codes, (B, Sq, Hq, Dh)), ("q_scales", q_scales, (B, Sq, Hq, D // 16)),
+              ("k_codes", k_codes, (B, Sk, Hkv, Dh)), ("k_scales", k_scales, (B, Sk, Hkv, D // 16)),
+              ("v_codes", v_codes, (B, Sk, Hkv, Dh)),
+              ("v_scales", v_scales, (B, (Sk + 31) // 32, Hkv, D)))
+    for name, t, shape in shapes:
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or not t.is_cuda \
+                or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise TypeError(f"{name} must be a contiguous CUDA uint8 tensor of shape {shape}")
+    for name, t, dt in (("o", o, torch.bfloat16), ("lse", lse, torch.float32),
+                        ("workspace", workspace, torch.uint8)):
+        if t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA {dt} tensor")
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    if doc_offsets is not None:
+        if doc_offsets.dtype != torch.int32 or not doc_offsets.is_cuda:
+            raise TypeError("doc_offsets must be a CUDA int32 tensor")
+        docs_ptr, nd = _ptr(doc_offsets), doc_offsets.numel() - 1
+    else:
+        docs_ptr, nd = None, 0
+    options = fp4_options() if options is None else Fp4Options.from_buffer_copy(options)
+    options.classifier = CLASSIFIERS[classifier]
+    st = lib().attn_fwd_fp4(_ptr(q_codes), _ptr(q_scales), float(q_global), _ptr(k_codes),
+                            _ptr(k_scales), float(k_global), _ptr(v_codes), _ptr(v_scales),
+                            float(v_global), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
+                            float(scale), int(bool(causal)), wl, wr, docs_ptr, nd,
+                            _ptr(workspace), workspace.numel(), ctypes.byref(options),
+                            _stream_handle(stream))
+    _check(st, "attn_fwd_fp4")
+
+
+def attention_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_codes, v_scales,
+                  v_global, *, scale=None, causal=False, window=None, doc_offsets=None,
+                  classifier="affine", options=None, stream=None, workspace=None):
+    """Allocate O, LSE (and the workspace unless given) with torch and run the
+    FP4 Direct-P forward.  Returns (O, LSE)."""
+    B, Sq, Hq, Dh = q_codes.shape
+    _, Sk, Hkv, _ = k_codes.shape
+    D = 2 * Dh
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dev = q_codes.device
+    o = torch.empty((B, Sq, Hq, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(fp4_workspace_size(B, Hq, Hkv, Sq, Sk, D), dtype=torch.uint8,
+                                device=dev)
+    if doc_offsets is not None and not torch.is_tensor(doc_offsets):
+        doc_offsets = torch.as_tensor(doc_offsets, dtype=torch.int32)
+    if doc_offsets is not None and not doc_offsets.is_cuda:
+        doc_offsets = doc_offsets.to(dev)
+    attn_fwd_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_codes, v_scales,
+                 v_global, o, lse, workspace, scale=scale, causal=causal, window=window,
+                 doc_offsets=doc_offsets, classifier=classifier, options=options, stream=stream)
     return o, lse
 
 

@@ -13,6 +13,7 @@
 
 #include "../../include/attn.h"
 #include "bwd_kernel.cuh"
+#include "fp4_dequant.cuh"
 #include "fwd_kernel.cuh"
 
 namespace {
@@ -131,12 +132,12 @@ attn_status_t make_map_tile(CUtensorMap *map, const void *base, int B, int S, in
 
 // --------------------------------------------------------------- launching
 
-template <int D, int NS, int EXP, int MOD = 0, int FP8 = 0>
+template <int D, int NS, int EXP, int MOD = 0, int PREC = 0>
 attn_status_t launch_fwd(const tab::FwdParams &p, int grid, cudaStream_t stream) {
-    using Smem = tab::FwdSmem<D, NS, FP8 ? 1 : 2>;
+    using Smem = tab::FwdSmem<D, NS, PREC == 1 ? 1 : 2>;
     constexpr size_t smem = sizeof(Smem) + 1024;
     static_assert(smem <= 232448, "shared memory budget");
-    auto kernel = tab::attn_fwd_kernel<D, NS, EXP, MOD, FP8>;
+    auto kernel = tab::attn_fwd_kernel<D, NS, EXP, MOD, PREC>;
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     int dev = 0;
@@ -200,7 +201,19 @@ attn_status_t dispatch_fp8(const tab::FwdParams &p, int grid, int exp_mode, cuda
     }
 }
 
+// Direct-P kernels: PREC 2 (affine classifier) or 3 (exponential).
+attn_status_t dispatch_direct_p(const tab::FwdParams &p, int grid, int D, int classifier,
+                                cudaStream_t s) {
+    if (D == 128)
+        return classifier ? launch_fwd<128, kStagesD128, 0, 0, 3>(p, grid, s)
+                          : launch_fwd<128, kStagesD128, 0, 0, 2>(p, grid, s);
+    return classifier ? launch_fwd<64, kStagesD64, 0, 0, 3>(p, grid, s)
+                      : launch_fwd<64, kStagesD64, 0, 0, 2>(p, grid, s);
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 
 // Shape and mask checks shared by the forward and the backward.
 attn_status_t check_common(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
@@ -461,6 +474,123 @@ attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *o, flo
                        window_right, doc_offsets, num_docs, nullptr, stream);
 }
 
+void attn_fp4_default_options(attn_fp4_options_t *opts) {
+    if (!opts) return;
+    *opts = attn_fp4_options_t{};
+    opts->rescale_threshold = 8.0f;
+    opts->classifier = ATTN_DIRECT_P_AFFINE;
+}
+
+size_t attn_fwd_fp4_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1 || D < 1) return 0;
+    const size_t nq = (size_t)B * Sq * Hq * D, nkv = (size_t)B * Sk * Hkv * D;
+    return align256(nq * 2) + 2 * align256(nkv * 2);
+}
+
+attn_status_t attn_fwd_fp4(const void *q_codes, const void *q_scales, float q_global,
+                           const void *k_codes, const void *k_scales, float k_global,
+                           const void *v_codes, const void *v_scales, float v_global, void *o,
+                           float *lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                           float scale, int causal, int window_left, int window_right,
+                           const int *doc_offsets, int num_docs, void *workspace,
+                           size_t workspace_bytes, const attn_fp4_options_t *opts,
+                           void *stream) {
+    attn_fp4_options_t op;
+    attn_fp4_default_options(&op);
+    if (opts) op = *opts;
+
+    // ----- validation (no CUDA call before this block completes)
+    const void *ptrs[] = {q_codes, q_scales, k_codes, k_scales, v_codes, v_scales, o, workspace};
+    for (const void *ptr : ptrs)
+        if (!ptr) return fail(ATTN_ERR_INVALID_ARG, "null pointer");
+    if (!lse) return fail(ATTN_ERR_INVALID_ARG, "null pointer");
+    attn_status_t s = check_common(B, Hq, Hkv, Sq, Sk, D, scale, window_left, window_right,
+                                   doc_offsets, num_docs);
+    if (s != ATTN_OK) return s;
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr))
+            return fail(ATTN_ERR_MISALIGNED, "codes, scales, o and workspace must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+        return fail(ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
+    for (float g : {q_global, k_global, v_global})
+        if (!(g > 0.0f) || !std::isfinite(g))
+            return fail(ATTN_ERR_INVALID_ARG, "per-tensor factors must be > 0 and finite");
+    if (!(op.rescale_threshold >= 0.0f && op.rescale_threshold <= 8.0f))
+        return fail(ATTN_ERR_INVALID_ARG, "rescale_threshold must lie in [0, 8]");
+    if (op.classifier != ATTN_DIRECT_P_AFFINE && op.classifier != ATTN_DIRECT_P_EXP2)
+        return fail(ATTN_ERR_INVALID_ARG, "classifier must be ATTN_DIRECT_P_AFFINE or ATTN_DIRECT_P_EXP2");
+    if (op.wait_timeout_us < 0 || op.wait_timeout_us > 60000000)
+        return fail(ATTN_ERR_INVALID_ARG, "wait_timeout_us must lie in [0, 60000000]");
+    for (int r : op.reserved)
+        if (r != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved option fields must be zero");
+    const size_t need = attn_fwd_fp4_workspace_size(B, Hq, Hkv, Sq, Sk, D);
+    if (workspace_bytes < need)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+    const long long num_qblocks = (Sq + 2LL * tab::kBlockM - 1) / (2LL * tab::kBlockM);
+    const long long grid = num_qblocks * Hq * B;
+    if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+
+    // ----- set-up
+    DeviceState *st = nullptr;
+    if ((s = device_state(&st)) != ATTN_OK) return s;
+    const size_t nq = (size_t)B * Sq * Hq * D, nkv = (size_t)B * Sk * Hkv * D;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *q16 = ws, *k16 = ws + align256(nq * 2), *v16 = ws + align256(nq * 2) + align256(nkv * 2);
+
+    tab::FwdParams p;
+    memset(&p, 0, sizeof p);
+    if ((s = make_map(&p.tm_q, q16, B, Sq, Hq, D)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_k, k16, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    if ((s = make_map(&p.tm_v, v16, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.doc_offsets = doc_offsets;
+    p.num_docs = num_docs;
+    p.status = st->status;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.group = Hq / Hkv;
+    p.causal = causal ? 1 : 0;
+    p.window_left = window_left;
+    p.window_right = window_right;
+    p.num_qblocks = (int)num_qblocks;
+    p.head_group = std::min(B * Hq, kFwdHeadGroup * (Hq / Hkv));
+    p.scale_log2 = (float)((double)scale * q_global * k_global * 1.4426950408889634);
+    p.v_descale = v_global;
+    // P = code * 2^E with E <= 13 below the f16 maximum: with scores at most
+    // rescale_threshold above the anchor, an offset of 15 - ceil(threshold)
+    // keeps floor(max y) - 2 <= 13.
+    p.p_offset = 15.0f - std::ceil(op.rescale_threshold);
+    p.rescale_threshold = op.rescale_threshold;
+    p.timeout_ns = op.wait_timeout_us > 0 ? 1000ull * (unsigned long long)op.wait_timeout_us
+                                          : tab::kWaitTimeoutNs;
+#ifdef ATTN_TRACE
+    p.trace = g_trace;
+    p.trace_ctas = g_trace_ctas;
+#endif
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    tab::Fp4DequantParams dp;
+    memset(&dp, 0, sizeof dp);
+    dp.job[0] = {static_cast<const uint8_t *>(q_codes), static_cast<const uint8_t *>(q_scales),
+                 static_cast<uint32_t *>(q16), (long long)(nq / 32), Sq, Hq, 0};
+    dp.job[1] = {static_cast<const uint8_t *>(k_codes), static_cast<const uint8_t *>(k_scales),
+                 static_cast<uint32_t *>(k16), (long long)(nkv / 32), Sk, Hkv, 0};
+    dp.job[2] = {static_cast<const uint8_t *>(v_codes), static_cast<const uint8_t *>(v_scales),
+                 static_cast<uint32_t *>(v16), (long long)(nkv / 32), Sk, Hkv, 1};
+    dp.D = D;
+    dp.status = st->status;
+    const long long groups = dp.job[0].groups + dp.job[1].groups + dp.job[2].groups;
+    const long long blocks = std::min<long long>((groups + 255) / 256, (long long)st->num_sms * 16);
+    tab::fp4_dequant_kernel<<<(unsigned)std::max<long long>(blocks, 1), 256, 0, cs>>>(dp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ATTN_ERR_LAUNCH, "launch: %s", cudaGetErrorString(e));
+    return dispatch_direct_p(p, (int)grid, D, op.classifier, cs);
+}
+
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
     (void)Hkv;
     (void)Sk;
@@ -609,6 +739,7 @@ const char *attn_status_string(attn_status_t status) {
         case ATTN_ERR_LAUNCH: return "kernel launch failed";
         case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
         case ATTN_ERR_CUDA: return "CUDA runtime error";
+        case ATTN_ERR_RANGE: return "input value outside the representable range";
     }
     return "unknown status";
 }

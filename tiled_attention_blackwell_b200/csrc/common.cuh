@@ -9,6 +9,7 @@ namespace tab {
 
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int kStatusTimeout = 5;                   // ATTN_ERR_DEVICE_TIMEOUT
+constexpr int kStatusRange = 7;                     // ATTN_ERR_RANGE
 
 // Causal (bottom-right aligned), sliding-window and document masks each
 // allow a contiguous range of keys for a query row, so their intersection is

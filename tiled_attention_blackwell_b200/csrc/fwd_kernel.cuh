@@ -32,10 +32,15 @@
 // Template variants: EXP_MODE picks the MUFU / polynomial split of the
 // exponentials; MOD (bit 0 soft-cap, bit 1 ALiBi, "El FlexAttention de
 // PyTorch con FlashAttention-4", intro) transforms the scores into log2
-// units before the mask and the max; FP8 takes e4m3 Q, K, V (one 128-byte
-// chunk per row at D = 128, kind::f8f6f4 MMAs) and writes P as four e4m3
-// values per TMEM column ("Hardware-Aware FP4 FlashAttention-4",
-// "Precisión": the FP8 path).
+// units before the mask and the max; PREC picks the operand precision:
+// 0 bf16; 1 e4m3 Q, K, V (one 128-byte chunk per row at D = 128,
+// kind::f8f6f4 MMAs) with P as four e4m3 values per TMEM column
+// ("Hardware-Aware FP4 FlashAttention-4", "Precisión": the FP8 path);
+// 2 and 3 the Direct-P forward of the same page ("Metodología", item 1):
+// f16 operands holding NVFP4 / MXFP4 values exactly, and P built as MXFP4
+// values -- E2M1 codes times one power-of-two scale per 32 keys -- by the
+// affine classifier (2) or the rounded exponential (3), with the row sum
+// taken from exactly those values.
 //
 // Online softmax in log2 units: x = s * scale * log2(e).  Each row keeps a
 // running max m and sum l; a new block changes m (and rescales O and l) only
@@ -95,8 +100,9 @@ struct FwdParams {
     float softcap_in;   // scale / cap
     float softcap_out;  // cap * log2(e)
     const float *alibi_slopes;
-    // fp8 kernels: V's dequantisation factor (Q's and K's are folded into
-    // scale_log2) and the exponent offset that puts P into (0, 2^8].
+    // fp8 and Direct-P kernels: V's dequantisation factor (Q's and K's are
+    // folded into scale_log2) and the integer exponent offset that puts P
+    // into the range of its container (e4m3: (0, 2^8]; f16: below 2^16).
     float v_descale;
     float p_offset;
 };
@@ -207,6 +213,75 @@ __device__ __forceinline__ float exp_pack_half_fp8(const float *s, float c, floa
     return (sum0 + sum1) + (sum2 + sum3);
 }
 
+// Maximum of 32 consecutive scores.
+__device__ __forceinline__ float block_max32(const float *s) {
+    float a = fmax3(s[0], s[1], s[2]), b = fmax3(s[3], s[4], s[5]);
+#pragma unroll
+    for (int e = 6; e < 30; e += 4) {
+        a = fmax3(a, s[e], s[e + 1]);
+        b = fmax3(b, s[e + 2], s[e + 3]);
+    }
+    return fmax3(a, b, fmaxf(s[30], s[31]));
+}
+
+// Direct-P probabilities of 64 scores of a row (two 32-key blocks whose
+// maxima are bm[0], bm[1]): f16 pairs to pk, returns their fp32 sum.
+// base = p_offset - m (m: the row's integer anchor), so y = s*c + base is
+// the log2 score relative to the anchor, raised by the container offset.
+// Per block: E = floor(max y) - 2 (the OCP MX exponent rule), r = y - E;
+// code = E2M1 magnitude of r by the affine classifier (PREC 2: index
+// rint(2r + 2) clamped to [0, 7]) or of 2^r rounded to nearest (PREC 3);
+// P = code * 2^E.  Blocks with E < -13 (far below the anchor, where
+// 0.5 * 2^E would leave f16's normal range) are dropped; E is at most 13 by
+// the choice of p_offset.  The codes of a block are summed exactly in f16.
+constexpr float kRintMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+template <int PREC>
+__device__ __forceinline__ float direct_p_half(const float *s, const float *bm, float c,
+                                               float base, uint32_t *pk) {
+    float sum = 0.0f;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const float ymax = fmaf(bm[u], c, base);
+        const float ef = floorf(ymax) - 2.0f;
+        const bool keep = ef >= -13.0f;  // false for an all-masked block (-inf)
+        const int ei = keep ? (int)fminf(ef, 13.0f) : 0;
+        const float nb = keep ? base - (float)ei : -INFINITY;  // r = s*c + nb
+        const uint32_t h = keep ? (uint32_t)(ei + 15) << 10 : 0u;  // f16 2^E (or 0)
+        const uint32_t scale2 = h | (h << 16);
+        // affine: t = 2r + 2 + magic, rounded to an integer by the FMA itself
+        const float c2 = 2.0f * c, nb2 = 2.0f * nb + (2.0f + kRintMagic);
+        uint32_t cs0 = 0u, cs1 = 0u;
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const float s0 = s[32 * u + e], s1 = s[32 * u + e + 1];
+            uint32_t codes;
+            if constexpr (PREC == 2) {
+                float t0, t1;
+                fma2(t0, t1, s0, s1, c2, c2, nb2, nb2);
+                t0 = fminf(fmaxf(t0, kRintMagic), kRintMagic + 7.0f);
+                t1 = fminf(fmaxf(t1, kRintMagic), kRintMagic + 7.0f);
+                codes = e2m1x2_to_f16x2((__float_as_uint(t0) & 7u) |
+                                        ((__float_as_uint(t1) & 7u) << 4));
+            } else {
+                float r0, r1;
+                fma2(r0, r1, s0, s1, c, c, nb, nb);
+                codes = e2m1_round_f16x2(ex2_mufu(r0), ex2_mufu(r1));
+            }
+            pk[(32 * u + e) >> 1] = hmul2_u32(codes, scale2);
+            if ((e & 2) == 0) cs0 = hadd2_u32(cs0, codes);
+            else cs1 = hadd2_u32(cs1, codes);
+        }
+        if (keep) sum += f16x2_sum(hadd2_u32(cs0, cs1)) * __uint_as_float((uint32_t)(ei + 127) << 23);
+    }
+    return sum;
+}
+
+// 2^d for an integer-valued d <= 0 (exact; 0 below fp32's normal range and
+// for d = -inf).
+__device__ __forceinline__ float exp2_neg_int(float d) {
+    return d >= -126.0f ? __uint_as_float((uint32_t)((int)d + 127) << 23) : 0.0f;
+}
+
 // Score modifiers of n consecutive scores (n even), in log2 units, in place:
 // MOD bit 0 soft-cap, bit 1 ALiBi.  v holds <q_i, k_j>; dist0 is
 // i + (Sk - Sq) - j of the first as a float.
@@ -230,10 +305,12 @@ __device__ __forceinline__ void modify_scores(float *v, float c, float k1, float
     }
 }
 
-template <int D, int NS, int EXP_MODE, int MOD = 0, int FP8 = 0>
+template <int D, int NS, int EXP_MODE, int MOD = 0, int PREC = 0>
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ FwdParams p) {
-    static_assert(!(FP8 && MOD), "the fp8 path has no score modifiers");
+    static_assert(!(PREC && MOD), "the low-precision paths have no score modifiers");
+    constexpr bool FP8 = PREC == 1;
+    constexpr bool DP = PREC >= 2;  // Direct-P
     constexpr int EB = FP8 ? 1 : 2;
     using Smem = FwdSmem<D, NS, EB>;
     extern __shared__ uint8_t smem_raw[];
@@ -374,10 +451,12 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             // tcgen05 instructions (and the commits that track them).
             if (n_blocks > 0) {
                 const bool leader = elect_one();
-                constexpr uint32_t kIdescQK = FP8 ? idesc_e4m3_f32(kBlockM, kBlockN, 0, 0)
-                                                  : idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
-                constexpr uint32_t kIdescPV = FP8 ? idesc_e4m3_f32(kBlockM, D, 0, 1)
-                                                  : idesc_bf16_f32(kBlockM, D, 0, 1);
+                constexpr uint32_t kIdescQK = FP8  ? idesc_e4m3_f32(kBlockM, kBlockN, 0, 0)
+                                              : DP ? idesc_f16_f32(kBlockM, kBlockN, 0, 0)
+                                                   : idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+                constexpr uint32_t kIdescPV = FP8  ? idesc_e4m3_f32(kBlockM, D, 0, 1)
+                                              : DP ? idesc_f16_f32(kBlockM, D, 0, 1)
+                                                   : idesc_bf16_f32(kBlockM, D, 0, 1);
                 constexpr uint32_t kQTileBytes = Smem::kChunks * Smem::kChunkBytes;
                 constexpr uint32_t kChunkBytes = Smem::kChunkBytes;
                 // One MMA consumes 32 bytes of each operand row: 16 bf16 or
@@ -555,9 +634,34 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
 
             const int key0 = j * kBlockN;
             const float dist0 = diag_f - (float)key0;  // distance to key0 of this block
-            if (MOD) modify_scores<MOD, kBlockN / 2>(s, c, k1, p.softcap_out, slope2, dist0);
             const bool need_mask = key0 < kr.lo || key0 + kBlockN - 1 > kr.hi;
             const bool masked = __any_sync(0xffffffffu, need_mask);
+            float alpha = 1.0f;
+            float neg_m;
+            float bm[4];  // Direct-P: maxima of the four 32-key blocks
+            if constexpr (DP) {
+                // Direct-P: the anchor m is the running max rounded up to an
+                // integer, so every rescale is an exact power of two and the
+                // block exponents (and codes) do not depend on it.
+                if (masked) {
+#pragma unroll
+                    for (int e = 0; e < kBlockN; ++e) {
+                        const int key = key0 + e;
+                        if (key < kr.lo || key > kr.hi) s[e] = -INFINITY;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) bm[u] = block_max32(s + 32 * u);
+                const float m_cand = fmax3(fmaxf(bm[0], bm[1]), bm[2], bm[3]) * c;
+                if (m_cand > m_run + tau) {
+                    const float m_new = ceilf(m_cand);
+                    alpha = exp2_neg_int(m_run - m_new);
+                    m_run = m_new;
+                }
+                neg_m = m_run == -INFINITY ? 0.0f : p.p_offset - m_run;
+                if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 3);
+            } else {
+            if (MOD) modify_scores<MOD, kBlockN / 2>(s, c, k1, p.softcap_out, slope2, dist0);
             if (masked) {
 #pragma unroll
                 for (int e = 0; e < kBlockN / 2; ++e) {
@@ -591,7 +695,6 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 2);
             const float row_max = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
             const float m_cand = MOD ? row_max : row_max * c;
-            float alpha = 1.0f;
             if (m_cand > m_run + tau) {
                 alpha = ex2_mufu(m_run - m_cand);
                 m_run = m_cand;
@@ -599,8 +702,9 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             // fp8: P = 2^(x - m + p_offset) <= 2^8 keeps e4m3's range for the
             // small probabilities (the same factor scales l, so O and LSE are
             // unchanged).
-            const float neg_m = m_run == -INFINITY ? 0.0f : (FP8 ? p.p_offset - m_run : -m_run);
+            neg_m = m_run == -INFINITY ? 0.0f : (FP8 ? p.p_offset - m_run : -m_run);
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 3);
+            }
 
             l_run *= alpha;
 
@@ -633,7 +737,11 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             // use MUFU only: ex2(-inf) = 0 exactly.
             uint32_t pk[kBlockN / 2];
             if (MOD) __syncwarp();  // converged before the warp-collective TMEM store
-            if constexpr (FP8) {
+            if constexpr (DP) {
+                l_run += direct_p_half<PREC>(s, bm, c, neg_m, pk);
+                __syncwarp();  // converged before the warp-collective TMEM store
+                tmem_st32(s_tmem + 0, pk + 0);
+            } else if constexpr (FP8) {
                 // 64 e4m3 probabilities per 16 columns.
                 l_run += masked ? exp_pack_half_fp8<0>(s, c_exp, neg_m, pk)
                                 : exp_pack_half_fp8<EXP_MODE>(s, c_exp, neg_m, pk);
@@ -646,7 +754,12 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.p_half[i]);
-            if constexpr (FP8) {
+            if constexpr (DP) {
+                l_run += direct_p_half<PREC>(s + 64, bm + 2, c, neg_m, pk + 32);
+                if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
+                __syncwarp();
+                tmem_st32(s_tmem + 32, pk + 32);
+            } else if constexpr (FP8) {
                 l_run += masked ? exp_pack_half_fp8<0>(s + 64, c_exp, neg_m, pk + 16)
                                 : exp_pack_half_fp8<EXP_MODE>(s + 64, c_exp, neg_m, pk + 16);
                 if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
@@ -672,7 +785,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         }
         if (ok) {
             const bool row_ok = row < p.Sq;
-            const float inv_l = l_run > 0.0f ? (FP8 ? p.v_descale : 1.0f) / l_run : 0.0f;
+            const float inv_l = l_run > 0.0f ? (PREC ? p.v_descale : 1.0f) / l_run : 0.0f;
             __nv_bfloat16 *o_row =
                 p.o + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)D;
 #pragma unroll
@@ -699,7 +812,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 }
             }
             if (row_ok) {
-                const float m_lse = FP8 ? m_run - p.p_offset : m_run;
+                const float m_lse = PREC ? m_run - p.p_offset : m_run;
                 const float lse = l_run > 0.0f ? (m_lse + log2f(l_run)) * 0.69314718055994531f
                                                : -INFINITY;
                 p.lse[((size_t)b * p.Hq + hq) * p.Sq + row] = lse;

@@ -274,6 +274,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
            ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f16 with f16 inputs (format code 0 in bits
+// 7-9 and 10-12) and an fp32 accumulator; other fields as above.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn_major,
+                                                     int b_mn_major) {
+    return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Instruction descriptor, kind::f8f6f4: fp32 accumulate, A and B e4m3
 // (format code 0 in bits 7-9 and 10-12), majors, N/8, M/16.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn_major,
@@ -349,6 +357,54 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, fl
         : "=r"(r)
         : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
     return r;
+}
+
+// Two fp32 values rounded to E2M1 (nearest, ties to even, saturating at
+// +-6) and widened back to an f16 pair, x0 in the low half.
+__device__ __forceinline__ uint32_t e2m1_round_f16x2(float x0, float x1) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(x0), "f"(x1));
+    return r;
+}
+
+// The f16 pair of two E2M1 codes held in the low byte of `codes` (low
+// nibble -> low half).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t codes) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t.reg .b16 h;\n\t"
+        "cvt.u16.u32 h, %1;\n\t"
+        "cvt.u8.u16 t, h;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(r)
+        : "r"(codes));
+    return r;
+}
+
+// Packed f16 pair arithmetic.
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// Sum of the two halves of an f16 pair, as fp32.
+__device__ __forceinline__ float f16x2_sum(uint32_t a) {
+    float lo, hi;
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.f32.f16 %0, l;\n\t"
+        "cvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(a));
+    return lo + hi;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
