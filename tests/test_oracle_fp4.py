@@ -194,6 +194,30 @@ def test_direct_p_blocks_follow_key_index(classifier):
     assert np.abs(oc - oa).max() > 1e-3
 
 
+@pytest.mark.parametrize("classifier", CLASSIFIERS)
+def test_direct_p_block_size_is_32(classifier):
+    # One 32-key block: key 3 at y = 3.4, keys 16-31 at y = 0.6, keys 0-15
+    # other than 3 masked.  E = floor(3.4) - 2 = 1 for the whole block:
+    #   key 3:     r = 2.4 -> exp2 2^2.4 = 5.28 -> 6; affine rint(6.8) = 7 -> 6: w = 12
+    #   keys 16-31: r = -0.4 -> exp2 2^-0.4 = 0.758 -> 1 (w = 2);
+    #               affine rint(1.2) = 1 -> 0.5 (w = 1)
+    # (16-key blocks would give keys 16-31 their own E = -2 and w = 1.5.)
+    y = np.zeros(32)
+    y[3] = 3.4
+    y[16:] = 0.6
+    allow = np.zeros(32, dtype=bool)
+    allow[3] = True
+    allow[16:] = True
+    a, b = rng.standard_normal(4), rng.standard_normal(4)
+    v = np.zeros((32, 4))
+    v[3] = a
+    v[16:] = b
+    w = 2.0 if classifier == "exp2" else 1.0
+    o, lse = oracle.direct_p_row(y, v, allow=allow, classifier=classifier)
+    np.testing.assert_allclose(o, (12 * a + 16 * w * b) / (12 + 16 * w), rtol=0, atol=1e-13)
+    assert lse == pytest.approx(math.log(12 + 16 * w), abs=1e-13)
+
+
 # ------------------------------------------------------- full entry point
 
 def _decode_nvfp4(codes, scales, g):
@@ -255,6 +279,21 @@ def test_fp4_forward_is_direct_p_of_decoded_scores(classifier, pow2):
             oi, li = oracle.direct_p_row(y[i], v[0, :, hk], allow=allow, classifier=classifier)
             np.testing.assert_allclose(o[0, i, h], oi, rtol=0, atol=1e-12)
             assert lse[0, h, i] == pytest.approx(li, abs=1e-12)
+
+
+def test_fp4_per_tensor_factors():
+    # v_global scales O exactly and leaves LSE alone; q_global and k_global
+    # enter only through their product (the score factor).
+    t = make_tensors_fp4(1, 2, 2, 40, 40, 64, seed=12, scale=0.125)
+    o1, l1 = oracle.attn_fwd_fp4(*_args(t), scale=0.125, causal=True)
+    t2 = dict(t, v_global=2.0 * t["v_global"])
+    o2, l2 = oracle.attn_fwd_fp4(*_args(t2), scale=0.125, causal=True)
+    np.testing.assert_array_equal(o2, 2.0 * o1)
+    np.testing.assert_array_equal(l2, l1)
+    t3 = dict(t, q_global=4.0 * t["q_global"], k_global=t["k_global"] / 4.0)
+    o3, l3 = oracle.attn_fwd_fp4(*_args(t3), scale=0.125, causal=True)
+    np.testing.assert_array_equal(o3, o1)
+    np.testing.assert_array_equal(l3, l1)
 
 
 def test_fp4_pow2_scores_are_dyadic():
