@@ -189,7 +189,10 @@ ATTN_API attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v,
  * log2 scores by an integer changes no code, so the result does not depend
  * on the anchor.  A block whose maximum lies more than
  * 26 - ceil(rescale_threshold) octaves below the anchor contributes nothing
- * (its values would leave the normal range of the f16 container).
+ * (its values would leave the normal range of the f16 container).  Scores
+ * are handled in fp32 as in attn_fwd; log2 scores must stay below 2^21 in
+ * magnitude (beyond that fp32 cannot resolve their fractional part, on which
+ * the codes depend).
  *
  * Inputs (device memory, 16-byte aligned, caller-owned):
  *   q_codes  uint8 [B, Sq, Hq,  D/2]  two E2M1 codes per byte, element 2j
