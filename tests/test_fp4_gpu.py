@@ -69,6 +69,9 @@ CASES = [
     (1, 2, 2, 1, 1000, 128, dict(causal=True)),
     (1, 1, 1, 1, 1, 64, dict(causal=False)),
     (1, 3, 3, 129, 129, 128, dict(causal=False)),
+    # Sq > Sk, causal (bottom-right): the first 190 rows see no key
+    (1, 2, 2, 450, 260, 128, dict(causal=True)),
+    (1, 2, 1, 3, 4100, 64, dict(causal=True)),
 ]
 
 
