@@ -609,9 +609,10 @@ static double *decode_mxfp4_v(const uint8_t *codes, const uint8_t *scales, int B
 /*
  * Direct-P forward of NVFP4 Q/K and MXFP4 V.  classifier 1 = affine,
  * 2 = exponential.  The log2 score is <q', k'> * c with q', k' decoded
- * without their per-tensor factors and c = fp32(scale * q_global *
- * k_global * log2 e): the code decisions are taken on that value, the
- * precision in which the kernel takes them.  O includes v_global; LSE is in
+ * without their per-tensor factors and c = scale * q_global * k_global *
+ * log2 e in fp64: the code decisions are taken on the exact score (where c
+ * and the block scales are powers of two, fp32 holds the same value, so a
+ * kernel computing in fp32 takes the same decisions).  O includes v_global; LSE is in
  * natural units of the scores scale * <q, k>.  Layouts as the kernel's:
  * codes [B][S][H][D/2], Q/K scales [B][S][H][D/16], V scales
  * [B][ceil(Sk/32)][Hkv][D].
@@ -627,7 +628,7 @@ int oracle_attn_fwd_fp4(const uint8_t *q_codes, const uint8_t *q_scales, double 
     if (D % 32 != 0) return -1;
     const double softcap = 0.0;
     const double *alibi_slopes = NULL;
-    const double c = (double)(float)(scale * q_global * k_global * 1.4426950408889634);
+    const double c = scale * q_global * k_global * 1.4426950408889634;
     ORACLE_SHAPE;
     s.scale = c;
     s.direct_p = classifier;

@@ -111,26 +111,70 @@ def test_fp4_rescale_threshold_does_not_change_the_result(tau):
     _tight(o, lse, o_ref, lse_ref, _vmax(t))
 
 
+def drop_bounds(t, rows, scale, tau, classifier):
+    """Per-row bound on what the kernel's range guard may drop.
+
+    The kernel drops a 32-key block (aligned to the key index) whose
+    maximum log2 score lies more than 26 - ceil(tau) octaves below its
+    anchor, the running maximum rounded up to an integer (never above
+    ceil(M), M the row maximum).  So only blocks with floor(block max) <
+    ceil(M) - 26 + ceil(tau) can be dropped, and the kernel's output is the
+    Direct-P output of the row without some subset of them: the weights of
+    the kept blocks do not depend on the dropped ones.  With W_d / W the
+    fraction of the Direct-P weight in those blocks (from the oracle's row
+    function with and without them), |O - O_ref| <= 2 max|V| W_d / W and
+    |LSE - LSE_ref| <= -ln(1 - W_d / W).  Returns (frac [n], vmax_row [n])."""
+    q, k, v = _decode(t, "q"), _decode(t, "k"), _decode_v(t)
+    Hq, Hkv = q.shape[2], k.shape[2]
+    Sq, Sk = q.shape[1], k.shape[1]
+    frac, vrow = np.zeros(len(rows)), np.zeros(len(rows))
+    for r, (b, h, i) in enumerate(rows):
+        hk = h // (Hq // Hkv)
+        allow = np.arange(Sk) <= i + Sk - Sq
+        if not allow.any():
+            continue
+        y = (k[b, :, hk] @ q[b, i, h]) * (scale * 1.4426950408889634)
+        M = y[allow].max()
+        ym = np.where(allow, y, -np.inf)
+        nblk = (Sk + 31) // 32
+        bmax = np.array([ym[32 * g:32 * g + 32].max() for g in range(nblk)])
+        droppable = np.floor(bmax) < math.ceil(M) - 26 + math.ceil(tau)
+        keep = allow & ~np.repeat(droppable, 32)[:Sk]
+        vrow[r] = np.abs(v[b, allow, hk]).max()
+        if not droppable[np.isfinite(bmax)].any():
+            continue
+        _, l_all = oracle.direct_p_row(y, v[b, :, hk], allow=allow, classifier=classifier)
+        _, l_keep = oracle.direct_p_row(y, v[b, :, hk], allow=keep, classifier=classifier)
+        frac[r] = 1.0 - math.exp(l_keep - l_all) if keep.any() else 1.0
+    return frac, vrow
+
+
 @pytest.mark.parametrize("classifier", ["affine", "exp2"])
-def test_fp4_wide_logits(classifier):
+@pytest.mark.parametrize("tau", [0.0, 8.0])
+def test_fp4_wide_logits(classifier, tau):
     # Score factor 2^3 instead of ~2^-3: log2 scores spread over hundreds of
-    # units, so the anchor moves by large steps and most blocks sit far below
-    # it (the range guard).  The kernel drops a block whose maximum lies more
-    # than 26 - ceil(threshold) octaves below the anchor; with threshold 0
-    # each dropped key weighs under 2^-24 of the row maximum's weight (the
-    # anchor is at most one octave above the maximum), so the output may
-    # differ from the oracle's by at most Sk * 2^-24 * 2 max|V| beyond the
-    # rounding bound.
+    # units, so the anchor moves by large steps and many blocks sit far below
+    # it (the range guard).  Element-wise parity with a per-row bound for
+    # what the guard may drop (drop_bounds), at the default threshold 8 and
+    # at 0.
     S, D = 400, 128
     t = make_tensors_fp4(1, 2, 2, S, S, D, seed=41, scale=8.0)
     o, lse = _run(t, classifier, scale=8.0, causal=True,
-                  options=attn.fp4_options(rescale_threshold=0.0))
+                  options=attn.fp4_options(rescale_threshold=tau))
     o_ref, lse_ref = _ref(t, classifier, scale=8.0, causal=True)
     assert np.abs(lse_ref).max() > 100
-    vmax = _vmax(t)
-    err = np.abs(o - o_ref)
-    assert (err <= 2.0 ** -8 * np.abs(o_ref) + S * 2.0 ** -23 * vmax).all(), float(err.max())
-    assert np.abs(lse - lse_ref).max() <= 1e-4 * np.abs(lse_ref).max()
+    rows = np.array([(0, h, i) for h in range(2) for i in range(S)])
+    frac, vrow = drop_bounds(t, rows, 8.0, tau, classifier)
+    assert (frac > 0).any(), "no row has a block the guard may drop: the case tests nothing"
+    got = o[rows[:, 0], rows[:, 2], rows[:, 1]]
+    want = o_ref[rows[:, 0], rows[:, 2], rows[:, 1]]
+    bound = 2.0 ** -8 * np.abs(want) + 2.0 ** -20 * _vmax(t) + 2.0 * (frac * vrow)[:, None]
+    err = np.abs(got - want)
+    assert (err <= bound).all(), (float((err - bound).max()), int((err > bound).sum()))
+    l_got = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
+    l_want = lse_ref[rows[:, 0], rows[:, 1], rows[:, 2]]
+    l_bound = 2e-5 + 1e-6 * np.abs(l_want) - np.log1p(-np.minimum(frac, 1 - 1e-16))
+    assert (np.abs(l_got - l_want) <= l_bound).all(), float(np.abs(l_got - l_want).max())
 
 
 @pytest.mark.parametrize("classifier", ["affine", "exp2"])

@@ -261,8 +261,8 @@ def test_fp4_zero_queries_give_mean_of_values(classifier):
 @pytest.mark.parametrize("pow2", [True, False])
 def test_fp4_forward_is_direct_p_of_decoded_scores(classifier, pow2):
     # The entry point = its decoded inputs' scores fed to the pinned row
-    # function: checks NVFP4 / MXFP4 decoding, the score scale (fp32 c), GQA
-    # and the causal mask together.
+    # function: checks NVFP4 / MXFP4 decoding, the score scale (c = scale x
+    # q_global x k_global x log2 e), GQA and the causal mask together.
     B, Hq, Hkv, S, D = 1, 4, 2, 70, 64
     scale = 0.125
     t = make_tensors_fp4(B, Hq, Hkv, S, S, D, seed=8, scale=scale, pow2_scales=pow2)
@@ -270,7 +270,7 @@ def test_fp4_forward_is_direct_p_of_decoded_scores(classifier, pow2):
     q = _decode_nvfp4(t["q_codes"], t["q_scales"], 1.0)
     k = _decode_nvfp4(t["k_codes"], t["k_scales"], 1.0)
     v = _decode_mxfp4(t["v_codes"], t["v_scales"], t["v_global"])
-    c = float(np.float32(scale * t["q_global"] * t["k_global"] * 1.4426950408889634))
+    c = scale * t["q_global"] * t["k_global"] * 1.4426950408889634
     for h in range(Hq):
         hk = h // (Hq // Hkv)
         y = (q[0, :, h] @ k[0, :, hk].T) * c
