@@ -222,42 +222,24 @@ def test_deterministic_and_stream_aware():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-# ------------------------------------------- full-size workloads (sampled)
-
-def sample_rows(B, H, S, n_random, seed):
-    rng = np.random.default_rng(seed)
-    fixed = [0, 1, 2, 127, 128, 129, 255, 256, S // 2, S - 257, S - 129, S - 2, S - 1]
-    rows = []
-    for b in range(B):
-        for h in sorted({0, H - 1, int(rng.integers(H))}):
-            for i in fixed:
-                rows.append((b, h, i))
-    for _ in range(n_random):
-        rows.append((int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(S))))
-    return np.array(rows, dtype=np.int64)
-
+# ---------------------------------------------- full-size workloads (full)
 
 @pytest.mark.parametrize("name", ["outlier_s4096", "causal_s8192", "gqa_doc_s16384",
                                   "causal_bwd_s4096", "window_s16384"])
-def test_full_size_workload_sampled(name):
+def test_full_size_workload_full(name):
     """The benchmark's workloads at full size, in the benchmark's launch
-    configuration: sampled rows against the oracle, plus properties of every
-    row (finite O, finite LSE: every row here has at least one key)."""
+    configuration, compared with the oracle on every element of O and LSE:
+    max-abs and mean-abs over the whole tensor (every row here has at least
+    one key)."""
     w = WORKLOADS[name]
     t = make_inputs(w)
     window = None if tuple(w.window) == (-1, -1) else w.window
     o, lse = run_gpu(t, causal=w.causal, window=window, doc_offsets=t["doc_offsets"],
                      scale=w.scale)
     assert np.isfinite(o).all() and np.isfinite(lse).all()
-    rows = sample_rows(w.B, w.Hq, w.S, 200, seed=w.seed)
     o_ref, lse_ref = oracle.attn_fwd(t["q"], t["k"], t["v"], scale=w.scale, causal=w.causal,
-                                     window=window, doc_offsets=t["doc_offsets"], rows=rows)
-    o_s = o[rows[:, 0], rows[:, 2], rows[:, 1]]
-    lse_s = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
-    err = np.abs(o_s - o_ref)
-    assert err.max() <= O_MAX, f"{name}: O max-abs {err.max():.3e}"
-    assert err.mean() <= O_MEAN, f"{name}: O mean-abs {err.mean():.3e}"
-    assert np.abs(lse_s - lse_ref).max() <= LSE_TOL
+                                     window=window, doc_offsets=t["doc_offsets"])
+    check(o, lse, o_ref, lse_ref, name)
 
 
 # ----------------------------------------------------------- failure path

@@ -161,12 +161,19 @@ __device__ __forceinline__ bool use_poly(int col) {
 }
 
 // Half a row of a block: p = 2^(s*c - m) for 64 scores (packed pairs), the
-// exponentials split between MUFU and the polynomial per EXP_MODE; returns
-// the row sum and writes the bf16 pairs to pk.
+// exponentials split between MUFU and the polynomial per EXP_MODE; writes
+// the bf16 pairs to pk and adds to `sum` the row sum of the unrounded p (for
+// the LSE) and to `sum_pv` the sum of the bf16-rounded values, the weights
+// the tensor cores apply in PV.  The output is normalised by the latter, so
+// O is a convex combination of V rows with exactly those weights: a row
+// dominated by one key reproduces that key's V row even when its p (scaled
+// by a running maximum that may lag the true one by up to the rescale
+// threshold) is not a bf16 value.
 template <int EXP_MODE>
-__device__ __forceinline__ float exp_pack_half(const float *s, float c, float neg_m,
-                                               uint32_t *pk) {
+__device__ __forceinline__ void exp_pack_half(const float *s, float c, float neg_m, uint32_t *pk,
+                                              float &sum, float &sum_pv) {
     float sum0 = 0.0f, sum1 = 0.0f, sum2 = 0.0f, sum3 = 0.0f;
+    float r0s = 0.0f, r1s = 0.0f;
 #pragma unroll
     for (int e = 0; e < kBlockN / 2; e += 2) {
         float x0, x1, p0, p1;
@@ -179,9 +186,12 @@ __device__ __forceinline__ float exp_pack_half(const float *s, float c, float ne
         }
         if ((e & 2) == 0) add2(sum0, sum1, sum0, sum1, p0, p1);
         else add2(sum2, sum3, sum2, sum3, p0, p1);
-        pk[e >> 1] = pack_bf16x2(p0, p1);
+        const uint32_t h = pack_bf16x2(p0, p1);
+        pk[e >> 1] = h;
+        add_bf16x2_f32(r0s, r1s, h);
     }
-    return (sum0 + sum1) + (sum2 + sum3);
+    sum += (sum0 + sum1) + (sum2 + sum3);
+    sum_pv += r0s + r1s;
 }
 
 // The same for 8-bit P: 64 probabilities of a row to e4m3, four per word.
@@ -605,7 +615,8 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         const float k1 = p.softcap_in * (2.0f * kLog2eF);  // soft-cap: 2 log2(e) scale / cap
         const float diag_f = (float)(row + p.Sk - p.Sq);
         float m_run = -INFINITY;
-        float l_run = 0.0f;
+        float l_run = 0.0f;   // row sum of the unrounded p (the LSE's normaliser)
+        float l_pv = 0.0f;    // row sum of the p that PV consumes (the output's normaliser)
         bool ok = true;
 
         for (int j = lo_b; j <= hi_b; ++j) {
@@ -707,6 +718,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             }
 
             l_run *= alpha;
+            l_pv *= alpha;
 
             // Correction first: rescale this row of O in TMEM (rare once the
             // max settles) before any P of this block is handed over.  PV of
@@ -747,8 +759,8 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                                 : exp_pack_half_fp8<EXP_MODE>(s, c_exp, neg_m, pk);
                 tmem_st16(s_tmem + 0, pk + 0);
             } else {
-                l_run += masked ? exp_pack_half<0>(s, c_exp, neg_m, pk)
-                                : exp_pack_half<EXP_MODE>(s, c_exp, neg_m, pk);
+                if (masked) exp_pack_half<0>(s, c_exp, neg_m, pk, l_run, l_pv);
+                else exp_pack_half<EXP_MODE>(s, c_exp, neg_m, pk, l_run, l_pv);
                 tmem_st32(s_tmem + 0, pk + 0);
             }
             tmem_wait_st();
@@ -765,8 +777,8 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
                 tmem_st16(s_tmem + 16, pk + 16);
             } else {
-                l_run += masked ? exp_pack_half<0>(s + 64, c_exp, neg_m, pk + 32)
-                                : exp_pack_half<EXP_MODE>(s + 64, c_exp, neg_m, pk + 32);
+                if (masked) exp_pack_half<0>(s + 64, c_exp, neg_m, pk + 32, l_run, l_pv);
+                else exp_pack_half<EXP_MODE>(s + 64, c_exp, neg_m, pk + 32, l_run, l_pv);
                 if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4);
                 tmem_st32(s_tmem + 32, pk + 32);
             }
@@ -785,7 +797,11 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         }
         if (ok) {
             const bool row_ok = row < p.Sq;
-            const float inv_l = l_run > 0.0f ? (PREC ? p.v_descale : 1.0f) / l_run : 0.0f;
+            // bf16 P: normalise by the sum of the rounded weights PV applied;
+            // fp8 and Direct-P: by the row sum (the fp8 bound is derived for
+            // it; Direct-P's sum is already over the values PV consumes).
+            const float l_out = PREC ? l_run : l_pv;
+            const float inv_l = l_out > 0.0f ? (PREC ? p.v_descale : 1.0f) / l_out : 0.0f;
             __nv_bfloat16 *o_row =
                 p.o + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)D;
 #pragma unroll

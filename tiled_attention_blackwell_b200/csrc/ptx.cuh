@@ -407,6 +407,15 @@ __device__ __forceinline__ float f16x2_sum(uint32_t a) {
     return lo + hi;
 }
 
+// a0 += low bf16 half of h, a1 += high half, each converted exactly and
+// added in fp32 (sm_100 mixed-precision add: no separate unpacking).
+__device__ __forceinline__ void add_bf16x2_f32(float &a0, float &a1, uint32_t h) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(h));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
