@@ -186,6 +186,102 @@ def test_bwd_invalid_arguments_rejected_before_launch(L, kw, status):
     assert call_bwd(L, opts=attn.BwdOptions(), **kw) == status
 
 
+def call_noalloc(L, **kw):
+    a = dict(ptr=P, lse=P, B=1, Hq=2, Hkv=2, Sq=16, Sk=16, D=128, scale=0.1, causal=1,
+             wl=-1, wr=-1, docs=None, nd=0)
+    a.update(kw)
+    vp = ctypes.c_void_p
+    ptrs = [vp(a.get(n, a["ptr"])) for n in ("q", "k", "v", "o")]
+    ptrs += [vp(a["lse"])]
+    ptrs += [vp(a.get(n, a["ptr"])) for n in ("dout", "dq", "dk", "dv")]
+    return L.attn_bwd_noalloc(*ptrs, a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Sk"], a["D"],
+                              a["scale"], a["causal"], a["wl"], a["wr"],
+                              vp(a["docs"]) if a["docs"] else None, a["nd"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(dq=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(lse=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(B=0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), attn.ATTN_ERR_INVALID_ARG),
+    (dict(D=80), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=0.0), attn.ATTN_ERR_INVALID_ARG),
+    (dict(wl=-2), attn.ATTN_ERR_INVALID_ARG),
+    (dict(dk=P + 8), attn.ATTN_ERR_MISALIGNED),
+    (dict(lse=P + 2), attn.ATTN_ERR_MISALIGNED),
+    (dict(docs=P, nd=1, Sk=20), attn.ATTN_ERR_INVALID_ARG),
+    (dict(B=1, Hq=32, Hkv=32, Sq=32769, Sk=32769), attn.ATTN_ERR_UNSUPPORTED),
+])
+def test_noalloc_invalid_arguments_rejected_before_cuda(L, kw, status):
+    """attn_bwd_noalloc checks its arguments like attn_bwd, before it looks up
+    its scratch or touches CUDA: on a machine without a GPU a bad argument
+    still reports the argument error, not a CUDA error."""
+    assert call_noalloc(L, **kw) == status
+    assert L.attn_last_error_detail().decode() != ""
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
+def test_valid_noalloc_call_without_gpu_reports_cuda_error(L):
+    assert call_noalloc(L) == attn.ATTN_ERR_CUDA
+
+
+class _CudaStandIn(torch.Tensor):
+    """A CPU tensor that reports itself as a CUDA tensor, so the binding's
+    own checks can be exercised on a machine without a GPU (they must raise
+    before anything is passed to the library)."""
+
+    @property
+    def is_cuda(self):
+        return True
+
+
+def _bwd_stand_ins(B=1, S=16, H=2, D=64):
+    def mk(shape, dt):
+        return torch.zeros(shape, dtype=dt).as_subclass(_CudaStandIn)
+    q, k, v, o, dout = (mk((B, S, H, D), torch.bfloat16) for _ in range(5))
+    lse = mk((B, H, S), torch.float32)
+    dq = mk((B, S, H, D), torch.float32)
+    dk, dv = mk((B, S, H, D), torch.bfloat16), mk((B, S, H, D), torch.bfloat16)
+    return dict(q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv)
+
+
+@pytest.mark.parametrize("fn", ["attn_bwd_noalloc", "attn_bwd"])
+def test_backward_bindings_check_tensors_and_doc_offsets(L, fn):
+    """Both backward bindings refuse a bf16 dq (the kernel would write fp32
+    rows past its end), a non-contiguous tensor, and doc_offsets that are
+    not a CUDA int32 tensor (a host pointer or a list), before any call into
+    the library."""
+    call = getattr(attn, fn)
+    extra = ([torch.zeros(1024, dtype=torch.uint8).as_subclass(_CudaStandIn)]
+             if fn == "attn_bwd" else [])
+
+    def run(t, **kw):
+        names = ("q", "k", "v", "o", "lse", "dout", "dq", "dk", "dv")
+        call(*[t[n] for n in names], *extra, scale=0.1, causal=True, stream=0, **kw)
+
+    t = _bwd_stand_ins()
+    t["dq"] = torch.zeros(t["dq"].shape, dtype=torch.bfloat16).as_subclass(_CudaStandIn)
+    with pytest.raises(TypeError, match="dq"):
+        run(t)
+    t = _bwd_stand_ins()
+    t["dk"] = torch.zeros((1, 2, 16, 64), dtype=torch.bfloat16).transpose(1, 2) \
+        .as_subclass(_CudaStandIn)
+    with pytest.raises(TypeError, match="dk"):
+        run(t)
+    t = _bwd_stand_ins()
+    t["dv"] = torch.zeros((1, 16, 2, 32), dtype=torch.bfloat16).as_subclass(_CudaStandIn)
+    with pytest.raises(TypeError, match="dv"):
+        run(t)
+    t = _bwd_stand_ins()
+    with pytest.raises(TypeError, match="doc_offsets"):
+        run(t, doc_offsets=torch.tensor([0, 16], dtype=torch.int32))
+    with pytest.raises(TypeError, match="doc_offsets"):
+        run(t, doc_offsets=[0, 16])
+    with pytest.raises(TypeError, match="doc_offsets"):
+        run(t, doc_offsets=torch.tensor([0, 16]).as_subclass(_CudaStandIn))
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
 def test_valid_bwd_calls_without_gpu_report_cuda_error(L):
     assert call_bwd(L) == attn.ATTN_ERR_CUDA

@@ -356,6 +356,37 @@ def attention_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_co
     return o, lse
 
 
+def _check_bwd_tensors(q, k, v, o, lse, dout, dq, dk, dv):
+    """Dtype, device and layout of every tensor the backward kernels touch:
+    a wrong dtype would make a kernel read or write past a buffer's end."""
+    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
+                        ("v", v, torch.bfloat16), ("o", o, torch.bfloat16),
+                        ("lse", lse, torch.float32), ("dout", dout, torch.bfloat16),
+                        ("dq", dq, torch.float32), ("dk", dk, torch.bfloat16),
+                        ("dv", dv, torch.bfloat16)):
+        if not torch.is_tensor(t) or t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA {dt} tensor")
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    for name, t, shape in (("k", k, (B, Sk, Hkv, D)), ("v", v, (B, Sk, Hkv, D)),
+                           ("o", o, (B, Sq, Hq, D)), ("dout", dout, (B, Sq, Hq, D)),
+                           ("dq", dq, (B, Sq, Hq, D)), ("dk", dk, (B, Sk, Hkv, D)),
+                           ("dv", dv, (B, Sk, Hkv, D)), ("lse", lse, (B, Hq, Sq))):
+        if tuple(t.shape) != shape:
+            raise TypeError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+
+
+def _docs_arg(doc_offsets):
+    """(pointer, num_docs) of a CUDA int32 doc_offsets tensor, or (None, 0).
+    Anything else raises: the kernels read the offsets on the device."""
+    if doc_offsets is None:
+        return None, 0
+    if not torch.is_tensor(doc_offsets) or doc_offsets.dtype != torch.int32 \
+            or not doc_offsets.is_cuda or not doc_offsets.is_contiguous():
+        raise TypeError("doc_offsets must be a contiguous CUDA int32 tensor")
+    return _ptr(doc_offsets), doc_offsets.numel() - 1
+
+
 def bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D) -> int:
     """Bytes of device workspace attn_bwd needs."""
     return int(lib().attn_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D))
@@ -367,24 +398,13 @@ def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, *, scale, causal=Fals
     [B,Sk,Hkv,D]; workspace a CUDA uint8 tensor of at least
     bwd_workspace_size() bytes.  softcap / alibi_slopes must match the
     forward that produced o and lse."""
-    for name, t, dt in (("q", q, torch.bfloat16), ("k", k, torch.bfloat16),
-                        ("v", v, torch.bfloat16), ("o", o, torch.bfloat16),
-                        ("lse", lse, torch.float32), ("dout", dout, torch.bfloat16),
-                        ("dq", dq, torch.float32), ("dk", dk, torch.bfloat16),
-                        ("dv", dv, torch.bfloat16)):
-        if t.dtype != dt or not t.is_cuda or not t.is_contiguous():
-            raise TypeError(f"{name} must be a contiguous CUDA {dt} tensor")
-    if not workspace.is_cuda or not workspace.is_contiguous():
+    _check_bwd_tensors(q, k, v, o, lse, dout, dq, dk, dv)
+    if not torch.is_tensor(workspace) or not workspace.is_cuda or not workspace.is_contiguous():
         raise TypeError("workspace must be a contiguous CUDA tensor")
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
     wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
-    if doc_offsets is not None:
-        if doc_offsets.dtype != torch.int32 or not doc_offsets.is_cuda:
-            raise TypeError("doc_offsets must be a CUDA int32 tensor")
-        docs_ptr, nd = _ptr(doc_offsets), doc_offsets.numel() - 1
-    else:
-        docs_ptr, nd = None, 0
+    docs_ptr, nd = _docs_arg(doc_offsets)
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
             _ptr(dv), B, Hq, Hkv, Sq, Sk, D, float(scale), int(bool(causal)), wl, wr,
             docs_ptr, nd, _ptr(workspace), workspace.numel() * workspace.element_size()]
@@ -426,12 +446,14 @@ def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, *, scale, causal=False, 
     """attn_bwd for callers that cannot allocate device memory: the library
     uses its own fixed scratch (B*Hq*Sq <= 1048576 rows) instead of a
     workspace.  Calls that may run on the GPU at the same time must be
-    ordered by the caller (they share that scratch)."""
+    ordered by the caller (they share that scratch).  Tensor checks are those
+    of attn_bwd; doc_offsets must already be a CUDA int32 tensor (this entry
+    point never copies or allocates)."""
+    _check_bwd_tensors(q, k, v, o, lse, dout, dq, dk, dv)
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
     wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
-    docs_ptr, nd = (None, 0) if doc_offsets is None else (_ptr(doc_offsets),
-                                                           doc_offsets.numel() - 1)
+    docs_ptr, nd = _docs_arg(doc_offsets)
     st = lib().attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
                                 _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, D,
                                 float(scale), int(bool(causal)), wl, wr, docs_ptr, nd,

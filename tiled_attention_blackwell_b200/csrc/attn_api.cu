@@ -313,6 +313,28 @@ attn_status_t check_modifiers(float softcap, int reserved0, const float *alibi_s
     return ATTN_OK;
 }
 
+// Checks of the backward's tensors and shapes, shared by attn_bwd_ex and
+// attn_bwd_noalloc; no CUDA call.
+attn_status_t check_bwd_args(const void *q, const void *k, const void *v, const void *o,
+                             const float *lse, const void *dout, const float *dq, const void *dk,
+                             const void *dv, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                             float scale, int window_left, int window_right,
+                             const int *doc_offsets, int num_docs) {
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv)
+        return fail(ATTN_ERR_INVALID_ARG, "null pointer");
+    attn_status_t s = check_common(B, Hq, Hkv, Sq, Sk, D, scale, window_left, window_right,
+                                   doc_offsets, num_docs);
+    if (s != ATTN_OK) return s;
+    for (const void *ptr : {q, k, v, o, dout, (const void *)dq, dk, dv})
+        if (!aligned16(ptr)) return fail(ATTN_ERR_MISALIGNED, "tensors must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+        return fail(ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
+    const long long num_qb = (Sq + 127LL) / 128, num_kb = (Sk + 127LL) / 128;
+    if (num_qb * Hq * B > 0x7fffffffLL || num_kb * Hkv * B > 0x7fffffffLL)
+        return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+    return ATTN_OK;
+}
+
 #ifdef ATTN_TRACE
 long long *g_trace = nullptr;
 int g_trace_ctas = 0;
@@ -617,27 +639,20 @@ attn_status_t attn_bwd_ex(const void *q, const void *k, const void *v, const voi
                           const int *doc_offsets, int num_docs, void *workspace,
                           size_t workspace_bytes, const attn_bwd_options_t *opts,
                           void *stream) {
-    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
-        return fail(ATTN_ERR_INVALID_ARG, "null pointer");
-    attn_status_t s = check_common(B, Hq, Hkv, Sq, Sk, D, scale, window_left, window_right,
-                                   doc_offsets, num_docs);
+    attn_status_t s = check_bwd_args(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D,
+                                     scale, window_left, window_right, doc_offsets, num_docs);
     if (s != ATTN_OK) return s;
     attn_bwd_options_t op;
     memset(&op, 0, sizeof op);
     if (opts) op = *opts;
     if ((s = check_modifiers(op.softcap, op.reserved0, op.alibi_slopes, op.reserved, 4)) != ATTN_OK)
         return s;
-    for (const void *ptr : {q, k, v, o, dout, (const void *)dq, (const void *)dk, (const void *)dv,
-                            (const void *)workspace})
-        if (!aligned16(ptr)) return fail(ATTN_ERR_MISALIGNED, "tensors and workspace must be 16-byte aligned");
-    if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
-        return fail(ATTN_ERR_MISALIGNED, "lse must be 4-byte aligned");
+    if (!workspace) return fail(ATTN_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(workspace)) return fail(ATTN_ERR_MISALIGNED, "workspace must be 16-byte aligned");
     const size_t need = attn_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D);
     if (workspace_bytes < need)
         return fail(ATTN_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
     const long long num_qb = (Sq + 127LL) / 128, num_kb = (Sk + 127LL) / 128;
-    if (num_qb * Hq * B > 0x7fffffffLL || num_kb * Hkv * B > 0x7fffffffLL)
-        return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
 
     DeviceState *st = nullptr;
     if ((s = device_state(&st)) != ATTN_OK) return s;
@@ -689,8 +704,10 @@ attn_status_t attn_bwd_noalloc(const void *q, const void *k, const void *v, cons
                                void *dv, int B, int Hq, int Hkv, int Sq, int Sk, int D,
                                float scale, int causal, int window_left, int window_right,
                                const int *doc_offsets, int num_docs, void *stream) {
-    if (B < 1 || Hq < 1 || Sq < 1)
-        return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Sq must be >= 1");
+    // Every argument check comes before the first CUDA call.
+    attn_status_t s = check_bwd_args(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D,
+                                     scale, window_left, window_right, doc_offsets, num_docs);
+    if (s != ATTN_OK) return s;
     const long long rows = (long long)B * Hq * Sq;
     if (rows > (long long)kNoAllocRows)
         return fail(ATTN_ERR_UNSUPPORTED,
