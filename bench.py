@@ -70,6 +70,8 @@ def parse_args(argv=None):
                     help="time with ALiBi slopes 2^(-8(h+1)/Hq)")
     ap.add_argument("--classifier", default="affine", choices=["affine", "exp2"],
                     help="Direct-P code classifier of the fp4 workloads")
+    ap.add_argument("--sustained-seconds", type=float, default=2.0,
+                    help="length of the back-to-back run of the 'sustained' record (0: skip)")
     return ap.parse_args(argv)
 
 
@@ -476,6 +478,7 @@ def run_ours(args):
         torch.cuda.synchronize(device)
     barrier(world)
     attn.check_device_status(stream)
+    burst_clocks = sampler.summary()
     total_ms = t_begin.elapsed_time(t_end)
     launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     if flush is not None:
@@ -539,6 +542,30 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     e2e_value = flops * args.steps * world / (e2e_ms / 1e3) / 1e12
 
+    # ---- sustained: the same step back to back for a few seconds, so the
+    # clock settles where the power limit puts it; its own clock samples.
+    sustained = None
+    if args.sustained_seconds > 0:
+        n_sus = max(1, int(math.ceil(args.sustained_seconds * 1e3 / max(launch_avg_ms, 1e-3))))
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sus_sampler = ClockSampler(local, period_s=0.01)
+        torch.cuda.synchronize(device)
+        with sus_sampler:
+            s0.record(stream)
+            for _ in range(n_sus):
+                if flush is not None:
+                    flush.zero_()
+                step()
+            s1.record(stream)
+            torch.cuda.synchronize(device)
+        attn.check_device_status(stream)
+        sus_ms = s0.elapsed_time(s1)
+        sustained = {"launches": n_sus, "seconds": round(sus_ms / 1e3, 3),
+                     "value": round(flops * n_sus / (sus_ms / 1e3) / 1e12, 2), "unit": UNIT,
+                     "clocks": sus_sampler.summary()}
+        if flush is not None:
+            sustained["note"] = "includes the L2 flush between steps"
+
     peaks, peak_kind = read_peaks()
     achieved = flops / (launch_avg_ms / 1e3) / 1e12
     # fp8 contractions: the measured bf16 peak times the nominal dense
@@ -563,6 +590,8 @@ def run_ours(args):
                      "frac_of_sustained": round(achieved / (peak_mult * float(
                          peaks.get("bf16_tflops_sustained", peak))), 4),
                      "flops_per_launch": flops, "launch_ms": round(launch_avg_ms, 4),
+                     "cycles_per_launch": (round(launch_avg_ms * 1e-3 * burst_clocks["sm_mhz"] * 1e6)
+                                           if burst_clocks["sm_mhz"] else None),
                      "kernel": "attn_bwd (preprocess, dK/dV, dQ kernels per step)"
                      if w.backward else
                      ("attn_fwd_fp4 (fp4_dequant_kernel + attn_fwd_kernel, timed together)"
@@ -571,8 +600,13 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h,
                 "pipelining": "two buffer sets, copy-in / compute / copy-out streams"},
         "gpu_launches": args.steps * (3 if w.backward else 2 if fp4 else 1),
-        "clocks": sampler.summary(),
+        "clocks": burst_clocks,
     }
+    if sustained is not None:
+        sus_peak = peak_mult * float(peaks.get("bf16_tflops_sustained", peak))
+        sustained["frac_of_sustained_peak"] = round(sustained["value"] / sus_peak, 4)
+        sustained["peak"] = sus_peak
+        result["sustained"] = sustained
     inp["classifier"] = args.classifier
     if (rank == 0 and world == 1 and not args.no_cpu_baseline
             and slopes is None and args.softcap is None):
