@@ -72,6 +72,8 @@ def parse_args(argv=None):
                     help="Direct-P code classifier of the fp4 workloads")
     ap.add_argument("--sustained-seconds", type=float, default=2.0,
                     help="length of the back-to-back run of the 'sustained' record (0: skip)")
+    ap.add_argument("--no-rescale-stats", action="store_true",
+                    help="skip the rescale statistics (a separate process on the counting build)")
     return ap.parse_args(argv)
 
 
@@ -302,6 +304,22 @@ def kv_heads_for_seconds(w, inputs, seconds: float) -> int:
     about `seconds` (at least one, at most all of batch 0's)."""
     t1, _, _ = oracle_bwd_sample(w, inputs, 1)
     return int(min(max(1, seconds // max(t1, 1e-3)), w.Hkv))
+
+
+def rescale_stats(config: str, tau):
+    """How often the threshold skips the running-maximum rescale on this
+    workload: forwards at the run's threshold and at 0 through the counting
+    build of the library, in a process of its own (it loads that library
+    instead of the product's)."""
+    import subprocess
+    cmd = [sys.executable, "-m", "tiled_attention_blackwell_b200.rescale_stats", "--config",
+           config, "--tau", str(8.0 if tau is None else float(tau))]
+    try:
+        out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300,
+                             check=True).stdout
+        return [json.loads(line) for line in out.splitlines() if line.startswith("{")][-1]
+    except (subprocess.SubprocessError, ValueError, IndexError) as e:
+        return {"unavailable": str(e).splitlines()[0][:200]}
 
 
 def metric_for(w, softcap=None, alibi=False, classifier="affine") -> str:
@@ -607,6 +625,9 @@ def run_ours(args):
         sustained["frac_of_sustained_peak"] = round(sustained["value"] / sus_peak, 4)
         sustained["peak"] = sus_peak
         result["sustained"] = sustained
+    if (rank == 0 and world == 1 and not args.no_rescale_stats and not w.backward
+            and w.dtype == "bf16" and slopes is None and args.softcap is None):
+        result["rescale_stats"] = rescale_stats(w.name, args.rescale_threshold)
     inp["classifier"] = args.classifier
     if (rank == 0 and world == 1 and not args.no_cpu_baseline
             and slopes is None and args.softcap is None):

@@ -339,6 +339,9 @@ attn_status_t check_bwd_args(const void *q, const void *k, const void *v, const 
 long long *g_trace = nullptr;
 int g_trace_ctas = 0;
 #endif
+#ifdef ATTN_COUNT_RESCALES
+unsigned long long *g_rescale_counts = nullptr;
+#endif
 
 // ------------------------------------------ scratch of attn_bwd_noalloc
 // D_i of up to kNoAllocRows rows for callers that cannot allocate a
@@ -461,6 +464,9 @@ static attn_status_t fwd_impl(const void *q, const void *k, const void *v, void 
 #ifdef ATTN_TRACE
     p.trace = g_trace;
     p.trace_ctas = g_trace_ctas;
+#endif
+#ifdef ATTN_COUNT_RESCALES
+    p.rescale_counts = g_rescale_counts;
 #endif
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -592,6 +598,9 @@ attn_status_t attn_fwd_fp4(const void *q_codes, const void *q_scales, float q_gl
 #ifdef ATTN_TRACE
     p.trace = g_trace;
     p.trace_ctas = g_trace_ctas;
+#endif
+#ifdef ATTN_COUNT_RESCALES
+    p.rescale_counts = g_rescale_counts;
 #endif
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -771,6 +780,14 @@ int attn_abi_version(void) { return ATTN_ABI_VERSION; }
 ATTN_API void attn_trace_set_buffer(long long *device_buffer, int trace_ctas) {
     g_trace = device_buffer;
     g_trace_ctas = device_buffer ? trace_ctas : 0;
+}
+#endif
+#ifdef ATTN_COUNT_RESCALES
+// Counting builds only: device buffer of 4 uint64 that the bf16 / fp8 / FP4
+// forward kernels add their rescale statistics to (NULL disables); see
+// FwdParams::rescale_counts.
+ATTN_API void attn_count_set_buffer(unsigned long long *device_buffer) {
+    g_rescale_counts = device_buffer;
 }
 #endif
 

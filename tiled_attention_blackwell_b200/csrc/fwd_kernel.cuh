@@ -91,6 +91,11 @@ struct FwdParams {
     float scale_log2;
     float rescale_threshold;
     long long *trace;  // clock64 event log (trace builds only), else null
+    // Rescale statistics (counting builds only, else null): [0] blocks after
+    // a row's first, [1] of those that raise the row's running maximum (each
+    // a rescale of O without a threshold), [2] rescales taken under the
+    // threshold, [3] warp-level O corrections executed.
+    unsigned long long *rescale_counts;
     int trace_ctas;
     unsigned long long timeout_ns;  // bound of every wait
     int debug_withhold_kv;          // testing: CTA 0 skips its first K copy
@@ -122,6 +127,26 @@ constexpr int kTraceEvents = 8;
 #else
 #define ATTN_TRACE_EVENT(role, iter, ev) \
     do {                                 \
+    } while (0)
+#endif
+
+// Opt-in rescale statistics (compile with -DATTN_COUNT_RESCALES): each
+// softmax thread counts for its row, per key block after the first, whether
+// the block raises the running maximum and whether the threshold lets the
+// rescale happen; the counts are reduced per warp and added to
+// p.rescale_counts at the end.
+#ifdef ATTN_COUNT_RESCALES
+#define ATTN_COUNT_BLOCK(t, raises, taken) \
+    do {                                   \
+        if ((t) > 0) {                     \
+            ++cnt_blocks;                  \
+            cnt_raise += (raises) ? 1u : 0u; \
+            cnt_taken += (taken) ? 1u : 0u;  \
+        }                                  \
+    } while (0)
+#else
+#define ATTN_COUNT_BLOCK(t, raises, taken) \
+    do {                                   \
     } while (0)
 #endif
 
@@ -614,6 +639,9 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         const float slope2 = (MOD & 2) ? __ldg(p.alibi_slopes + hq) * kLog2eF : 0.0f;
         const float k1 = p.softcap_in * (2.0f * kLog2eF);  // soft-cap: 2 log2(e) scale / cap
         const float diag_f = (float)(row + p.Sk - p.Sq);
+#ifdef ATTN_COUNT_RESCALES
+        uint32_t cnt_blocks = 0, cnt_raise = 0, cnt_taken = 0, cnt_warp = 0;
+#endif
         float m_run = -INFINITY;
         float l_run = 0.0f;   // row sum of the unrounded p (the LSE's normaliser)
         float l_pv = 0.0f;    // row sum of the p that PV consumes (the output's normaliser)
@@ -664,6 +692,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) bm[u] = block_max32(s + 32 * u);
                 const float m_cand = fmax3(fmaxf(bm[0], bm[1]), bm[2], bm[3]) * c;
+                ATTN_COUNT_BLOCK(t, m_cand > m_run, m_cand > m_run + tau);
                 if (m_cand > m_run + tau) {
                     const float m_new = ceilf(m_cand);
                     alpha = exp2_neg_int(m_run - m_new);
@@ -706,6 +735,7 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 2);
             const float row_max = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
             const float m_cand = MOD ? row_max : row_max * c;
+            ATTN_COUNT_BLOCK(t, m_cand > m_run, m_cand > m_run + tau);
             if (m_cand > m_run + tau) {
                 alpha = ex2_mufu(m_run - m_cand);
                 m_run = m_cand;
@@ -725,6 +755,9 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
             // the previous block is complete: the commit that signalled S of
             // this block covers every earlier MMA.
             if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#ifdef ATTN_COUNT_RESCALES
+                ++cnt_warp;
+#endif
 #pragma unroll
                 for (int ch = 0; ch < D / 32; ++ch) {
                     uint32_t r[32];
@@ -834,6 +867,21 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
                 p.lse[((size_t)b * p.Hq + hq) * p.Sq + row] = lse;
             }
         }
+#ifdef ATTN_COUNT_RESCALES
+        if (p.rescale_counts) {
+            for (int o = 16; o > 0; o >>= 1) {
+                cnt_blocks += __shfl_xor_sync(0xffffffffu, cnt_blocks, o);
+                cnt_raise += __shfl_xor_sync(0xffffffffu, cnt_raise, o);
+                cnt_taken += __shfl_xor_sync(0xffffffffu, cnt_taken, o);
+            }
+            if (lane == 0) {
+                atomicAdd(p.rescale_counts + 0, (unsigned long long)cnt_blocks);
+                atomicAdd(p.rescale_counts + 1, (unsigned long long)cnt_raise);
+                atomicAdd(p.rescale_counts + 2, (unsigned long long)cnt_taken);
+                atomicAdd(p.rescale_counts + 3, (unsigned long long)cnt_warp);
+            }
+        }
+#endif
     }
 
     // ------------------------------------------------------------ teardown
