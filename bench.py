@@ -411,8 +411,8 @@ def run_ours(args):
         cfg["alibi"] = "slopes 2^(-8(h+1)/Hq)"
     if w.backward:
         # Backward workload: O and LSE come from one forward (with the same
-        # score modifiers) before timing; a step is one attn_bwd (preprocess,
-        # dK/dV and dQ kernels).
+        # score modifiers) before timing; a step is one attn_bwd (the dQ
+        # kernel, which also forms the D_i row terms, then the dK/dV kernel).
         flops *= 2.5
         attn.attn_fwd(dev["q"], dev["k"], dev["v"], o, lse, scale=w.scale, causal=w.causal,
                       window=window, doc_offsets=docs, softcap=args.softcap,
@@ -610,14 +610,14 @@ def run_ours(args):
                      "flops_per_launch": flops, "launch_ms": round(launch_avg_ms, 4),
                      "cycles_per_launch": (round(launch_avg_ms * 1e-3 * burst_clocks["sm_mhz"] * 1e6)
                                            if burst_clocks["sm_mhz"] else None),
-                     "kernel": "attn_bwd (preprocess, dK/dV, dQ kernels per step)"
+                     "kernel": "attn_bwd (dQ kernel with the D_i row terms, then dK/dV kernel)"
                      if w.backward else
                      ("attn_fwd_fp4 (fp4_dequant_kernel + attn_fwd_kernel, timed together)"
                       if fp4 else "attn_fwd_kernel")},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "pipelining": "two buffer sets, copy-in / compute / copy-out streams"},
-        "gpu_launches": args.steps * (3 if w.backward else 2 if fp4 else 1),
+        "gpu_launches": args.steps * (2 if w.backward or fp4 else 1),
         "clocks": burst_clocks,
     }
     if sustained is not None:

@@ -269,7 +269,6 @@ attn_status_t launch_bwd(const tab::BwdParams &p, cudaStream_t stream) {
     constexpr size_t smem_dkdv = sizeof(DkdvS) + 1024;
     constexpr size_t smem_dq = sizeof(DqS) + 1024;
     static_assert(smem_dkdv <= 232448 && smem_dq <= 232448, "shared memory budget");
-    auto k_pre = tab::attn_bwd_preprocess_kernel<D>;
     auto k_dkdv = tab::attn_bwd_dkdv_kernel<D, kBwdStagesQ, MOD>;
     auto k_dq = tab::attn_bwd_dq_kernel<D, bwd_k_stages(D), bwd_v_stages(D), MOD>;
     static std::once_flag once[kMaxDevices];
@@ -281,10 +280,10 @@ attn_status_t launch_bwd(const tab::BwdParams &p, cudaStream_t stream) {
         if (prep[dev] == ATTN_OK) prep[dev] = prepare_kernel(k_dq, smem_dq, tab::kBwdThreads, 0);
     });
     if (prep[dev] != ATTN_OK) return fail(prep[dev], "backward kernels could not be prepared");
-    const long long rows = (long long)p.B * p.Sq * p.Hq;
-    k_pre<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p);
-    k_dkdv<<<p.num_kb * p.Hkv * p.B, tab::kBwdThreads, smem_dkdv, stream>>>(p);
+    // dQ first: it also computes D_i into the workspace, which the dK/dV
+    // kernel reads.
     k_dq<<<p.num_qb * p.Hq * p.B, tab::kBwdThreads, smem_dq, stream>>>(p);
+    k_dkdv<<<p.num_kb * p.Hkv * p.B, tab::kBwdThreads, smem_dkdv, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ATTN_ERR_LAUNCH, "launch: %s", cudaGetErrorString(e));
     return ok();

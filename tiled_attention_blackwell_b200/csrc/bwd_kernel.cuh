@@ -8,18 +8,19 @@
 // D_i = sum_d dO_id O_id, P = exp(s - LSE), dP = dO V^T, dS = P (dP - D):
 //   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
 //
-// Three kernels, no atomics (deterministic):
-//   attn_bwd_preprocess_kernel  D_i into the caller's workspace
+// Two kernels, no atomics (deterministic), dQ first:
+//   attn_bwd_dq_kernel          one CTA per (batch, query head, 128-row
+//                               block): D_i of its rows (from O and dO,
+//                               also stored in the caller's workspace),
+//                               S = Q K^T, dP = dO V^T, dS into TMEM,
+//                               dQ += dS K.
 //   attn_bwd_dkdv_kernel        one CTA per (batch, kv head, 128-key block):
 //                               keys in TMEM lanes, S^T = K Q^T and
 //                               dP^T = V dO^T per query block, P^T and dS^T
 //                               written back into TMEM as bf16, then
 //                               dV += P^T dO and dK += dS^T Q (A from TMEM);
 //                               the query heads of a GQA group accumulate
-//                               into the same TMEM.
-//   attn_bwd_dq_kernel          one CTA per (batch, query head, 128-row
-//                               block): S = Q K^T, dP = dO V^T, dS into
-//                               TMEM, dQ += dS K.
+//                               into the same TMEM; D_i from the workspace.
 // Warp roles in both main kernels (320 threads): warps 0-7 elementwise
 // (warps 0-3 take columns [0, 64) of each 128-wide tile, warps 4-7 columns
 // [64, 128); one TMEM lane per thread; the work is purely elementwise, so the
@@ -128,37 +129,6 @@ __device__ __forceinline__ void bwd_modified_pair(float &x0, float &x1, float &f
     } while (0)
 #endif
 
-// --------------------------------------------------------------- preprocess
-
-// One warp per (b, i, hq) row: D_i = sum_d dO_id * O_id in fp32.
-template <int D>
-__global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const BwdParams p) {
-    const long long rows = (long long)p.B * p.Sq * p.Hq;
-    const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (w >= rows) return;
-    const int lane = threadIdx.x & 31;
-    float acc = 0.0f;
-    for (int d = lane * 4; d < D; d += 128) {
-        const uint2 ov = *reinterpret_cast<const uint2 *>(p.o + w * D + d);
-        const uint2 gv = *reinterpret_cast<const uint2 *>(p.dout + w * D + d);
-        const __nv_bfloat162 *o2 = reinterpret_cast<const __nv_bfloat162 *>(&ov);
-        const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&gv);
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const float2 of = __bfloat1622float2(o2[e]);
-            const float2 gf = __bfloat1622float2(g2[e]);
-            acc = fmaf(of.x, gf.x, acc);
-            acc = fmaf(of.y, gf.y, acc);
-        }
-    }
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-        const int hq = (int)(w % p.Hq);
-        const int i = (int)((w / p.Hq) % p.Sq);
-        const int b = (int)(w / ((long long)p.Hq * p.Sq));
-        p.dval[((size_t)b * p.Hq + hq) * p.Sq + i] = acc;
-    }
-}
 
 // --------------------------------------------------------------- dK and dV
 
@@ -633,6 +603,7 @@ struct DqSmem {
     uint32_t tmem_base;
     int abort_flag;
     int range[2];
+    float dpart[2][128];  // D_i of each row, per half of the columns
 };
 
 template <int D, int NK, int NV, int MOD = 0>
@@ -832,7 +803,33 @@ attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
         const KeyRange kr = row_ok ? row_key_range(p, row) : KeyRange{1, 0};
         const size_t ri = ((size_t)b * p.Hq + hq) * p.Sq + (row_ok ? row : 0);
         const float l2 = row_ok ? __ldg(p.lse + ri) * kLog2e : INFINITY;
-        const float dval = row_ok ? p.dval[ri] : 0.0f;
+        // D_i = sum_d dO_id O_id of this row: each warpgroup over its half of
+        // the columns, the halves added in a fixed order through shared
+        // memory; warpgroup 0 stores it for the dK/dV kernel, which runs after
+        // this one.  (The loads overlap the first S and dP products.)
+        float dval;
+        {
+            float a0 = 0.0f, a1 = 0.0f;
+            if (row_ok) {
+                const size_t off = (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)D + h * (D / 2);
+                const uint4 *o4 = reinterpret_cast<const uint4 *>(p.o + off);
+                const uint4 *g4 = reinterpret_cast<const uint4 *>(p.dout + off);
+#pragma unroll
+                for (int ch = 0; ch < D / 16; ++ch) {
+                    const uint4 ov = ld_nc_v4(o4 + ch), gv = ld_nc_v4(g4 + ch);
+                    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+                    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        fma2(a0, a1, __uint_as_float(ow[e] << 16), __uint_as_float(ow[e] & 0xffff0000u),
+                             __uint_as_float(gw[e] << 16), __uint_as_float(gw[e] & 0xffff0000u), a0, a1);
+                }
+            }
+            sm.dpart[h][row_in] = a0 + a1;
+            named_bar_sync(1, 256);  // the 256 elementwise threads, all of which reach it
+            dval = sm.dpart[0][row_in] + sm.dpart[1][row_in];
+            if (h == 0 && row_ok) p.dval[ri] = dval;
+        }
         const float c = p.scale_log2;
         const float slope2 = (MOD & 2) ? __ldg(p.alibi_slopes + hq) * kLog2e : 0.0f;
         bool ok = true;

@@ -75,6 +75,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Named barrier `id` (1..15; 0 is __syncthreads) over `count` threads, a
+// multiple of 32; every participating thread must reach it.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// 16 bytes of read-only global data.
+__device__ __forceinline__ uint4 ld_nc_v4(const void *ptr) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(ptr));
+    return v;
+}
+
 // Read-only global load issued where it stands (volatile: the compiler
 // neither drops nor sinks it toward its use).
 __device__ __forceinline__ float ld_nc_f32(const float *ptr) {
