@@ -43,6 +43,8 @@ UNIT = "TFLOP/s"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["tiled_attention_blackwell_b200/csrc/fwd_kernel.cuh",
+                  "tiled_attention_blackwell_b200/csrc/fwd_persistent.cuh",
+                  "tiled_attention_blackwell_b200/csrc/bwd_kernel.cuh",
                   "tiled_attention_blackwell_b200/csrc/common.cuh",
                   "tiled_attention_blackwell_b200/csrc/ptx.cuh",
                   "tiled_attention_blackwell_b200/csrc/exp2_poly.cuh",

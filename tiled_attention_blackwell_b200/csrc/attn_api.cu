@@ -10,11 +10,13 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/attn.h"
 #include "bwd_kernel.cuh"
 #include "fp4_dequant.cuh"
 #include "fwd_kernel.cuh"
+#include "fwd_persistent.cuh"
 
 namespace {
 
@@ -132,12 +134,18 @@ attn_status_t make_map_tile(CUtensorMap *map, const void *base, int B, int S, in
 
 // --------------------------------------------------------------- launching
 
-template <int D, int NS, int EXP, int MOD = 0, int PREC = 0>
+// PERSIST selects the persistent kernel (fwd_persistent.cuh: one CTA per SM
+// running many items), otherwise one CTA per item.
+template <int D, int NS, int EXP, int MOD = 0, int PREC = 0, bool PERSIST = false>
 attn_status_t launch_fwd(const tab::FwdParams &p, int grid, cudaStream_t stream) {
-    using Smem = tab::FwdSmem<D, NS, PREC == 1 ? 1 : 2>;
+    using Smem = std::conditional_t<PERSIST, tab::FwdSmemPersistent<D, NS, PREC == 1 ? 1 : 2>,
+                                    tab::FwdSmem<D, NS, PREC == 1 ? 1 : 2>>;
     constexpr size_t smem = sizeof(Smem) + 1024;
     static_assert(smem <= 232448, "shared memory budget");
-    auto kernel = tab::attn_fwd_kernel<D, NS, EXP, MOD, PREC>;
+    auto kernel = []() {
+        if constexpr (PERSIST) return tab::attn_fwd_persistent_kernel<D, NS, EXP, MOD, PREC>;
+        else return tab::attn_fwd_kernel<D, NS, EXP, MOD, PREC>;
+    }();
     static std::once_flag once[kMaxDevices];
     static cudaError_t attr_err[kMaxDevices];
     int dev = 0;
@@ -173,6 +181,19 @@ constexpr int kStagesD128 = 4;
 // 8 beats 4, 16 and all heads for the first two; with 4 query heads per
 // key/value head the group covers 32 query heads.
 constexpr int kFwdHeadGroup = 8;
+
+// (batch, query head) pairs per schedule group of the persistent forward.
+// A group's items are dealt to the CTAs in snake rounds, so the group should
+// span several rounds (a round boundary falling inside a group costs
+// balance) while keeping each round's items on few heads (K/V reuse in L2):
+// at least the kFwdHeadGroup key/value heads' query heads and a quarter of
+// a round of pairs, rounded up to whole key/value heads.
+int fwd_schedule_group(int B, int Hq, int Hkv, int ctas) {
+    const int qpk = Hq / Hkv;
+    int g = std::max(kFwdHeadGroup * qpk, (ctas + 3) / 4);
+    g = (g + qpk - 1) / qpk * qpk;
+    return std::min(B * Hq, g);
+}
 constexpr int kStagesD64 = 8;
 constexpr int kStagesFp8 = 8;  // fp8 K/V tiles are 16 KB at D = 128
 
@@ -193,11 +214,13 @@ attn_status_t dispatch_exp(const tab::FwdParams &p, int grid, int exp_mode, int 
     }
 }
 
+// The fp8 forward runs persistent (measured 6 % faster than one CTA per item
+// at causal S=8192; for bf16 operands the persistent kernel is slower).
 attn_status_t dispatch_fp8(const tab::FwdParams &p, int grid, int exp_mode, cudaStream_t s) {
     switch (exp_mode) {
-        case 0: return launch_fwd<128, kStagesFp8, 0, 0, 1>(p, grid, s);
-        case 1: return launch_fwd<128, kStagesFp8, 1, 0, 1>(p, grid, s);
-        default: return launch_fwd<128, kStagesFp8, 2, 0, 1>(p, grid, s);
+        case 0: return launch_fwd<128, kStagesFp8, 0, 0, 1, true>(p, grid, s);
+        case 1: return launch_fwd<128, kStagesFp8, 1, 0, 1, true>(p, grid, s);
+        default: return launch_fwd<128, kStagesFp8, 2, 0, 1, true>(p, grid, s);
     }
 }
 
@@ -412,13 +435,15 @@ static attn_status_t fwd_impl(const void *q, const void *k, const void *v, void 
             return fail(ATTN_ERR_INVALID_ARG, "the fp8 forward needs rescale_threshold <= 8");
     }
     const long long num_qblocks = (Sq + 2LL * tab::kBlockM - 1) / (2LL * tab::kBlockM);
-    const long long grid = num_qblocks * Hq * B;
-    if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+    const long long items = num_qblocks * Hq * B;
+    if (items > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
 
     // ----- set-up
     DeviceState *st = nullptr;
     attn_status_t s = device_state(&st);
     if (s != ATTN_OK) return s;
+    // One CTA per item, or (persistent fp8 kernel) one per SM.
+    const int grid = fp8 ? (int)std::min<long long>(items, st->num_sms) : (int)items;
 
     tab::FwdParams p;
     memset(&p, 0, sizeof p);
@@ -441,7 +466,8 @@ static attn_status_t fwd_impl(const void *q, const void *k, const void *v, void 
     p.window_left = window_left;
     p.window_right = window_right;
     p.num_qblocks = (int)num_qblocks;
-    p.head_group = std::min(B * Hq, kFwdHeadGroup * (Hq / Hkv));
+    p.head_group = fp8 ? fwd_schedule_group(B, Hq, Hkv, grid)
+                       : std::min(B * Hq, kFwdHeadGroup * (Hq / Hkv));
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     if (fp8) {
         p.scale_log2 = (float)((double)scale * q_descale * k_descale * 1.4426950408889634);
@@ -469,9 +495,9 @@ static attn_status_t fwd_impl(const void *q, const void *k, const void *v, void 
 #endif
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (fp8) return dispatch_fp8(p, (int)grid, op.exp2_mode, cs);
-    if (D == 128) return dispatch_exp<128, kStagesD128>(p, (int)grid, op.exp2_mode, mod, cs);
-    return dispatch_exp<64, kStagesD64>(p, (int)grid, op.exp2_mode, mod, cs);
+    if (fp8) return dispatch_fp8(p, grid, op.exp2_mode, cs);
+    if (D == 128) return dispatch_exp<128, kStagesD128>(p, grid, op.exp2_mode, mod, cs);
+    return dispatch_exp<64, kStagesD64>(p, grid, op.exp2_mode, mod, cs);
 }
 
 attn_status_t attn_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse,
