@@ -465,7 +465,8 @@ int oracle_attn_fwd_e4m3(const uint8_t *q, const uint8_t *k, const uint8_t *v,
  *     mantissa; exponent field 0 holds the subnormal m * 0.5.  The eight
  *     magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6.
  *   NVFP4: one e4m3 scale per 16 consecutive elements of a row (along D)
- *     times a per-tensor fp32 factor: x = g * e4m3(scale) * e2m1(code).
+ *     times a per-tensor fp32 factor: x = g * e4m3(scale) * e2m1(code); the
+ *     scale is an unsigned magnitude (nvfp4_scale_to_double).
  *   MXFP4: one UE8M0 scale (2^(u - 127), u = 255 is NaN) per 32 elements:
  *     here 32 consecutive keys of one (batch, head, d) column of V, the
  *     contraction direction of PV, times a per-tensor factor.
@@ -573,6 +574,16 @@ int oracle_direct_p_row(const double *y, const unsigned char *allow, int64_t n,
     return 0;
 }
 
+/* An NVFP4 block scale: an unsigned e4m3 magnitude (the pages name NVFP4
+ * for Q and K without a sign rule; the format's scale, as the FP4 tensor
+ * cores read it, has none).  A byte outside the format -- NaN, or the sign
+ * bit set with a nonzero magnitude -- makes its block read as 0 (the library
+ * reports ATTN_ERR_RANGE for it); -0 is a zero scale. */
+static double nvfp4_scale_to_double(uint8_t s) {
+    if ((s & 0x7F) == 0x7F || s > 0x80) return 0.0;
+    return e4m3_to_double((uint8_t)(s & 0x7F));
+}
+
 /* NVFP4 tensor of n elements (rows of D, D a multiple of 16) to doubles,
  * times `mul`. */
 static double *decode_nvfp4(const uint8_t *codes, const uint8_t *scales, size_t n,
@@ -581,7 +592,7 @@ static double *decode_nvfp4(const uint8_t *codes, const uint8_t *scales, size_t 
     if (!d) return NULL;
     for (size_t t = 0; t < n; ++t) {
         const unsigned c = (codes[t / 2] >> (4 * (t & 1))) & 15u;
-        d[t] = mul * e4m3_to_double(scales[t / 16]) * e2m1_to_double(c);
+        d[t] = mul * nvfp4_scale_to_double(scales[t / 16]) * e2m1_to_double(c);
     }
     return d;
 }

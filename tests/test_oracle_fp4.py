@@ -296,6 +296,32 @@ def test_fp4_per_tensor_factors():
     np.testing.assert_array_equal(l3, l1)
 
 
+def test_fp4_out_of_format_nvfp4_scales_read_as_zero():
+    # An NVFP4 scale is an unsigned e4m3 magnitude: a block whose scale byte
+    # is NaN or has the sign bit set with a nonzero magnitude reads as 0,
+    # exactly as if its 16 codes were zero; -0 (0x80) is a zero scale.
+    t = make_tensors_fp4(1, 2, 2, 50, 50, 64, seed=13, scale=0.125)
+    base, base_l = oracle.attn_fwd_fp4(*_args(t), scale=0.125, causal=True)
+    zeroed = dict(t, q_codes=t["q_codes"].clone(), k_codes=t["k_codes"].clone())
+    zeroed["q_codes"][0, 7, 1, 8:16] = 0      # Q row 7, head 1, elements 16-31
+    zeroed["k_codes"][0, 20, 0, 0:8] = 0      # K row 20, head 0, elements 0-15
+    want, want_l = oracle.attn_fwd_fp4(*_args(zeroed), scale=0.125, causal=True)
+    assert not np.array_equal(want, base)     # the blocks mattered
+    for qs, ks in ((0x7F, 0xFF), (0xB8, 0x81), (0x80 | 0x30, 0x80 | 0x7E)):
+        bad = dict(t, q_scales=t["q_scales"].clone(), k_scales=t["k_scales"].clone())
+        bad["q_scales"][0, 7, 1, 1] = qs
+        bad["k_scales"][0, 20, 0, 0] = ks
+        got, got_l = oracle.attn_fwd_fp4(*_args(bad), scale=0.125, causal=True)
+        np.testing.assert_array_equal(got, want)
+        np.testing.assert_array_equal(got_l, want_l)
+    neg0 = dict(t, q_scales=t["q_scales"].clone(), k_scales=t["k_scales"].clone())
+    neg0["q_scales"][0, 7, 1, 1] = 0x80
+    neg0["k_scales"][0, 20, 0, 0] = 0x80
+    got, got_l = oracle.attn_fwd_fp4(*_args(neg0), scale=0.125, causal=True)
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal(got_l, want_l)
+
+
 def test_fp4_pow2_scores_are_dyadic():
     # With power-of-two block scales and c a power of two, every log2 score
     # is a multiple of a small power of two far inside fp32's 24 bits: the

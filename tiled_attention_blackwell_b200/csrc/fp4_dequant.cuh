@@ -15,8 +15,9 @@
 //          of each (b, h, d) column, scales [B][ceil(S/32)][H][D];
 //          value = 2^(u - 127) * e2m1(code), exact in f16 (and in its normal
 //          range) for u - 127 in [-13, 13].
-// A nonzero code whose scale is NaN or outside that range is written as 0
-// and makes the kernel record ATTN_ERR_RANGE in the device status word.
+// A nonzero code whose scale is NaN, negative (NVFP4: the scale is an
+// unsigned magnitude) or outside that range (MXFP4) is written as 0 and
+// makes the kernel record ATTN_ERR_RANGE in the device status word.
 #pragma once
 
 #include "common.cuh"
@@ -94,12 +95,14 @@ __global__ void __launch_bounds__(256) fp4_dequant_kernel(const __grid_constant_
             for (int half = 0; half < 2; ++half) {
                 const uint32_t sb = (s2 >> (8 * half)) & 0xFFu;
                 const uint32_t scale2 = e4m3x2_to_f16x2(sb | (sb << 8));
-                const bool nan_scale = (sb & 0x7Fu) == 0x7Fu;
+                // NaN, or negative with a nonzero magnitude: outside the format
+                // (the scale is an unsigned e4m3 magnitude; -0 scales to zero).
+                const bool bad_scale = (sb & 0x7Fu) == 0x7Fu || sb > 0x80u;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t byte = (cws[2 * half + (k >> 2)] >> (8 * (k & 3))) & 0xFFu;
-                    bad |= nan_scale && (byte & 0x77u) != 0u;
-                    w[8 * half + k] = nan_scale ? 0u : hmul2_u32(w[8 * half + k], scale2);
+                    bad |= bad_scale && (byte & 0x77u) != 0u;
+                    w[8 * half + k] = bad_scale ? 0u : hmul2_u32(w[8 * half + k], scale2);
                 }
             }
         } else {
