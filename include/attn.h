@@ -189,7 +189,9 @@ ATTN_API attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v,
  * log2 scores by an integer changes no code, so the result does not depend
  * on the anchor.  A block whose maximum lies more than
  * 26 - ceil(rescale_threshold) octaves below the anchor contributes nothing
- * (its values would leave the normal range of the f16 container).  Scores
+ * (its values would leave the normal range of the f16 container; both
+ * product paths below apply the same rule, so they compute the same codes
+ * and weights).  Scores
  * are handled in fp32 as in attn_fwd; log2 scores must stay below 2^21 in
  * magnitude (beyond that fp32 cannot resolve their fractional part, on which
  * the codes depend).
@@ -203,18 +205,33 @@ ATTN_API attn_status_t attn_fwd_fp8(const void *q, const void *k, const void *v,
  *   v_scales uint8 [B, ceil(Sk/32), Hkv, D]  UE8M0 scale (2^(u - 127)) per
  *            32 keys of each (batch, head, d) column of V
  *   q_global, k_global, v_global: per-tensor fp32 factors, > 0 and finite.
- * A nonzero code whose scale is NaN, or (V) whose u - 127 lies outside
- * [-13, 13], reads as 0 and makes attn_get_device_status() report
- * ATTN_ERR_RANGE.
+ * An NVFP4 block scale is an unsigned e4m3 magnitude (the scale format of
+ * the FP4 tensor cores; -0 is a zero scale).  A nonzero code whose scale is
+ * NaN or negative (sign bit set, nonzero magnitude), or (V) whose u - 127
+ * lies outside [-13, 13], reads as 0 and makes attn_get_device_status()
+ * report ATTN_ERR_RANGE.
  * Outputs: o bf16 [B, Sq, Hq, D], lse fp32 [B, Hq, Sq].
  * workspace: at least attn_fwd_fp4_workspace_size() bytes, 16-byte aligned
- * (Q, K, V widened to f16, exactly; contents on entry ignored).
+ * (contents on entry ignored).
  * D must be 64 or 128; masks, GQA and shape rules as attn_fwd; no score
- * modifiers.  Both products run on the tensor cores with f16 operands that
- * hold the FP4 values exactly and fp32 accumulation.  opts may be NULL.
+ * modifiers.  opts may be NULL.
+ *
+ * Products (opts->mma).  ATTN_FP4_MMA_BLOCK_SCALED (D = 128): both run on
+ * the block-scaled FP4 tensor cores, Q K^T as NVFP4 x NVFP4 (kind::mxf4nvf4,
+ * UE4M3 scale per 16) and P V as MXFP4 x MXFP4 (kind::mxf4, UE8M0 scale per
+ * 32 keys: P's codes with their 2^E_g, V's with its scales); a preparation
+ * pass lays the scales out for tensor memory and transposes V's codes into
+ * the workspace.  ATTN_FP4_MMA_F16: a pass widens Q, K, V to f16 (exactly)
+ * in the workspace and both products run as f16 MMAs.  Every product of two
+ * FP4 values is exact in fp32, so the paths differ only in the order of the
+ * fp32 accumulation.  ATTN_FP4_MMA_AUTO (default): block-scaled for D = 128,
+ * f16 for D = 64.
  */
 #define ATTN_DIRECT_P_AFFINE 0
 #define ATTN_DIRECT_P_EXP2 1
+#define ATTN_FP4_MMA_AUTO 0
+#define ATTN_FP4_MMA_F16 1
+#define ATTN_FP4_MMA_BLOCK_SCALED 2
 
 typedef struct {
     /* Online rescale threshold of the integer anchor, in log2 units,
@@ -225,7 +242,10 @@ typedef struct {
     /* Bound of every device-side wait, microseconds (0 = 1 s); as in
      * attn_fwd_options_t.  Valid range [0, 60000000]. */
     int wait_timeout_us;
-    int reserved[5]; /* must be zero */
+    /* ATTN_FP4_MMA_AUTO (default), ATTN_FP4_MMA_F16 or
+     * ATTN_FP4_MMA_BLOCK_SCALED (D = 128 only, else ATTN_ERR_UNSUPPORTED). */
+    int mma;
+    int reserved[4]; /* must be zero */
 } attn_fp4_options_t;
 
 /* Fills *opts with the defaults. */

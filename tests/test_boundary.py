@@ -347,7 +347,8 @@ def test_option_structs_match_the_c_layout(tmp_path):
         "  F(attn_bwd_options_t, softcap); F(attn_bwd_options_t, reserved0);\n"
         "  F(attn_bwd_options_t, alibi_slopes); F(attn_bwd_options_t, reserved);\n"
         "  F(attn_fp4_options_t, rescale_threshold); F(attn_fp4_options_t, classifier);\n"
-        "  F(attn_fp4_options_t, wait_timeout_us); F(attn_fp4_options_t, reserved);\n"
+        "  F(attn_fp4_options_t, wait_timeout_us); F(attn_fp4_options_t, mma);\n"
+        "  F(attn_fp4_options_t, reserved);\n"
         "  return 0;\n}\n")
     exe = tmp_path / "layout"
     import subprocess
@@ -370,10 +371,15 @@ def test_option_structs_match_the_c_layout(tmp_path):
 def test_fp4_defaults_and_workspace(L):
     o = attn.fp4_options()
     assert o.rescale_threshold == 8.0 and o.classifier == attn.ATTN_DIRECT_P_AFFINE
-    assert o.wait_timeout_us == 0 and list(o.reserved) == [0] * 5
-    # Q, K, V widened to f16, each rounded up to 256 bytes
+    assert o.wait_timeout_us == 0 and list(o.reserved) == [0] * 4
+    assert o.mma == attn.ATTN_FP4_MMA_AUTO
+    # Room for either path: Q, K, V widened to f16 (each rounded up to 256
+    # bytes), or the block-scaled path's scale atoms (two 512-byte atoms per
+    # 128-row tile of Q -- both tiles of every 256-row query block -- K and V)
+    # and V's transposed codes (128 rows of 64 bytes per key tile).
     assert attn.fp4_workspace_size(2, 16, 16, 8192, 8192, 128) == 3 * 2 * 2 * 8192 * 16 * 128
     assert attn.fp4_workspace_size(1, 2, 1, 3, 5, 64) == 768 + 2 * 768  # 768 B, 640 B -> 768
+    assert attn.fp4_workspace_size(1, 1, 1, 1, 1, 128) == 2 * 1024 + 1024 + 1024 + 128 * 64
     assert attn.fp4_workspace_size(0, 2, 1, 3, 5, 64) == 0
 
 
@@ -408,6 +414,10 @@ def call_fp4(L, **kw):
     (dict(opts=attn.fp4_options(rescale_threshold=8.5)), attn.ATTN_ERR_INVALID_ARG),
     (dict(opts=attn.fp4_options(rescale_threshold=-1.0)), attn.ATTN_ERR_INVALID_ARG),
     (dict(opts=attn.fp4_options(wait_timeout_us=-5)), attn.ATTN_ERR_INVALID_ARG),
+    (dict(opts=attn.fp4_options(mma=3)), attn.ATTN_ERR_INVALID_ARG),
+    (dict(opts=attn.fp4_options(mma=-1)), attn.ATTN_ERR_INVALID_ARG),
+    (dict(D=64, opts=attn.fp4_options(mma=attn.ATTN_FP4_MMA_BLOCK_SCALED)),
+     attn.ATTN_ERR_UNSUPPORTED),
 ])
 def test_fp4_invalid_arguments_rejected_before_launch(L, kw, status):
     assert call_fp4(L, **kw) == status
@@ -415,14 +425,16 @@ def test_fp4_invalid_arguments_rejected_before_launch(L, kw, status):
 
 def test_fp4_reserved_options_must_be_zero(L):
     o = attn.fp4_options()
-    o.reserved[4] = 1
+    o.reserved[3] = 1
     assert call_fp4(L, opts=o) == attn.ATTN_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path only")
 def test_valid_fp4_call_without_gpu_reports_cuda_error(L):
     for classifier in (0, 1):
-        assert call_fp4(L, opts=attn.fp4_options(classifier=classifier)) == attn.ATTN_ERR_CUDA
+        for mma in (attn.ATTN_FP4_MMA_AUTO, attn.ATTN_FP4_MMA_F16, attn.ATTN_FP4_MMA_BLOCK_SCALED):
+            assert call_fp4(L, opts=attn.fp4_options(classifier=classifier, mma=mma)) == \
+                attn.ATTN_ERR_CUDA
 
 
 def test_fp4_binding_checks_shapes(L):

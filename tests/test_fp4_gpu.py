@@ -38,8 +38,18 @@ def _vmax(t):
     return [0, 0.5, 1, 1.5, 2, 3, 4, 6][mag] * 2.0 ** (int(t["v_scales"].numpy().max()) - 127)
 
 
-def _run(t, classifier, **kw):
-    o, lse = attn.attention_fp4(*_dev(t), classifier=classifier, **kw)
+# The two tensor-core paths of the D = 128 forward: block-scaled FP4 products
+# (the default there) and f16 products of the widened values.  D = 64 has the
+# f16 path only.
+MMAS = ("block_scaled", "f16")
+
+
+def _mma_ok(mma, D):
+    return mma != "block_scaled" or D == 128
+
+
+def _run(t, classifier, mma="auto", **kw):
+    o, lse = attn.attention_fp4(*_dev(t), classifier=classifier, mma=mma, **kw)
     attn.check_device_status()
     return o.float().cpu().numpy(), lse.cpu().numpy()
 
@@ -75,40 +85,64 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("mma", MMAS)
 @pytest.mark.parametrize("classifier", ["affine", "exp2"])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[:6]}-{sorted(c[6].items())}")
-def test_fp4_parity_exact_decisions(case, classifier):
+def test_fp4_parity_exact_decisions(case, classifier, mma):
     B, Hq, Hkv, Sq, Sk, D, mask = case
+    if not _mma_ok(mma, D):
+        pytest.skip("block-scaled products are built for D = 128")
     scale = 1.0 / math.sqrt(D)
     t = make_tensors_fp4(B, Hq, Hkv, Sq, Sk, D, seed=11 + Sq + D, scale=scale)
-    o, lse = _run(t, classifier, scale=scale, **mask)
+    o, lse = _run(t, classifier, mma=mma, scale=scale, **mask)
     o_ref, lse_ref = _ref(t, classifier, scale=scale, **mask)
     _tight(o, lse, o_ref, lse_ref, _vmax(t))
 
 
+@pytest.mark.parametrize("mma", MMAS)
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("classifier", ["affine", "exp2"])
-def test_fp4_parity_document_mask(classifier):
-    S, D = 700, 64
+def test_fp4_parity_document_mask(classifier, D, mma):
+    if not _mma_ok(mma, D):
+        pytest.skip("block-scaled products are built for D = 128")
+    S = 700
     scale = 1.0 / math.sqrt(D)
     t = make_tensors_fp4(1, 4, 2, S, S, D, seed=21, scale=scale)
     docs = np.array([0, 100, 450, 451, 700], dtype=np.int32)
-    o, lse = _run(t, classifier, scale=scale, causal=True,
+    o, lse = _run(t, classifier, mma=mma, scale=scale, causal=True,
                   doc_offsets=torch.from_numpy(docs).cuda())
     o_ref, lse_ref = _ref(t, classifier, scale=scale, causal=True, doc_offsets=docs)
     _tight(o, lse, o_ref, lse_ref, _vmax(t))
 
 
+@pytest.mark.parametrize("mma", MMAS)
 @pytest.mark.parametrize("tau", [0.0, 3.0, 8.0])
-def test_fp4_rescale_threshold_does_not_change_the_result(tau):
+def test_fp4_rescale_threshold_does_not_change_the_result(tau, mma):
     # The anchor is an integer and every rescale an exact power of two: the
     # result for any threshold matches the oracle, which has no anchor.
     S, D = 520, 128
     scale = 1.0 / math.sqrt(D)
     t = make_tensors_fp4(1, 2, 2, S, S, D, seed=31, scale=scale)
-    o, lse = _run(t, "affine", scale=scale, causal=True,
+    o, lse = _run(t, "affine", mma=mma, scale=scale, causal=True,
                   options=attn.fp4_options(rescale_threshold=tau))
     o_ref, lse_ref = _ref(t, "affine", scale=scale, causal=True)
     _tight(o, lse, o_ref, lse_ref, _vmax(t))
+
+
+@pytest.mark.parametrize("classifier", ["affine", "exp2"])
+def test_fp4_block_scaled_matches_f16_products(classifier):
+    # Every product of two FP4 values is exact in fp32, so the two paths
+    # differ only in the order of the fp32 accumulation: O within one bf16
+    # rounding step of each other (plus accumulation noise), LSE to fp32
+    # rounding.
+    S, D = 900, 128
+    scale = 1.0 / math.sqrt(D)
+    t = make_tensors_fp4(2, 4, 2, S, S, D, seed=33, scale=scale, pow2_scales=False)
+    o_bs, l_bs = _run(t, classifier, mma="block_scaled", scale=scale, causal=True)
+    o_f, l_f = _run(t, classifier, mma="f16", scale=scale, causal=True)
+    err = np.abs(o_bs - o_f)
+    assert (err <= 2.0 ** -7 * np.abs(o_f) + 1e-6).all(), float(err.max())
+    assert np.abs(l_bs - l_f).max() <= 1e-5 + 1e-6 * np.abs(l_f).max()
 
 
 def drop_bounds(t, rows, scale, tau, classifier):
@@ -149,9 +183,10 @@ def drop_bounds(t, rows, scale, tau, classifier):
     return frac, vrow
 
 
+@pytest.mark.parametrize("mma", MMAS)
 @pytest.mark.parametrize("classifier", ["affine", "exp2"])
 @pytest.mark.parametrize("tau", [0.0, 8.0])
-def test_fp4_wide_logits(classifier, tau):
+def test_fp4_wide_logits(classifier, tau, mma):
     # Score factor 2^3 instead of ~2^-3: log2 scores spread over hundreds of
     # units, so the anchor moves by large steps and many blocks sit far below
     # it (the range guard).  Element-wise parity with a per-row bound for
@@ -159,7 +194,7 @@ def test_fp4_wide_logits(classifier, tau):
     # at 0.
     S, D = 400, 128
     t = make_tensors_fp4(1, 2, 2, S, S, D, seed=41, scale=8.0)
-    o, lse = _run(t, classifier, scale=8.0, causal=True,
+    o, lse = _run(t, classifier, mma=mma, scale=8.0, causal=True,
                   options=attn.fp4_options(rescale_threshold=tau))
     o_ref, lse_ref = _ref(t, classifier, scale=8.0, causal=True)
     assert np.abs(lse_ref).max() > 100
@@ -177,61 +212,78 @@ def test_fp4_wide_logits(classifier, tau):
     assert (np.abs(l_got - l_want) <= l_bound).all(), float(np.abs(l_got - l_want).max())
 
 
+@pytest.mark.parametrize("mma", MMAS)
 @pytest.mark.parametrize("classifier", ["affine", "exp2"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_fp4_general_nvfp4_scales(classifier, D):
+def test_fp4_general_nvfp4_scales(classifier, D, mma):
+    if not _mma_ok(mma, D):
+        pytest.skip("block-scaled products are built for D = 128")
     S = 300
     scale = 1.0 / math.sqrt(D)
     t = make_tensors_fp4(1, 2, 2, S, S, D, seed=51, scale=scale, pow2_scales=False)
-    o, lse = _run(t, classifier, scale=scale, causal=True)
+    o, lse = _run(t, classifier, mma=mma, scale=scale, causal=True)
     o_ref, lse_ref = _ref(t, classifier, scale=scale, causal=True)
     err = np.abs(o - o_ref)
     assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
     assert np.abs(lse - lse_ref).max() <= 1e-3
 
 
-def test_fp4_full_size_sampled_rows():
-    # The benchmark's workload and launch (B2 H16 S8192 D128 causal), checked
-    # on sampled rows the oracle computes one by one.
+@pytest.mark.parametrize("mma", MMAS)
+def test_fp4_full_size_sampled_rows(mma):
+    # The benchmark's workload and launch (B2 H16 S8192 D128 causal; the
+    # benchmark runs the block-scaled path), checked on sampled rows the
+    # oracle computes one by one.
     w = WORKLOADS["causal_s8192_fp4"]
     t = make_inputs(w)
-    o, lse = _run(t, "affine", scale=w.scale, causal=True)
     rng = np.random.default_rng(5)
     rows = np.stack([rng.integers(0, w.B, 48), rng.integers(0, w.Hq, 48),
                      rng.integers(0, w.S, 48)], 1)
     rows = np.concatenate([rows, [[0, 0, 0], [1, 15, w.S - 1], [0, 3, 127], [1, 8, 128]]])
     for classifier in ("affine", "exp2"):
-        if classifier == "exp2":
-            o, lse = _run(t, classifier, scale=w.scale, causal=True)
+        o, lse = _run(t, classifier, mma=mma, scale=w.scale, causal=True)
         o_ref, lse_ref = _ref(t, classifier, scale=w.scale, causal=True, rows=rows)
         got = o[rows[:, 0], rows[:, 2], rows[:, 1]]
         got_lse = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
         _tight(got, got_lse, o_ref, lse_ref, _vmax(t))
 
 
-def test_fp4_range_error_reported():
-    S, D = 64, 64
-    t = make_tensors_fp4(1, 1, 1, S, S, D, seed=61)
+@pytest.mark.parametrize("mma,D", [("f16", 64), ("f16", 128), ("block_scaled", 128)])
+def test_fp4_range_error_reported(mma, D):
+    S = 64
+    scale = 1.0 / math.sqrt(D)
+    t = make_tensors_fp4(1, 1, 1, S, S, D, seed=61, scale=scale)
     # an out-of-range V scale under nonzero codes: reported, read as zero
     t["v_scales"] = t["v_scales"].clone()
     t["v_scales"][0, 0, 0, 0] = 200
     t["v_codes"] = t["v_codes"].clone()
     t["v_codes"][0, 0, 0, 0] = 0x11
-    attn.attention_fp4(*_dev(t), causal=True)
+    o, _ = attn.attention_fp4(*_dev(t), causal=True, scale=scale, mma=mma)
     assert attn.device_status() == attn.ATTN_ERR_RANGE
     assert attn.device_status() == attn.ATTN_OK  # reading clears it
+    zeroed = dict(t, v_codes=t["v_codes"].clone())
+    zeroed["v_codes"][0, :32, 0, 0] &= 0xF0  # column d = 0 of keys 0-31 reads as zero
+    o_ref, _ = _ref(zeroed, "affine", scale=scale, causal=True)
+    assert np.abs(o.float().cpu().numpy() - o_ref).max() <= 2e-2
     # the same scale under zero codes is harmless
     t["v_codes"][:, :32, 0, 0] = 0
-    attn.attention_fp4(*_dev(t), causal=True)
+    attn.attention_fp4(*_dev(t), causal=True, scale=scale, mma=mma)
     assert attn.device_status() == attn.ATTN_OK
-    # a NaN NVFP4 scale under nonzero codes
-    t2 = make_tensors_fp4(1, 1, 1, S, S, D, seed=62)
-    t2["q_scales"] = t2["q_scales"].clone()
-    t2["q_scales"][0, 3, 0, 1] = 0x7F
-    t2["q_codes"] = t2["q_codes"].clone()
-    t2["q_codes"][0, 3, 0, 8] = 0x22
-    attn.attention_fp4(*_dev(t2), causal=True)
-    assert attn.device_status() == attn.ATTN_ERR_RANGE
+    # NaN and negative NVFP4 scales under nonzero codes: reported, and the
+    # output is the oracle's, which reads those blocks as zero; -0 is a zero
+    # scale and reports nothing
+    for bad in (0x7F, 0xB8):
+        t2 = make_tensors_fp4(1, 1, 1, S, S, D, seed=62, scale=scale)
+        t2["q_scales"] = t2["q_scales"].clone()
+        t2["q_scales"][0, 3, 0, 1] = bad
+        t2["q_codes"] = t2["q_codes"].clone()
+        t2["q_codes"][0, 3, 0, 8] = 0x22
+        o2, _ = attn.attention_fp4(*_dev(t2), causal=True, scale=scale, mma=mma)
+        assert attn.device_status() == attn.ATTN_ERR_RANGE
+        o2_ref, _ = _ref(t2, "affine", scale=scale, causal=True)
+        assert np.abs(o2.float().cpu().numpy() - o2_ref).max() <= 2e-2
+    t2["q_scales"][0, 3, 0, 1] = 0x80
+    attn.attention_fp4(*_dev(t2), causal=True, scale=scale, mma=mma)
+    assert attn.device_status() == attn.ATTN_OK
 
 
 def test_fp4_cosine_against_bf16_exact():

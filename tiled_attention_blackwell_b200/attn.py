@@ -29,6 +29,11 @@ ATTN_ERR_RANGE = 7
 ATTN_DIRECT_P_AFFINE = 0
 ATTN_DIRECT_P_EXP2 = 1
 CLASSIFIERS = {"affine": ATTN_DIRECT_P_AFFINE, "exp2": ATTN_DIRECT_P_EXP2}
+ATTN_FP4_MMA_AUTO = 0
+ATTN_FP4_MMA_F16 = 1
+ATTN_FP4_MMA_BLOCK_SCALED = 2
+FP4_MMA = {"auto": ATTN_FP4_MMA_AUTO, "f16": ATTN_FP4_MMA_F16,
+           "block_scaled": ATTN_FP4_MMA_BLOCK_SCALED}
 
 EXPORTED = ("attn_fwd", "attn_fwd_ex", "attn_fwd_fp8", "attn_fwd_default_options",
             "attn_fp4_default_options", "attn_fwd_fp4_workspace_size", "attn_fwd_fp4", "attn_bwd",
@@ -59,7 +64,8 @@ class BwdOptions(ctypes.Structure):
 class Fp4Options(ctypes.Structure):
     """Mirror of attn_fp4_options_t."""
     _fields_ = [("rescale_threshold", ctypes.c_float), ("classifier", ctypes.c_int),
-                ("wait_timeout_us", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
+                ("wait_timeout_us", ctypes.c_int), ("mma", ctypes.c_int),
+                ("reserved", ctypes.c_int * 4)]
 
 
 _FWD_ARGS = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [ctypes.c_float] + \
@@ -288,14 +294,16 @@ def fp4_workspace_size(B, Hq, Hkv, Sq, Sk, D) -> int:
 
 def attn_fwd_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_codes, v_scales,
                  v_global, o, lse, workspace, *, scale, causal=False, window=None,
-                 doc_offsets=None, classifier="affine", options=None, stream=None):
+                 doc_offsets=None, classifier="affine", mma=None, options=None, stream=None):
     """Enqueue the FP4 Direct-P forward.
 
     q_codes uint8 CUDA [B,Sq,Hq,D/2], q_scales uint8 [B,Sq,Hq,D/16] (e4m3
     bytes), likewise k_*; v_codes [B,Sk,Hkv,D/2], v_scales uint8
     [B,ceil(Sk/32),Hkv,D] (UE8M0 bytes); o bf16 [B,Sq,Hq,D]; lse fp32
     [B,Hq,Sq]; workspace uint8 CUDA of fp4_workspace_size() bytes.  All
-    contiguous.  classifier: "affine" or "exp2" (overrides `options`).
+    contiguous.  classifier: "affine" or "exp2" (overrides `options`); mma:
+    None (keep `options`), "auto", "f16" or "block_scaled" (which tensor-core
+    products run, see attn_fp4_options_t).
     """
     B, Sq, Hq, Dh = q_codes.shape
     _, Sk, Hkv, _ = k_codes.shape
@@ -321,6 +329,8 @@ def attn_fwd_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_cod
         docs_ptr, nd = None, 0
     options = fp4_options() if options is None else Fp4Options.from_buffer_copy(options)
     options.classifier = CLASSIFIERS[classifier]
+    if mma is not None:
+        options.mma = FP4_MMA[mma]
     st = lib().attn_fwd_fp4(_ptr(q_codes), _ptr(q_scales), float(q_global), _ptr(k_codes),
                             _ptr(k_scales), float(k_global), _ptr(v_codes), _ptr(v_scales),
                             float(v_global), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
@@ -332,7 +342,7 @@ def attn_fwd_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_cod
 
 def attention_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_codes, v_scales,
                   v_global, *, scale=None, causal=False, window=None, doc_offsets=None,
-                  classifier="affine", options=None, stream=None, workspace=None):
+                  classifier="affine", mma=None, options=None, stream=None, workspace=None):
     """Allocate O, LSE (and the workspace unless given) with torch and run the
     FP4 Direct-P forward.  Returns (O, LSE)."""
     B, Sq, Hq, Dh = q_codes.shape
@@ -352,7 +362,8 @@ def attention_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_co
         doc_offsets = doc_offsets.to(dev)
     attn_fwd_fp4(q_codes, q_scales, q_global, k_codes, k_scales, k_global, v_codes, v_scales,
                  v_global, o, lse, workspace, scale=scale, causal=causal, window=window,
-                 doc_offsets=doc_offsets, classifier=classifier, options=options, stream=stream)
+                 doc_offsets=doc_offsets, classifier=classifier, mma=mma, options=options,
+                 stream=stream)
     return o, lse
 
 

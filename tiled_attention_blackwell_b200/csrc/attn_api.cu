@@ -15,6 +15,7 @@
 #include "../../include/attn.h"
 #include "bwd_kernel.cuh"
 #include "fp4_dequant.cuh"
+#include "fwd_fp4_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "fwd_persistent.cuh"
 
@@ -132,6 +133,27 @@ attn_status_t make_map_tile(CUtensorMap *map, const void *base, int B, int S, in
     return ATTN_OK;
 }
 
+// 4-D map of packed FP4 codes, 64 bytes (128 codes) per row: dims (64,
+// rows, H, B) with the given row / head / batch strides in bytes; box one
+// 128-row tile, 64-byte swizzle (the layout of the block-scaled MMA
+// operands), zero fill out of bounds.
+attn_status_t make_map_fp4(CUtensorMap *map, const void *base, long long inner, int rows, int H,
+                           int B, long long row_stride, long long head_stride,
+                           long long batch_stride) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)row_stride, (cuuint64_t)head_stride,
+                                   (cuuint64_t)batch_stride};
+    const cuuint32_t box[4] = {64, (cuuint32_t)tab::kBlockM, 1, 1};
+    const cuuint32_t estride[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides,
+                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled (fp4) failed (%d)", (int)r);
+    return ATTN_OK;
+}
+
 // --------------------------------------------------------------- launching
 
 // PERSIST selects the persistent kernel (fwd_persistent.cuh: one CTA per SM
@@ -234,9 +256,61 @@ attn_status_t dispatch_direct_p(const tab::FwdParams &p, int grid, int D, int cl
                       : launch_fwd<64, kStagesD64, 0, 0, 2>(p, grid, s);
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// The block-scaled FP4 Direct-P kernel (fwd_fp4_kernel.cuh), D = 128.
+constexpr int kStagesFp4 = 8;  // K or V^T slots of 9 KB
+template <int CLS>
+attn_status_t launch_fp4bs(const tab::FwdParams &p, int grid, cudaStream_t stream) {
+    using Smem = tab::FwdSmemFp4<kStagesFp4>;
+    constexpr size_t smem = sizeof(Smem) + 1024;
+    static_assert(smem <= 232448, "shared memory budget");
+    auto kernel = tab::attn_fwd_fp4bs_kernel<kStagesFp4, CLS>;
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t attr_err[kMaxDevices];
+    static cudaFuncAttributes attrs[kMaxDevices];
+    static cudaError_t attrs_err[kMaxDevices];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::call_once(once[dev], [&]() {
+        attr_err[dev] = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        attrs_err[dev] = cudaFuncGetAttributes(&attrs[dev], kernel);
+    });
+    if (attr_err[dev] != cudaSuccess)
+        return fail(ATTN_ERR_LAUNCH, "cudaFuncSetAttribute: %s", cudaGetErrorString(attr_err[dev]));
+    if (attrs_err[dev] != cudaSuccess)
+        return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes: %s", cudaGetErrorString(attrs_err[dev]));
+    // setmaxnreg split: see launch_fwd.
+    if (attrs[dev].numRegs < tab::kLaunchRegs)
+        return fail(ATTN_ERR_LAUNCH, "kernel compiled with %d registers per thread, %d needed",
+                    attrs[dev].numRegs, tab::kLaunchRegs);
+    kernel<<<grid, tab::kFwdThreads, smem, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ATTN_ERR_LAUNCH, "launch: %s", cudaGetErrorString(e));
+    return ok();
+}
 
 size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// Workspace of the block-scaled path: scale atoms of Q (tiles of both of a
+// CTA's query blocks), K and V, then V^T's codes.
+struct Fp4BsLayout {
+    int nqt, nkt;
+    size_t sf_q, sf_k, sf_v, vt, total;
+};
+Fp4BsLayout fp4bs_layout(int B, int Hq, int Hkv, int Sq, int Sk) {
+    Fp4BsLayout L;
+    L.nqt = 2 * ((Sq + 2 * tab::kBlockM - 1) / (2 * tab::kBlockM));
+    L.nkt = (Sk + tab::kBlockN - 1) / tab::kBlockN;
+    const size_t atoms = 2 * tab::kSfAtom;
+    L.sf_q = 0;
+    L.sf_k = L.sf_q + align256((size_t)B * Hq * L.nqt * atoms);
+    L.sf_v = L.sf_k + align256((size_t)B * Hkv * L.nkt * atoms);
+    L.vt = L.sf_v + align256((size_t)B * Hkv * L.nkt * atoms);
+    L.total = L.vt + align256((size_t)B * Hkv * 128 * L.nkt * 64);
+    return L;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape and mask checks shared by the forward and the backward.
 attn_status_t check_common(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
@@ -532,12 +606,15 @@ void attn_fp4_default_options(attn_fp4_options_t *opts) {
     *opts = attn_fp4_options_t{};
     opts->rescale_threshold = 8.0f;
     opts->classifier = ATTN_DIRECT_P_AFFINE;
+    opts->mma = ATTN_FP4_MMA_AUTO;
 }
 
 size_t attn_fwd_fp4_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Sk < 1 || D < 1) return 0;
     const size_t nq = (size_t)B * Sq * Hq * D, nkv = (size_t)B * Sk * Hkv * D;
-    return align256(nq * 2) + 2 * align256(nkv * 2);
+    const size_t widened = align256(nq * 2) + 2 * align256(nkv * 2);
+    // Room for either path (the options pick one per call).
+    return D == 128 ? std::max(widened, fp4bs_layout(B, Hq, Hkv, Sq, Sk).total) : widened;
 }
 
 attn_status_t attn_fwd_fp4(const void *q_codes, const void *q_scales, float q_global,
@@ -574,8 +651,14 @@ attn_status_t attn_fwd_fp4(const void *q_codes, const void *q_scales, float q_gl
         return fail(ATTN_ERR_INVALID_ARG, "classifier must be ATTN_DIRECT_P_AFFINE or ATTN_DIRECT_P_EXP2");
     if (op.wait_timeout_us < 0 || op.wait_timeout_us > 60000000)
         return fail(ATTN_ERR_INVALID_ARG, "wait_timeout_us must lie in [0, 60000000]");
+    if (op.mma < ATTN_FP4_MMA_AUTO || op.mma > ATTN_FP4_MMA_BLOCK_SCALED)
+        return fail(ATTN_ERR_INVALID_ARG, "mma must be ATTN_FP4_MMA_AUTO, _F16 or _BLOCK_SCALED");
+    if (op.mma == ATTN_FP4_MMA_BLOCK_SCALED && D != 128)
+        return fail(ATTN_ERR_UNSUPPORTED, "the block-scaled FP4 products are built for D = 128");
     for (int r : op.reserved)
         if (r != 0) return fail(ATTN_ERR_INVALID_ARG, "reserved option fields must be zero");
+    const bool block_scaled = op.mma == ATTN_FP4_MMA_BLOCK_SCALED ||
+                              (op.mma == ATTN_FP4_MMA_AUTO && D == 128);
     const size_t need = attn_fwd_fp4_workspace_size(B, Hq, Hkv, Sq, Sk, D);
     if (workspace_bytes < need)
         return fail(ATTN_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
@@ -589,12 +672,33 @@ attn_status_t attn_fwd_fp4(const void *q_codes, const void *q_scales, float q_gl
     const size_t nq = (size_t)B * Sq * Hq * D, nkv = (size_t)B * Sk * Hkv * D;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     void *q16 = ws, *k16 = ws + align256(nq * 2), *v16 = ws + align256(nq * 2) + align256(nkv * 2);
+    const Fp4BsLayout L = fp4bs_layout(B, Hq, Hkv, Sq, Sk);
 
     tab::FwdParams p;
     memset(&p, 0, sizeof p);
-    if ((s = make_map(&p.tm_q, q16, B, Sq, Hq, D)) != ATTN_OK) return s;
-    if ((s = make_map(&p.tm_k, k16, B, Sk, Hkv, D)) != ATTN_OK) return s;
-    if ((s = make_map(&p.tm_v, v16, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    if (block_scaled) {
+        // Q and K codes straight from the caller (64 bytes per row); V^T codes
+        // and all scale atoms from the preparation pass.
+        if ((s = make_map_fp4(&p.tm_q, q_codes, 64, Sq, Hq, B, (long long)Hq * 64, 64,
+                              (long long)Sq * Hq * 64)) != ATTN_OK)
+            return s;
+        if ((s = make_map_fp4(&p.tm_k, k_codes, 64, Sk, Hkv, B, (long long)Hkv * 64, 64,
+                              (long long)Sk * Hkv * 64)) != ATTN_OK)
+            return s;
+        const long long vt_row = (long long)L.nkt * 64;
+        if ((s = make_map_fp4(&p.tm_v, ws + L.vt, vt_row, 128, Hkv, B, vt_row, 128 * vt_row,
+                              (long long)Hkv * 128 * vt_row)) != ATTN_OK)
+            return s;
+        p.sf_q = ws + L.sf_q;
+        p.sf_k = ws + L.sf_k;
+        p.sf_v = ws + L.sf_v;
+        p.nq_tiles = L.nqt;
+        p.nk_tiles = L.nkt;
+    } else {
+        if ((s = make_map(&p.tm_q, q16, B, Sq, Hq, D)) != ATTN_OK) return s;
+        if ((s = make_map(&p.tm_k, k16, B, Sk, Hkv, D)) != ATTN_OK) return s;
+        if ((s = make_map(&p.tm_v, v16, B, Sk, Hkv, D)) != ATTN_OK) return s;
+    }
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.lse = lse;
     p.doc_offsets = doc_offsets;
@@ -629,6 +733,37 @@ attn_status_t attn_fwd_fp4(const void *q_codes, const void *q_scales, float q_gl
 #endif
 
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (block_scaled) {
+        tab::Fp4PrepParams pp;
+        memset(&pp, 0, sizeof pp);
+        pp.q_codes = static_cast<const uint8_t *>(q_codes);
+        pp.q_scales = static_cast<const uint8_t *>(q_scales);
+        pp.k_codes = static_cast<const uint8_t *>(k_codes);
+        pp.k_scales = static_cast<const uint8_t *>(k_scales);
+        pp.v_codes = static_cast<const uint8_t *>(v_codes);
+        pp.v_scales = static_cast<const uint8_t *>(v_scales);
+        pp.sf_q = ws + L.sf_q;
+        pp.sf_k = ws + L.sf_k;
+        pp.sf_v = ws + L.sf_v;
+        pp.vt = ws + L.vt;
+        pp.B = B;
+        pp.Hq = Hq;
+        pp.Hkv = Hkv;
+        pp.Sq = Sq;
+        pp.Sk = Sk;
+        pp.nqt = L.nqt;
+        pp.nkt = L.nkt;
+        pp.status = st->status;
+        const long long v_ctas = (long long)B * Hkv * L.nkt;
+        const long long rows = ((long long)B * Hq * L.nqt + (long long)B * Hkv * L.nkt) * 128;
+        const long long sf_ctas = std::min<long long>((rows + 255) / 256, (long long)st->num_sms * 8);
+        if (v_ctas + sf_ctas > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+        pp.v_ctas = (int)v_ctas;
+        tab::fp4_prepare_kernel<<<(unsigned)(v_ctas + sf_ctas), 256, 0, cs>>>(pp);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return fail(ATTN_ERR_LAUNCH, "launch: %s", cudaGetErrorString(e));
+        return op.classifier ? launch_fp4bs<1>(p, (int)grid, cs) : launch_fp4bs<0>(p, (int)grid, cs);
+    }
     tab::Fp4DequantParams dp;
     memset(&dp, 0, sizeof dp);
     dp.job[0] = {static_cast<const uint8_t *>(q_codes), static_cast<const uint8_t *>(q_scales),

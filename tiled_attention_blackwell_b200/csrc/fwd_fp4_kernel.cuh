@@ -1,0 +1,570 @@
+// Direct-P forward on the block-scaled FP4 tensor cores (sm_100a), D = 128.
+//
+// "Hardware-Aware FP4 FlashAttention-4", "Metodología", item 1: Q K^T as an
+// NVFP4 product (E2M1 codes, one e4m3 scale per 16 elements), then the
+// probabilities built directly as MXFP4 values -- E2M1 codes with one
+// power-of-two scale per 32 keys, chosen by the affine classifier or the
+// rounded exponential -- and P V as an MXFP4 product, the softmax
+// normaliser being the sum of exactly those values.  The codes, block
+// exponents and sums are those of the f16-operand Direct-P kernel
+// (direct_p_half in fwd_kernel.cuh): only where the products run differs.
+//
+// CTA shape and roles as in attn_fwd_kernel: two 128-row query tiles of one
+// (batch, query head), warps 0-3 / 4-7 softmax + correction + epilogue of
+// tile 0 / 1, warp 8 MMA issue, warp 9 TMA producer.
+//
+// Tensor memory is where this kernel differs ("Contribuciones Clave":
+// tensor-memory ownership bounds the overlap).  Block-scaled products read
+// their scale factors from tensor memory and take P from shared memory, and
+// the 512 columns cannot hold two S tiles, two O tiles and the scales, so
+// the two query tiles share one S region: Q_i K^T of the other tile is
+// issued once this tile's softmax has loaded its scores.  At FP4 rates the
+// products are short against the softmax, which is what bounds the loop.
+//   [  0,128) S (tile 0 and tile 1 in turn)
+//   [128,256) O0, [256,384) O1
+//   [384,400) Q scales  (tile i, K step ks: 384 + 4 (2i + ks))
+//   [400,416) K scales  (block parity, K step)
+//   [416,432) V scales  (block parity, K step)
+//   [432,448) P scales  (tile, K step)
+//
+// Shared memory: Q0, Q1 and a ring of NS slots (K codes or V^T codes, each
+// 128 rows x 64 bytes with the 64-byte swizzle, followed by their two
+// scale atoms), P0 and P1 as codes in the same layout, and the P scale
+// atoms the softmax warps write.
+//
+// Ordering (all products of one thread execute in issue order): per block
+// j and tile i the MMA warp issues P_i V(j) and then Q_i K^T(j+1), so the
+// arrival of S(i, j+1) proves that P_i V(j) has completed -- the softmax may
+// then rescale O_i and overwrite P_i and its scales.  Scale columns of K
+// and V alternate by block parity; every reuse is two blocks apart, after a
+// commit the MMA warp has already waited on.
+#pragma once
+
+#include "fp4_prepare.cuh"
+#include "fwd_kernel.cuh"
+
+namespace tab {
+
+constexpr int kFp4Tile = kBlockM * 64;               // 8 KB of codes
+constexpr int kFp4Slot = kFp4Tile + 2 * kSfAtom;     // codes + two scale atoms
+constexpr uint32_t kColS = 0, kColO = 128, kColSfQ = 384, kColSfK = 400, kColSfV = 416,
+                   kColSfP = 432;
+
+template <int NS>
+struct FwdSmemFp4 {
+    alignas(1024) uint8_t q[2][kFp4Tile];
+    uint8_t qsf[2][2][kSfAtom];  // [tile][K step]
+    alignas(1024) uint8_t kv[NS][kFp4Slot];
+    alignas(1024) uint8_t p[2][kFp4Tile];
+    uint8_t psf[2][2][kSfAtom];
+    uint64_t q_full;
+    uint64_t kv_full[NS];
+    uint64_t kv_empty[NS];
+    uint64_t s_full[2];
+    uint64_t s_free;     // the scores in the shared S region have been loaded
+    uint64_t p_half[2];  // codes and scales of keys [0, 64) are in shared memory
+    uint64_t p_full[2];  // all of P (and any O correction)
+    uint64_t o_final[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int range[2][2];
+};
+
+// Codes of 64 scores of a row (two 32-key blocks with maxima bm[0], bm[1]):
+// per block the exponent E, the 16 bytes of E2M1 codes (key 2k in the low
+// nibble of byte k) and the UE8M0 byte E + 127; returns the fp32 sum of the
+// represented values code * 2^E.  Same steps and constants as direct_p_half.
+template <int CLS>
+__device__ __forceinline__ float direct_p_codes(const float *s, const float *bm, float c,
+                                                float base, uint4 *codes, uint32_t &sf2) {
+    float sum = 0.0f;
+    sf2 = 0u;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const float ymax = fmaf(bm[u], c, base);
+        const float ef = floorf(ymax) - 2.0f;
+        const bool keep = ef >= -13.0f;  // false for an all-masked block (-inf)
+        const int ei = keep ? (int)fminf(ef, 13.0f) : 0;
+        const float nb = keep ? base - (float)ei : -INFINITY;  // r = s*c + nb
+        sf2 |= (uint32_t)(ei + 127) << (8 * u);
+        const float c2 = 2.0f * c, nb2 = 2.0f * nb + (2.0f + kRintMagic);
+        uint32_t cs0 = 0u, cs1 = 0u;
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t word = 0u;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const float s0 = s[32 * u + 8 * q + e], s1 = s[32 * u + 8 * q + e + 1];
+                uint32_t byte;
+                if constexpr (CLS == 0) {
+                    float t0, t1;
+                    fma2(t0, t1, s0, s1, c2, c2, nb2, nb2);
+                    t0 = fminf(fmaxf(t0, kRintMagic), kRintMagic + 7.0f);
+                    t1 = fminf(fmaxf(t1, kRintMagic), kRintMagic + 7.0f);
+                    byte = (__float_as_uint(t0) & 7u) | ((__float_as_uint(t1) & 7u) << 4);
+                } else {
+                    float r0, r1;
+                    fma2(r0, r1, s0, s1, c, c, nb, nb);
+                    byte = e2m1x2_round(ex2_mufu(r0), ex2_mufu(r1));
+                }
+                word |= byte << (4 * e);
+                const uint32_t h = e2m1x2_to_f16x2(byte);
+                if ((e & 2) == 0) cs0 = hadd2_u32(cs0, h);
+                else cs1 = hadd2_u32(cs1, h);
+            }
+            w[q] = word;
+        }
+        codes[u] = make_uint4(w[0], w[1], w[2], w[3]);
+        if (keep) sum += f16x2_sum(hadd2_u32(cs0, cs1)) * __uint_as_float((uint32_t)(ei + 127) << 23);
+    }
+    return sum;
+}
+
+template <int NS, int CLS>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
+    using Smem = FwdSmemFp4<NS>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_off = smem_u32(smem_raw);
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (raw_off & 1023u)) & 1023u));
+
+    const int warp = warp_id();
+    const int lane = lane_id();
+
+    // Work item: the order of attn_fwd_kernel (head groups, heaviest query
+    // blocks first).
+    const int bh_count = p.Hq * p.B;
+    const int G = p.head_group;
+    const int nq = p.num_qblocks;
+    const int full_groups = bh_count / G;
+    const int lin = (int)blockIdx.x;
+    int grp, r, ge;
+    if (lin < full_groups * G * nq) {
+        grp = lin / (G * nq);
+        r = lin % (G * nq);
+        ge = G;
+    } else {
+        grp = full_groups;
+        r = lin - full_groups * G * nq;
+        ge = bh_count - full_groups * G;
+    }
+    const int qb = nq - 1 - r / ge;
+    const int bh = grp * G + r % ge;
+    const int hq = bh % p.Hq;
+    const int b = bh / p.Hq;
+    const int hkv = hq / p.group;
+    const int q0 = qb * 2 * kBlockM;
+
+    // ------------------------------------------------------------ prologue
+    if (threadIdx.x == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.s_full[i], 1);
+            mbar_init(&sm.p_half[i], kBlockM);
+            mbar_init(&sm.p_full[i], kBlockM);
+            mbar_init(&sm.o_final[i], 1);
+        }
+        mbar_init(&sm.s_free, kBlockM);
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        for (int i = 0; i < 2; ++i) {
+            const int r0 = q0 + i * kBlockM;
+            KeyRange kr{1, 0};
+            if (r0 < p.Sq) kr = tile_key_range(p, r0, min(r0 + kBlockM - 1, p.Sq - 1), lane);
+            if (lane == 0) {
+                if (kr.lo > kr.hi) {
+                    sm.range[i][0] = 1;
+                    sm.range[i][1] = 0;
+                } else {
+                    sm.range[i][0] = kr.lo / kBlockN;
+                    sm.range[i][1] = kr.hi / kBlockN;
+                }
+            }
+        }
+    }
+    if (warp == 8) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem = sm.tmem_base;
+    volatile int *abort_flag = &sm.abort_flag;
+    const int lo0 = sm.range[0][0], hi0 = sm.range[0][1];
+    const int lo1 = sm.range[1][0], hi1 = sm.range[1][1];
+    const bool has0 = lo0 <= hi0, has1 = lo1 <= hi1;
+    const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : lo1;
+    const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : hi1;
+    const int n_blocks = (has0 || has1) ? (uhi - ulo + 1) : 0;
+
+    if (warp >= 8) {
+        setmaxnreg_dec<kOtherRegs>();
+        if (warp == 9) {
+            // ------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                prefetch_tensormap(&p.tm_q);
+                prefetch_tensormap(&p.tm_k);
+                prefetch_tensormap(&p.tm_v);
+                mbar_arrive_expect_tx(&sm.q_full, 2 * kFp4Tile + 4 * kSfAtom);
+                for (int i = 0; i < 2; ++i)
+                    tma_load_4d(sm.q[i], &p.tm_q, &sm.q_full, 0, q0 + i * kBlockM, hq, b);
+                // Both tiles' scale atoms (tiles 2 qb and 2 qb + 1) are adjacent.
+                bulk_load(sm.qsf, p.sf_q + (((size_t)b * p.Hq + hq) * p.nq_tiles + 2 * qb) * (2 * kSfAtom),
+                          4 * kSfAtom, &sm.q_full);
+                uint32_t it = 0;
+                bool ok = true;
+                for (int t = 0; t < n_blocks && ok; ++t) {
+                    const int j = ulo + t;
+                    for (int which = 0; which < 2 && ok; ++which, ++it) {
+                        const uint32_t slot = it % NS;
+                        ok = wait_bounded(&sm.kv_empty[slot], ((it / NS) & 1u) ^ 1u, abort_flag,
+                                          p.status, true, p.timeout_ns);
+                        if (!ok) break;
+                        // Testing only: the first CTA withholds its first K copy.
+                        if (p.debug_withhold_kv && blockIdx.x == 0 && it == 0) continue;
+                        mbar_arrive_expect_tx(&sm.kv_full[slot], kFp4Slot);
+                        const size_t atoms = (((size_t)b * p.Hkv + hkv) * p.nk_tiles + j) * (2 * kSfAtom);
+                        if (which == 0) {
+                            tma_load_4d(sm.kv[slot], &p.tm_k, &sm.kv_full[slot], 0, j * kBlockN, hkv, b);
+                            bulk_load(sm.kv[slot] + kFp4Tile, p.sf_k + atoms, 2 * kSfAtom, &sm.kv_full[slot]);
+                        } else {
+                            tma_load_4d(sm.kv[slot], &p.tm_v, &sm.kv_full[slot], j * 64, 0, hkv, b);
+                            bulk_load(sm.kv[slot] + kFp4Tile, p.sf_v + atoms, 2 * kSfAtom, &sm.kv_full[slot]);
+                        }
+                    }
+                }
+                wait_bounded(&sm.q_full, 0, abort_flag, p.status, false, p.timeout_ns);
+                const uint32_t first = it > NS ? it - NS : 0;
+                for (uint32_t L = first; L < it; ++L)
+                    wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status, false, p.timeout_ns);
+            }
+            __syncwarp();
+        } else if (warp == 8) {
+            // --------------------------------------------------- MMA issuer
+            if (n_blocks > 0) {
+                const bool leader = elect_one();
+                constexpr uint32_t kIdescQK = idesc_fp4_bs(kBlockM, kBlockN, 0);  // UE4M3 scales
+                constexpr uint32_t kIdescPV = idesc_fp4_bs(kBlockM, 128, 1);      // UE8M0 scales
+                const uint64_t q_desc = smem_desc_sw64(smem_u32(sm.q[0]));
+                const uint64_t kv_desc = smem_desc_sw64(smem_u32(sm.kv[0]));
+                const uint64_t p_desc = smem_desc_sw64(smem_u32(sm.p[0]));
+                bool ok = __all_sync(0xffffffffu,
+                                     wait_bounded(&sm.q_full, 0, abort_flag, p.status, true, p.timeout_ns));
+                tc_fence_after();
+                if (ok && leader) {
+                    for (int i = 0; i < 2; ++i)
+                        for (int ks = 0; ks < 2; ++ks)
+                            tc_cp_sf(tmem + kColSfQ + 4 * (2 * i + ks),
+                                     smem_desc_sf_atom(smem_u32(sm.qsf[i][ks])));
+                }
+                __syncwarp();
+                auto ring_pos = [&](int j, int which) -> uint32_t {
+                    return 2u * (uint32_t)(j - ulo) + (uint32_t)which;
+                };
+                int k_ready = ulo - 1;  // last key block whose K slot was waited on
+                uint32_t n_qk = 0;      // Q K^T products issued (the shared S region's turns)
+                auto wait_k = [&](int j) {
+                    const uint32_t L = ring_pos(j, 0);
+                    if (ok)
+                        ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u,
+                                                                  abort_flag, p.status, true, p.timeout_ns));
+                    tc_fence_after();
+                    if (ok && leader) {
+                        const uint8_t *atoms = sm.kv[L % NS] + kFp4Tile;
+                        for (int ks = 0; ks < 2; ++ks)
+                            tc_cp_sf(tmem + kColSfK + 4 * (2 * (j & 1) + ks),
+                                     smem_desc_sf_atom(smem_u32(atoms + ks * kSfAtom)));
+                    }
+                    __syncwarp();
+                    k_ready = j;
+                };
+                auto issue_s = [&](int i, int j) {
+                    if (k_ready < j) wait_k(j);
+                    if (!ok) return;
+                    if (n_qk > 0) {
+                        ok = __all_sync(0xffffffffu, wait_bounded(&sm.s_free, (n_qk - 1) & 1u, abort_flag,
+                                                                  p.status, true, p.timeout_ns));
+                        if (!ok) return;
+                        tc_fence_after();
+                    }
+                    const uint64_t a0 = q_desc + ((i * kFp4Tile) >> 4);
+                    const uint64_t b0 = kv_desc + (((ring_pos(j, 0) % NS) * kFp4Slot) >> 4);
+                    if (leader) {
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks)
+                            mma_nvf4(tmem + kColS, a0 + 2 * ks, b0 + 2 * ks, kIdescQK,
+                                     tmem + kColSfQ + 4 * (2 * i + ks),
+                                     tmem + kColSfK + 4 * (2 * (j & 1) + ks), ks > 0 ? 1u : 0u);
+                        tc_commit(&sm.s_full[i]);
+                    }
+                    __syncwarp();
+                    ++n_qk;
+                };
+                auto active = [&](int i, int j) -> bool {
+                    return i == 0 ? (has0 && j >= lo0 && j <= hi0)
+                                  : (has1 && j >= lo1 && j <= hi1);
+                };
+
+                for (int i = 0; i < 2; ++i)
+                    if (active(i, ulo)) issue_s(i, ulo);
+                if (ok && k_ready < ulo) wait_k(ulo);
+                if (ok && leader) tc_commit(&sm.kv_empty[ring_pos(ulo, 0) % NS]);
+                __syncwarp();
+
+                for (int j = ulo; j <= uhi && ok; ++j) {
+                    const uint32_t Lv = ring_pos(j, 1);
+                    const uint32_t vslot = Lv % NS;
+                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[vslot], (Lv / NS) & 1u,
+                                                              abort_flag, p.status, true, p.timeout_ns));
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (leader)
+                        for (int ks = 0; ks < 2; ++ks)
+                            tc_cp_sf(tmem + kColSfV + 4 * (2 * (j & 1) + ks),
+                                     smem_desc_sf_atom(smem_u32(sm.kv[vslot] + kFp4Tile + ks * kSfAtom)));
+                    __syncwarp();
+                    const uint64_t vb = kv_desc + ((vslot * kFp4Slot) >> 4);
+                    for (int i = 0; i < 2 && ok; ++i) {
+                        if (active(i, j)) {
+                            const int lo_i = i == 0 ? lo0 : lo1;
+                            const int hi_i = i == 0 ? hi0 : hi1;
+                            const uint32_t par = (uint32_t)(j - lo_i) & 1u;
+                            const uint32_t o_tmem = tmem + kColO + i * 128;
+                            const uint64_t pa = p_desc + ((i * kFp4Tile) >> 4);
+                            // Keys [0, 64) as soon as their codes are in shared memory.
+                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_half[i], par, abort_flag,
+                                                                      p.status, true, p.timeout_ns));
+                            if (!ok) break;
+                            tc_fence_after();
+                            if (leader) {
+                                tc_cp_sf(tmem + kColSfP + 4 * (2 * i), smem_desc_sf_atom(smem_u32(sm.psf[i][0])));
+                                mma_mxf4(o_tmem, pa, vb, kIdescPV, tmem + kColSfP + 4 * (2 * i),
+                                         tmem + kColSfV + 4 * (2 * (j & 1)), j > lo_i ? 1u : 0u);
+                            }
+                            __syncwarp();
+                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_full[i], par, abort_flag,
+                                                                      p.status, true, p.timeout_ns));
+                            if (!ok) break;
+                            tc_fence_after();
+                            if (leader) {
+                                tc_cp_sf(tmem + kColSfP + 4 * (2 * i + 1),
+                                         smem_desc_sf_atom(smem_u32(sm.psf[i][1])));
+                                mma_mxf4(o_tmem, pa + 2, vb + 2, kIdescPV, tmem + kColSfP + 4 * (2 * i + 1),
+                                         tmem + kColSfV + 4 * (2 * (j & 1) + 1), 1u);
+                                if (j == hi_i) tc_commit(&sm.o_final[i]);
+                            }
+                            __syncwarp();
+                        }
+                        if (j + 1 <= uhi && active(i, j + 1)) issue_s(i, j + 1);
+                    }
+                    if (!ok) break;
+                    if (j + 1 <= uhi && k_ready < j + 1) wait_k(j + 1);
+                    if (!ok) break;
+                    if (leader) {
+                        tc_commit(&sm.kv_empty[vslot]);
+                        if (j + 1 <= uhi) tc_commit(&sm.kv_empty[ring_pos(j + 1, 0) % NS]);
+                    }
+                    __syncwarp();
+                }
+                if (!ok) {
+                    // Let every product and copy already issued finish before TMEM is freed.
+                    if (leader) tc_commit(&sm.drain);
+                    __syncwarp();
+                    wait_bounded(&sm.drain, 0, abort_flag, p.status, false, p.timeout_ns);
+                }
+            }
+            __syncwarp();
+        }
+        // warps 10-11: idle
+    } else {
+        // ------------------------------------- softmax / correction / epilogue
+        setmaxnreg_inc<kSoftmaxRegs>();
+        const int i = warp >> 2;
+        const int row_in_tile = threadIdx.x & (kBlockM - 1);
+        const int row = q0 + i * kBlockM + row_in_tile;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t s_tmem = tmem + lane_base + kColS;
+        const uint32_t o_tmem = tmem + lane_base + kColO + i * 128;
+        const KeyRange kr = row_key_range(p, row);
+        const int lo_b = i == 0 ? lo0 : lo1;
+        const int hi_b = i == 0 ? hi0 : hi1;
+        const float c = p.scale_log2;
+        const float tau = p.rescale_threshold;
+        // This row's 64 bytes of P codes: 16-byte chunk u (keys [32u, 32u + 32))
+        // at chunk u ^ ((row >> 1) & 3), the 64-byte swizzle; its scale word at
+        // 16 (row % 32) + 4 (row / 32) of the K step's atom.
+        uint8_t *p_row = sm.p[i] + row_in_tile * 64;
+        const int swz = (row_in_tile >> 1) & 3;
+        const int sf_off = 16 * (row_in_tile & 31) + 4 * (row_in_tile >> 5);
+#ifdef ATTN_COUNT_RESCALES
+        uint32_t cnt_blocks = 0, cnt_raise = 0, cnt_taken = 0, cnt_warp = 0;
+#endif
+        float m_run = -INFINITY;
+        float l_run = 0.0f;
+        bool ok = true;
+
+        for (int j = lo_b; j <= hi_b; ++j) {
+            const int t = j - lo_b;
+            ok = wait_bounded(&sm.s_full[i], (uint32_t)t & 1u, abort_flag, p.status, true, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+
+            uint32_t sr[kBlockN];
+            tmem_ld32(s_tmem + 0, sr + 0);
+            tmem_ld32(s_tmem + 32, sr + 32);
+            tmem_ld32(s_tmem + 64, sr + 64);
+            tmem_ld32(s_tmem + 96, sr + 96);
+            tmem_wait_ld();
+            reg_fence32(sr + 0);
+            reg_fence32(sr + 32);
+            reg_fence32(sr + 64);
+            reg_fence32(sr + 96);
+            // The S region is free for the other tile's next product.
+            tc_fence_before();
+            mbar_arrive(&sm.s_free);
+            float *s = reinterpret_cast<float *>(sr);
+
+            const int key0 = j * kBlockN;
+            const bool need_mask = key0 < kr.lo || key0 + kBlockN - 1 > kr.hi;
+            if (__any_sync(0xffffffffu, need_mask)) {
+#pragma unroll
+                for (int e = 0; e < kBlockN; ++e) {
+                    const int key = key0 + e;
+                    if (key < kr.lo || key > kr.hi) s[e] = -INFINITY;
+                }
+            }
+            float bm[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) bm[u] = block_max32(s + 32 * u);
+            const float m_cand = fmax3(fmaxf(bm[0], bm[1]), bm[2], bm[3]) * c;
+            float alpha = 1.0f;
+            ATTN_COUNT_BLOCK(t, m_cand > m_run, m_cand > m_run + tau);
+            if (m_cand > m_run + tau) {
+                const float m_new = ceilf(m_cand);
+                alpha = exp2_neg_int(m_run - m_new);
+                m_run = m_new;
+            }
+            const float neg_m = m_run == -INFINITY ? 0.0f : p.p_offset - m_run;
+            l_run *= alpha;
+
+            // Correction: P_i V(j-1) is complete (S of this block was committed
+            // after it), P_i V(j) is not yet issued.
+            if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#ifdef ATTN_COUNT_RESCALES
+                ++cnt_warp;
+#endif
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t rr[32];
+                    tmem_ld32(o_tmem + ch * 32, rr);
+                    tmem_wait_ld();
+                    reg_fence32(rr);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        float a0, a1;
+                        mul2(a0, a1, __uint_as_float(rr[e]), __uint_as_float(rr[e + 1]), alpha, alpha);
+                        rr[e] = __float_as_uint(a0);
+                        rr[e + 1] = __float_as_uint(a1);
+                    }
+                    tmem_st32(o_tmem + ch * 32, rr);
+                }
+                tmem_wait_st();
+            }
+
+            // Keys [0, 64), then [64, 128): codes and scale bytes to shared
+            // memory, made visible to the tensor cores, then signalled.
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint4 codes[2];
+                uint32_t sf2;
+                l_run += direct_p_codes<CLS>(s + 64 * half, bm + 2 * half, c, neg_m, codes, sf2);
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+                    *reinterpret_cast<uint4 *>(p_row + (((2 * half + u) ^ swz) << 4)) = codes[u];
+                *reinterpret_cast<uint32_t *>(sm.psf[i][half] + sf_off) = sf2;
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(half == 0 ? &sm.p_half[i] : &sm.p_full[i]);
+            }
+        }
+
+        // ----------------------------------------------------------- epilogue
+        const bool has_blocks = lo_b <= hi_b;
+        if (ok && has_blocks) {
+            ok = wait_bounded(&sm.o_final[i], 0, abort_flag, p.status, true, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+        }
+        if (ok) {
+            const bool row_ok = row < p.Sq;
+            const float inv_l = l_run > 0.0f ? p.v_descale / l_run : 0.0f;
+            __nv_bfloat16 *o_row = p.o + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)128;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t rr[32];
+                if (has_blocks) {
+                    tmem_ld32(o_tmem + ch * 32, rr);
+                    tmem_wait_ld();
+                    reg_fence32(rr);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) rr[e] = 0u;
+                }
+                uint4 out[4];
+                uint32_t *w = reinterpret_cast<uint32_t *>(out);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(rr[2 * e]) * inv_l,
+                                       __uint_as_float(rr[2 * e + 1]) * inv_l);
+                if (row_ok) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(o_row + ch * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = out[e];
+                }
+            }
+            if (row_ok) {
+                const float lse = l_run > 0.0f
+                                      ? (m_run - p.p_offset + log2f(l_run)) * 0.69314718055994531f
+                                      : -INFINITY;
+                p.lse[((size_t)b * p.Hq + hq) * p.Sq + row] = lse;
+            }
+        }
+#ifdef ATTN_COUNT_RESCALES
+        if (p.rescale_counts) {
+            for (int o = 16; o > 0; o >>= 1) {
+                cnt_blocks += __shfl_xor_sync(0xffffffffu, cnt_blocks, o);
+                cnt_raise += __shfl_xor_sync(0xffffffffu, cnt_raise, o);
+                cnt_taken += __shfl_xor_sync(0xffffffffu, cnt_taken, o);
+            }
+            if (lane == 0) {
+                atomicAdd(p.rescale_counts + 0, (unsigned long long)cnt_blocks);
+                atomicAdd(p.rescale_counts + 1, (unsigned long long)cnt_raise);
+                atomicAdd(p.rescale_counts + 2, (unsigned long long)cnt_taken);
+                atomicAdd(p.rescale_counts + 3, (unsigned long long)cnt_warp);
+            }
+        }
+#endif
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace tab

@@ -110,6 +110,10 @@ struct FwdParams {
     // into the range of its container (e4m3: (0, 2^8]; f16: below 2^16).
     float v_descale;
     float p_offset;
+    // Block-scaled FP4 kernel: scale-factor atoms (Q per 128-row tile, K and
+    // V per 128-key block; two 512-byte atoms each) and the tile counts.
+    const uint8_t *sf_q, *sf_k, *sf_v;
+    int nq_tiles, nk_tiles;
 };
 
 // Opt-in event trace (compile with -DATTN_TRACE): lane 0 of warps 0 and 4

@@ -120,6 +120,22 @@ __device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// Plain (untiled) bulk copy global -> shared, completing on `bar` with its
+// byte count; addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the
+// async proxy (tensor-core operand reads, tcgen05.cp) before it signals.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -208,6 +224,43 @@ __device__ __forceinline__ void mma_ts_k(uint32_t d_tmem, uint32_t a_tmem, uint6
     }
 }
 
+// Block-scaled FP4 products (both operands packed E2M1 in shared memory,
+// K = 64 per instruction, fp32 accumulator): NVFP4 with one UE4M3 scale per
+// 16 elements (kind::mxf4nvf4, block16), or MXFP4 with one UE8M0 scale per
+// 32 (kind::mxf4, block32).  sfa / sfb: tensor-memory addresses of the
+// scale factors, 128 rows in the 32-lane x 4-column layout tcgen05.cp
+// 32x128b.warpx4 writes (row m at lane m % 32, column m / 32, byte = block
+// within the K step).
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// 32 rows x 16 bytes of shared memory (the 512-byte scale-factor atom) into
+// tensor-memory columns [taddr, taddr + 4) of all four 32-lane quarters.
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -276,6 +329,32 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
                                                     uint32_t sbo_bytes) {
     return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16) |
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Shared-memory descriptor of a K-major tile with 64-byte rows and the
+// 64-byte swizzle (layout code 4): 16-byte chunk c of row r sits at chunk
+// c ^ ((r >> 1) & 3); 8-row groups are 512 bytes apart (SBO).  Tile base
+// 512-byte aligned; a K step of 32 bytes adds 2 to the start address.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(16 >> 4) << 16) |
+           ((uint64_t)(512 >> 4) << 32) | (1ull << 46) | (4ull << 61);
+}
+
+// Descriptor of a 512-byte scale-factor atom for tcgen05.cp: no swizzle,
+// 8-row groups of 16-byte rows 128 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sf_atom(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) |
+           ((uint64_t)(128 >> 4) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor of the block-scaled FP4 kinds: A and B E2M1 (format
+// code 1 in bits 7-9 and 10-12), both K-major, N >> 3 in bits 17-22, scale
+// format in bit 23 (0 UE4M3, 1 UE8M0), M >> 4 in bits 24-28; scale-factor
+// IDs (bits 4-5, 29-30) 0: each K step reads bytes from the first of its
+// scale words.
+__host__ __device__ constexpr uint32_t idesc_fp4_bs(int M, int N, int ue8m0) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)ue8m0 << 23) |
+           ((uint32_t)(M >> 4) << 24);
 }
 
 // Instruction descriptor, kind::f16 with bf16 inputs and an fp32
@@ -381,6 +460,18 @@ __device__ __forceinline__ uint32_t e2m1_round_f16x2(float x0, float x1) {
     asm("{\n\t.reg .b8 t;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
         "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(x0), "f"(x1));
+    return r;
+}
+
+// Two fp32 values rounded to E2M1 (nearest, ties to even, saturating at
+// +-6): one byte, x0 in the low nibble.
+__device__ __forceinline__ uint32_t e2m1x2_round(float x0, float x1) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
         : "=r"(r)
         : "f"(x0), "f"(x1));
     return r;
