@@ -5,9 +5,13 @@
 // probabilities built directly as MXFP4 values -- E2M1 codes with one
 // power-of-two scale per 32 keys, chosen by the affine classifier or the
 // rounded exponential -- and P V as an MXFP4 product, the softmax
-// normaliser being the sum of exactly those values.  The codes, block
-// exponents and sums are those of the f16-operand Direct-P kernel
-// (direct_p_half in fwd_kernel.cuh): only where the products run differs.
+// normaliser being the sum of exactly those values.  The codes and block
+// exponents are those of the f16-operand Direct-P kernel (direct_p_half in
+// fwd_kernel.cuh).  The normaliser -- the sum of the represented values --
+// comes from the tensor cores too: each V^T tile carries an extra row of
+// E2M1 ones (scale 2^0), so P V with N = 136 leaves sum_j w_j in column 128
+// of O, accumulated exactly as the output is.  The softmax warps then only
+// classify and pack codes.
 //
 // CTA shape and roles as in attn_fwd_kernel: two 128-row query tiles of one
 // (batch, query head), warps 0-3 / 4-7 softmax + correction + epilogue of
@@ -21,16 +25,18 @@
 // issued once this tile's softmax has loaded its scores.  At FP4 rates the
 // products are short against the softmax, which is what bounds the loop.
 //   [  0,128) S (tile 0 and tile 1 in turn)
-//   [128,256) O0, [256,384) O1
-//   [384,400) Q scales  (tile i, K step ks: 384 + 4 (2i + ks))
-//   [400,416) K scales  (block parity, K step)
-//   [416,432) V scales  (block parity, K step)
-//   [432,448) P scales  (tile, K step)
+//   [128,264) O0 (column 128 of it: the row sum), [272,408) O1
+//   [416,432) Q scales  (tile i, K step ks: 416 + 4 (2i + ks))
+//   [432,448) K scales  (block parity, K step)
+//   [448,480) V scales  (block parity, K step; 8 columns: rows 0-127, then
+//             rows 128-135 -- the ones row -- written once)
+//   [480,496) P scales  (tile, K step)
 //
 // Shared memory: Q0, Q1 and a ring of NS slots (K codes or V^T codes, each
-// 128 rows x 64 bytes with the 64-byte swizzle, followed by their two
-// scale atoms), P0 and P1 as codes in the same layout, and the P scale
-// atoms the softmax warps write.
+// 128 rows x 64 bytes with the 64-byte swizzle, then 8 more rows -- the ones
+// row and seven zero rows, written once -- then their two scale atoms), P0
+// and P1 as codes in the same layout, and the P scale atoms the softmax
+// warps write.
 //
 // Ordering (all products of one thread execute in issue order): per block
 // j and tile i the MMA warp issues P_i V(j) and then Q_i K^T(j+1), so the
@@ -46,9 +52,13 @@
 namespace tab {
 
 constexpr int kFp4Tile = kBlockM * 64;               // 8 KB of codes
-constexpr int kFp4Slot = kFp4Tile + 2 * kSfAtom;     // codes + two scale atoms
-constexpr uint32_t kColS = 0, kColO = 128, kColSfQ = 384, kColSfK = 400, kColSfV = 416,
-                   kColSfP = 432;
+constexpr int kFp4Extra = 8 * 64;                    // rows 128-135 of a V^T tile
+constexpr int kFp4SfOff = kFp4Tile + kFp4Extra;      // the slot's two scale atoms
+constexpr int kFp4Slot = 10 * 1024;                  // slot stride, 1024-aligned
+static_assert(kFp4SfOff + 2 * kSfAtom <= kFp4Slot, "slot layout");
+constexpr int kPvN = 136;                            // D columns of O plus the sum rows
+constexpr uint32_t kColS = 0, kColO = 128, kOStride = 144, kColSfQ = 416, kColSfK = 432,
+                   kColSfV = 448, kColSfP = 480;
 
 template <int NS>
 struct FwdSmemFp4 {
@@ -57,6 +67,7 @@ struct FwdSmemFp4 {
     alignas(1024) uint8_t kv[NS][kFp4Slot];
     alignas(1024) uint8_t p[2][kFp4Tile];
     uint8_t psf[2][2][kSfAtom];
+    uint8_t ones_sf[kSfAtom];  // scales of V^T rows 128-159 (2^0)
     uint64_t q_full;
     uint64_t kv_full[NS];
     uint64_t kv_empty[NS];
@@ -73,12 +84,11 @@ struct FwdSmemFp4 {
 
 // Codes of 64 scores of a row (two 32-key blocks with maxima bm[0], bm[1]):
 // per block the exponent E, the 16 bytes of E2M1 codes (key 2k in the low
-// nibble of byte k) and the UE8M0 byte E + 127; returns the fp32 sum of the
-// represented values code * 2^E.  Same steps and constants as direct_p_half.
+// nibble of byte k) and the UE8M0 byte E + 127.  Same steps and constants
+// as direct_p_half.
 template <int CLS>
-__device__ __forceinline__ float direct_p_codes(const float *s, const float *bm, float c,
-                                                float base, uint4 *codes, uint32_t &sf2) {
-    float sum = 0.0f;
+__device__ __forceinline__ void direct_p_codes(const float *s, const float *bm, float c,
+                                               float base, uint4 *codes, uint32_t &sf2) {
     sf2 = 0u;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -89,7 +99,6 @@ __device__ __forceinline__ float direct_p_codes(const float *s, const float *bm,
         const float nb = keep ? base - (float)ei : -INFINITY;  // r = s*c + nb
         sf2 |= (uint32_t)(ei + 127) << (8 * u);
         const float c2 = 2.0f * c, nb2 = 2.0f * nb + (2.0f + kRintMagic);
-        uint32_t cs0 = 0u, cs1 = 0u;
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -110,16 +119,11 @@ __device__ __forceinline__ float direct_p_codes(const float *s, const float *bm,
                     byte = e2m1x2_round(ex2_mufu(r0), ex2_mufu(r1));
                 }
                 word |= byte << (4 * e);
-                const uint32_t h = e2m1x2_to_f16x2(byte);
-                if ((e & 2) == 0) cs0 = hadd2_u32(cs0, h);
-                else cs1 = hadd2_u32(cs1, h);
             }
             w[q] = word;
         }
         codes[u] = make_uint4(w[0], w[1], w[2], w[3]);
-        if (keep) sum += f16x2_sum(hadd2_u32(cs0, cs1)) * __uint_as_float((uint32_t)(ei + 127) << 23);
     }
-    return sum;
 }
 
 template <int NS, int CLS>
@@ -175,6 +179,18 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
         sm.abort_flag = 0;
         fence_mbar_init();
     }
+    // Rows 128-135 of every slot: row 128 all E2M1 ones (code 2), the rest
+    // zero (the 64-byte swizzle permutes chunks within a row: a constant row
+    // is the same either way); their scale atom: 2^0 (UE8M0 127) for the two
+    // 32-key blocks of each K step.
+    for (int x = threadIdx.x; x < NS * kFp4Extra / 16; x += kFwdThreads) {
+        const int slot = x / (kFp4Extra / 16), off = x % (kFp4Extra / 16);
+        const uint32_t v = off < 4 ? 0x22222222u : 0u;
+        *reinterpret_cast<uint4 *>(sm.kv[slot] + kFp4Tile + off * 16) = make_uint4(v, v, v, v);
+    }
+    for (int x = threadIdx.x; x < kSfAtom / 4; x += kFwdThreads)
+        reinterpret_cast<uint32_t *>(sm.ones_sf)[x] = 0x00007F7Fu;
+    fence_proxy_async_smem();
     if (warp == 9) {
         for (int i = 0; i < 2; ++i) {
             const int r0 = q0 + i * kBlockM;
@@ -233,14 +249,14 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                         if (!ok) break;
                         // Testing only: the first CTA withholds its first K copy.
                         if (p.debug_withhold_kv && blockIdx.x == 0 && it == 0) continue;
-                        mbar_arrive_expect_tx(&sm.kv_full[slot], kFp4Slot);
+                        mbar_arrive_expect_tx(&sm.kv_full[slot], kFp4Tile + 2 * kSfAtom);
                         const size_t atoms = (((size_t)b * p.Hkv + hkv) * p.nk_tiles + j) * (2 * kSfAtom);
                         if (which == 0) {
                             tma_load_4d(sm.kv[slot], &p.tm_k, &sm.kv_full[slot], 0, j * kBlockN, hkv, b);
-                            bulk_load(sm.kv[slot] + kFp4Tile, p.sf_k + atoms, 2 * kSfAtom, &sm.kv_full[slot]);
+                            bulk_load(sm.kv[slot] + kFp4SfOff, p.sf_k + atoms, 2 * kSfAtom, &sm.kv_full[slot]);
                         } else {
                             tma_load_4d(sm.kv[slot], &p.tm_v, &sm.kv_full[slot], j * 64, 0, hkv, b);
-                            bulk_load(sm.kv[slot] + kFp4Tile, p.sf_v + atoms, 2 * kSfAtom, &sm.kv_full[slot]);
+                            bulk_load(sm.kv[slot] + kFp4SfOff, p.sf_v + atoms, 2 * kSfAtom, &sm.kv_full[slot]);
                         }
                     }
                 }
@@ -255,7 +271,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
             if (n_blocks > 0) {
                 const bool leader = elect_one();
                 constexpr uint32_t kIdescQK = idesc_fp4_bs(kBlockM, kBlockN, 0);  // UE4M3 scales
-                constexpr uint32_t kIdescPV = idesc_fp4_bs(kBlockM, 128, 1);      // UE8M0 scales
+                constexpr uint32_t kIdescPV = idesc_fp4_bs(kBlockM, kPvN, 1);     // UE8M0 scales
                 const uint64_t q_desc = smem_desc_sw64(smem_u32(sm.q[0]));
                 const uint64_t kv_desc = smem_desc_sw64(smem_u32(sm.kv[0]));
                 const uint64_t p_desc = smem_desc_sw64(smem_u32(sm.p[0]));
@@ -267,6 +283,9 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                         for (int ks = 0; ks < 2; ++ks)
                             tc_cp_sf(tmem + kColSfQ + 4 * (2 * i + ks),
                                      smem_desc_sf_atom(smem_u32(sm.qsf[i][ks])));
+                    // Scales of the ones row, once for the four V scale groups.
+                    for (int g = 0; g < 4; ++g)
+                        tc_cp_sf(tmem + kColSfV + 8 * g + 4, smem_desc_sf_atom(smem_u32(sm.ones_sf)));
                 }
                 __syncwarp();
                 auto ring_pos = [&](int j, int which) -> uint32_t {
@@ -281,7 +300,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                                                                   abort_flag, p.status, true, p.timeout_ns));
                     tc_fence_after();
                     if (ok && leader) {
-                        const uint8_t *atoms = sm.kv[L % NS] + kFp4Tile;
+                        const uint8_t *atoms = sm.kv[L % NS] + kFp4SfOff;
                         for (int ks = 0; ks < 2; ++ks)
                             tc_cp_sf(tmem + kColSfK + 4 * (2 * (j & 1) + ks),
                                      smem_desc_sf_atom(smem_u32(atoms + ks * kSfAtom)));
@@ -331,8 +350,8 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                     tc_fence_after();
                     if (leader)
                         for (int ks = 0; ks < 2; ++ks)
-                            tc_cp_sf(tmem + kColSfV + 4 * (2 * (j & 1) + ks),
-                                     smem_desc_sf_atom(smem_u32(sm.kv[vslot] + kFp4Tile + ks * kSfAtom)));
+                            tc_cp_sf(tmem + kColSfV + 8 * (2 * (j & 1) + ks),
+                                     smem_desc_sf_atom(smem_u32(sm.kv[vslot] + kFp4SfOff + ks * kSfAtom)));
                     __syncwarp();
                     const uint64_t vb = kv_desc + ((vslot * kFp4Slot) >> 4);
                     for (int i = 0; i < 2 && ok; ++i) {
@@ -340,7 +359,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                             const int lo_i = i == 0 ? lo0 : lo1;
                             const int hi_i = i == 0 ? hi0 : hi1;
                             const uint32_t par = (uint32_t)(j - lo_i) & 1u;
-                            const uint32_t o_tmem = tmem + kColO + i * 128;
+                            const uint32_t o_tmem = tmem + kColO + i * kOStride;
                             const uint64_t pa = p_desc + ((i * kFp4Tile) >> 4);
                             // Keys [0, 64) as soon as their codes are in shared memory.
                             ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_half[i], par, abort_flag,
@@ -350,7 +369,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                             if (leader) {
                                 tc_cp_sf(tmem + kColSfP + 4 * (2 * i), smem_desc_sf_atom(smem_u32(sm.psf[i][0])));
                                 mma_mxf4(o_tmem, pa, vb, kIdescPV, tmem + kColSfP + 4 * (2 * i),
-                                         tmem + kColSfV + 4 * (2 * (j & 1)), j > lo_i ? 1u : 0u);
+                                         tmem + kColSfV + 8 * (2 * (j & 1)), j > lo_i ? 1u : 0u);
                             }
                             __syncwarp();
                             ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_full[i], par, abort_flag,
@@ -361,7 +380,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                                 tc_cp_sf(tmem + kColSfP + 4 * (2 * i + 1),
                                          smem_desc_sf_atom(smem_u32(sm.psf[i][1])));
                                 mma_mxf4(o_tmem, pa + 2, vb + 2, kIdescPV, tmem + kColSfP + 4 * (2 * i + 1),
-                                         tmem + kColSfV + 4 * (2 * (j & 1) + 1), 1u);
+                                         tmem + kColSfV + 8 * (2 * (j & 1) + 1), 1u);
                                 if (j == hi_i) tc_commit(&sm.o_final[i]);
                             }
                             __syncwarp();
@@ -395,7 +414,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
         const int row = q0 + i * kBlockM + row_in_tile;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t s_tmem = tmem + lane_base + kColS;
-        const uint32_t o_tmem = tmem + lane_base + kColO + i * 128;
+        const uint32_t o_tmem = tmem + lane_base + kColO + i * kOStride;
         const KeyRange kr = row_key_range(p, row);
         const int lo_b = i == 0 ? lo0 : lo1;
         const int hi_b = i == 0 ? hi0 : hi1;
@@ -411,7 +430,6 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
         uint32_t cnt_blocks = 0, cnt_raise = 0, cnt_taken = 0, cnt_warp = 0;
 #endif
         float m_run = -INFINITY;
-        float l_run = 0.0f;
         bool ok = true;
 
         for (int j = lo_b; j <= hi_b; ++j) {
@@ -457,10 +475,10 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                 m_run = m_new;
             }
             const float neg_m = m_run == -INFINITY ? 0.0f : p.p_offset - m_run;
-            l_run *= alpha;
 
-            // Correction: P_i V(j-1) is complete (S of this block was committed
-            // after it), P_i V(j) is not yet issued.
+            // Correction (of O and of its sum column): P_i V(j-1) is complete
+            // (S of this block was committed after it), P_i V(j) is not yet
+            // issued.
             if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #ifdef ATTN_COUNT_RESCALES
                 ++cnt_warp;
@@ -480,6 +498,12 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                     }
                     tmem_st32(o_tmem + ch * 32, rr);
                 }
+                uint32_t r8[8];
+                tmem_ld8(o_tmem + 128, r8);
+                tmem_wait_ld();
+                reg_fence8(r8);
+                r8[0] = __float_as_uint(__uint_as_float(r8[0]) * alpha);
+                tmem_st8(o_tmem + 128, r8);
                 tmem_wait_st();
             }
 
@@ -489,7 +513,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
             for (int half = 0; half < 2; ++half) {
                 uint4 codes[2];
                 uint32_t sf2;
-                l_run += direct_p_codes<CLS>(s + 64 * half, bm + 2 * half, c, neg_m, codes, sf2);
+                direct_p_codes<CLS>(s + 64 * half, bm + 2 * half, c, neg_m, codes, sf2);
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
                     *reinterpret_cast<uint4 *>(p_row + (((2 * half + u) ^ swz) << 4)) = codes[u];
@@ -509,6 +533,14 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
         }
         if (ok) {
             const bool row_ok = row < p.Sq;
+            float l_run = 0.0f;  // sum of the represented weights, from the ones row
+            if (has_blocks) {
+                uint32_t r8[8];
+                tmem_ld8(o_tmem + 128, r8);
+                tmem_wait_ld();
+                reg_fence8(r8);
+                l_run = __uint_as_float(r8[0]);
+            }
             const float inv_l = l_run > 0.0f ? p.v_descale / l_run : 0.0f;
             __nv_bfloat16 *o_row = p.o + (((size_t)b * p.Sq + row) * p.Hq + hq) * (size_t)128;
 #pragma unroll
