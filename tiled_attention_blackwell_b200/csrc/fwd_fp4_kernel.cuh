@@ -84,11 +84,22 @@ struct FwdSmemFp4 {
 
 // Codes of 64 scores of a row (two 32-key blocks with maxima bm[0], bm[1]):
 // per block the exponent E, the 16 bytes of E2M1 codes (key 2k in the low
-// nibble of byte k) and the UE8M0 byte E + 127.  Same steps and constants
-// as direct_p_half.
+// nibble of byte k) and the UE8M0 byte E + 127.  Same block exponents and
+// decisions as direct_p_half, with work moved off the ALU pipe:
+//   affine: index clamp(rint(2r + 2), 0, 7) as u = sat((2r + 2) / 8) (one
+//     FFMA with saturation; the scaling by 1/4 and 8 is exact), rint(8u)
+//     through the 1.5 * 2^23 offset (packed FFMA), the eight indices of a
+//     word summed into their nibbles by shifted adds of the raw float bits
+//     (the offset's bits are a known constant), then 8 -> 7;
+//   exp2: 2^r rounded by the E2M1 conversion, four conversions per word.
 template <int CLS>
 __device__ __forceinline__ void direct_p_codes(const float *s, const float *bm, float c,
                                                float base, uint4 *codes, uint32_t &sf2) {
+    constexpr uint32_t kMagicBits = 0x4B400000u;  // kRintMagic
+    constexpr uint32_t kMagicNibbles = kMagicBits + (kMagicBits << 4) + (kMagicBits << 8) +
+                                       (kMagicBits << 12) + (kMagicBits << 16) +
+                                       (kMagicBits << 20) + (kMagicBits << 24) +
+                                       (kMagicBits << 28);
     sf2 = 0u;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -98,29 +109,36 @@ __device__ __forceinline__ void direct_p_codes(const float *s, const float *bm, 
         const int ei = keep ? (int)fminf(ef, 13.0f) : 0;
         const float nb = keep ? base - (float)ei : -INFINITY;  // r = s*c + nb
         sf2 |= (uint32_t)(ei + 127) << (8 * u);
-        const float c2 = 2.0f * c, nb2 = 2.0f * nb + (2.0f + kRintMagic);
         uint32_t w[4];
+        if constexpr (CLS == 0) {
+            const float c4 = 0.25f * c, nb4 = 0.25f * (nb + 1.0f);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint32_t word = 0u;
+            for (int q = 0; q < 4; ++q) {
+                uint32_t word = 0u;
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                const float s0 = s[32 * u + 8 * q + e], s1 = s[32 * u + 8 * q + e + 1];
-                uint32_t byte;
-                if constexpr (CLS == 0) {
+                for (int e = 0; e < 8; e += 2) {
+                    const float u0 = __saturatef(fmaf(s[32 * u + 8 * q + e], c4, nb4));
+                    const float u1 = __saturatef(fmaf(s[32 * u + 8 * q + e + 1], c4, nb4));
                     float t0, t1;
-                    fma2(t0, t1, s0, s1, c2, c2, nb2, nb2);
-                    t0 = fminf(fmaxf(t0, kRintMagic), kRintMagic + 7.0f);
-                    t1 = fminf(fmaxf(t1, kRintMagic), kRintMagic + 7.0f);
-                    byte = (__float_as_uint(t0) & 7u) | ((__float_as_uint(t1) & 7u) << 4);
-                } else {
-                    float r0, r1;
-                    fma2(r0, r1, s0, s1, c, c, nb, nb);
-                    byte = e2m1x2_round(ex2_mufu(r0), ex2_mufu(r1));
+                    fma2(t0, t1, u0, u1, 8.0f, 8.0f, kRintMagic, kRintMagic);
+                    word += (__float_as_uint(t0) << (4 * e)) + (__float_as_uint(t1) << (4 * e + 4));
                 }
-                word |= byte << (4 * e);
+                word -= kMagicNibbles;                    // nibbles k in [0, 8]
+                w[q] = word - ((word >> 3) & 0x11111111u);  // 8 -> 7
             }
-            w[q] = word;
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    float r0, r1;
+                    fma2(r0, r1, s[32 * u + 8 * q + e], s[32 * u + 8 * q + e + 1], c, c, nb, nb);
+                    x[e] = ex2_mufu(r0);
+                    x[e + 1] = ex2_mufu(r1);
+                }
+                w[q] = e2m1x8_round(x);
+            }
         }
         codes[u] = make_uint4(w[0], w[1], w[2], w[3]);
     }

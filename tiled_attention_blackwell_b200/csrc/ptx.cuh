@@ -494,6 +494,21 @@ __device__ __forceinline__ uint32_t e2m1x2_round(float x0, float x1) {
     return r;
 }
 
+// Eight fp32 values rounded to E2M1 (nearest, ties to even, saturating at
+// +-6), packed into one word: x[k] in nibble k.
+__device__ __forceinline__ uint32_t e2m1x8_round(const float *x) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
+    return r;
+}
+
 // The f16 pair of two E2M1 codes held in the low byte of `codes` (low
 // nibble -> low half).
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t codes) {
