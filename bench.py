@@ -49,6 +49,8 @@ KERNEL_SOURCES = ["tiled_attention_blackwell_b200/csrc/fwd_kernel.cuh",
                   "tiled_attention_blackwell_b200/csrc/ptx.cuh",
                   "tiled_attention_blackwell_b200/csrc/exp2_poly.cuh",
                   "tiled_attention_blackwell_b200/csrc/fp4_dequant.cuh",
+                  "tiled_attention_blackwell_b200/csrc/fp4_prepare.cuh",
+                  "tiled_attention_blackwell_b200/csrc/fwd_fp4_kernel.cuh",
                   "tiled_attention_blackwell_b200/csrc/attn_api.cu"]
 FP4_INPUTS = ("q_codes", "q_scales", "k_codes", "k_scales", "v_codes", "v_scales")
 
@@ -72,6 +74,9 @@ def parse_args(argv=None):
                     help="time with ALiBi slopes 2^(-8(h+1)/Hq)")
     ap.add_argument("--classifier", default="affine", choices=["affine", "exp2"],
                     help="Direct-P code classifier of the fp4 workloads")
+    ap.add_argument("--fp4-mma", default="block_scaled", choices=["block_scaled", "f16"],
+                    help="tensor-core products of the fp4 workloads: block-scaled FP4 "
+                         "(default) or f16 operands after a widening pass")
     ap.add_argument("--sustained-seconds", type=float, default=2.0,
                     help="length of the back-to-back run of the 'sustained' record (0: skip)")
     ap.add_argument("--no-rescale-stats", action="store_true",
@@ -404,6 +409,7 @@ def run_ours(args):
                           dtype=torch.uint8, device=device)
         cfg["classifier"] = args.classifier
         cfg["formats"] = "NVFP4 Q/K (power-of-two e4m3 block scales), MXFP4 V and P"
+        cfg["products"] = args.fp4_mma
     lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=device)
     window = None if w.window == (-1, -1) else w.window
     slopes = None
@@ -460,7 +466,7 @@ def run_ours(args):
                               d["k_scales"], inp["k_global"], d["v_codes"], d["v_scales"],
                               inp["v_global"], outs[0], outs[1], ws4, scale=w.scale,
                               causal=w.causal, window=window, doc_offsets=docs,
-                              classifier=args.classifier, stream=s)
+                              classifier=args.classifier, mma=args.fp4_mma, stream=s)
         elif fp8:
             attn.attn_fwd_fp8(d["q"], d["k"], d["v"], outs[0], outs[1],
                               q_descale=inp["q_descale"], k_descale=inp["k_descale"],
@@ -588,17 +594,19 @@ def run_ours(args):
 
     peaks, peak_kind = read_peaks()
     achieved = flops / (launch_avg_ms / 1e3) / 1e12
-    # fp8 contractions: the measured bf16 peak times the nominal dense
-    # fp8 / bf16 ratio (4.5 / 2.25 PFLOP/s).
-    peak_mult = 2.0 if fp8 else 1.0
+    # fp8 and block-scaled fp4 contractions: the measured bf16 peak times the
+    # nominal dense fp8 / bf16 (4.5 / 2.25) or fp4 / bf16 (9 / 2.25) ratio.
+    fp4_bs = fp4 and args.fp4_mma == "block_scaled"
+    peak_mult = 2.0 if fp8 else (4.0 if fp4_bs else 1.0)
     peak = float(peaks["bf16_tflops"]) * peak_mult
     metric = metric_for(w, args.softcap, slopes is not None, args.classifier)
     result = {
         "metric": metric, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": ("fp8e4m3" if fp8 else "fp4e2m1 (NVFP4/MXFP4) on f16 tensor operands"
-                  if fp4 else "bf16"),
+        "dtype": ("fp8e4m3" if fp8 else
+                  ("fp4e2m1 (NVFP4 Q/K, MXFP4 P/V) on block-scaled FP4 tensor cores" if fp4_bs
+                   else "fp4e2m1 (NVFP4/MXFP4) on f16 tensor operands") if fp4 else "bf16"),
         "data": "synthetic", "config": cfg,
         "pct_of_peak": round(100.0 * value / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
@@ -606,7 +614,8 @@ def run_ours(args):
                      "traffic": profiled_traffic(w.name),
                      "peak_source": (f"{peak_kind} bf16 burst (MEASURED_PEAKS.json)"
                                      if peak_kind == "measured" else "fallback 1590 TFLOP/s")
-                     + (" x 2 (nominal fp8/bf16 dense ratio)" if fp8 else ""),
+                     + (" x 2 (nominal fp8/bf16 dense ratio)" if fp8 else "")
+                     + (" x 4 (nominal fp4/bf16 dense ratio)" if fp4_bs else ""),
                      "frac_of_sustained": round(achieved / (peak_mult * float(
                          peaks.get("bf16_tflops_sustained", peak))), 4),
                      "flops_per_launch": flops, "launch_ms": round(launch_avg_ms, 4),
@@ -614,7 +623,9 @@ def run_ours(args):
                                            if burst_clocks["sm_mhz"] else None),
                      "kernel": "attn_bwd (dQ kernel with the D_i row terms, then dK/dV kernel)"
                      if w.backward else
-                     ("attn_fwd_fp4 (fp4_dequant_kernel + attn_fwd_kernel, timed together)"
+                     (("attn_fwd_fp4 (fp4_prepare_kernel + attn_fwd_fp4bs_kernel, timed together)"
+                       if fp4_bs else
+                       "attn_fwd_fp4 (fp4_dequant_kernel + attn_fwd_kernel, timed together)")
                       if fp4 else "attn_fwd_kernel")},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,

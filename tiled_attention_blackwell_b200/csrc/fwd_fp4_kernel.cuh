@@ -13,9 +13,12 @@
 // of O, accumulated exactly as the output is.  The softmax warps then only
 // classify and pack codes.
 //
-// CTA shape and roles as in attn_fwd_kernel: two 128-row query tiles of one
-// (batch, query head), warps 0-3 / 4-7 softmax + correction + epilogue of
-// tile 0 / 1, warp 8 MMA issue, warp 9 TMA producer.
+// CTA shape as in attn_fwd_kernel: two 128-row query tiles of one (batch,
+// query head).  Roles: warps 0-3 / 4-7 softmax + correction + epilogue of
+// tile 0 / 1, warp 8 issues Q K^T (and allocates TMEM), warp 9 is the TMA
+// producer, warp 10 issues P V.  Two issuers because the two products wait
+// on different things: Q K^T on the shared S region being loaded, P V on P
+// being written; one in-order issuer would hold each behind the other.
 //
 // Tensor memory is where this kernel differs ("Contribuciones Clave":
 // tensor-memory ownership bounds the overlap).  Block-scaled products read
@@ -38,12 +41,12 @@
 // and P1 as codes in the same layout, and the P scale atoms the softmax
 // warps write.
 //
-// Ordering (all products of one thread execute in issue order): per block
-// j and tile i the MMA warp issues P_i V(j) and then Q_i K^T(j+1), so the
-// arrival of S(i, j+1) proves that P_i V(j) has completed -- the softmax may
-// then rescale O_i and overwrite P_i and its scales.  Scale columns of K
-// and V alternate by block parity; every reuse is two blocks apart, after a
-// commit the MMA warp has already waited on.
+// Ordering.  Each issuer's tensor-core operations execute in its issue
+// order, so a scale column or shared-memory operand that one of them
+// rewrites has been read by its earlier products.  Scale columns of K and V
+// alternate by block parity.  The softmax warps learn from pv_done[i] (a
+// commit after P_i V(j)) that O_i may be rescaled and P_i rewritten for
+// block j + 1; s_free orders the tiles' use of the S region.
 #pragma once
 
 #include "fp4_prepare.cuh"
@@ -76,7 +79,9 @@ struct FwdSmemFp4 {
     uint64_t p_half[2];  // codes and scales of keys [0, 64) are in shared memory
     uint64_t p_full[2];  // all of P (and any O correction)
     uint64_t o_final[2];
+    uint64_t pv_done[2];  // P_i V(j) has completed: P_i and O_i are free again
     uint64_t drain;
+    uint64_t drain_pv;
     uint32_t tmem_base;
     int abort_flag;
     int range[2][2];
@@ -193,7 +198,10 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
             mbar_init(&sm.o_final[i], 1);
         }
         mbar_init(&sm.s_free, kBlockM);
+        mbar_init(&sm.pv_done[0], 1);
+        mbar_init(&sm.pv_done[1], 1);
         mbar_init(&sm.drain, 1);
+        mbar_init(&sm.drain_pv, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -285,82 +293,91 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
             }
             __syncwarp();
         } else if (warp == 8) {
-            // --------------------------------------------------- MMA issuer
+            // ------------------------------------------- Q K^T issuer (S ring)
+            // One S region serves both tiles in turn: the n-th product waits
+            // until the tile that owned the region has loaded its scores.
             if (n_blocks > 0) {
                 const bool leader = elect_one();
                 constexpr uint32_t kIdescQK = idesc_fp4_bs(kBlockM, kBlockN, 0);  // UE4M3 scales
-                constexpr uint32_t kIdescPV = idesc_fp4_bs(kBlockM, kPvN, 1);     // UE8M0 scales
                 const uint64_t q_desc = smem_desc_sw64(smem_u32(sm.q[0]));
                 const uint64_t kv_desc = smem_desc_sw64(smem_u32(sm.kv[0]));
-                const uint64_t p_desc = smem_desc_sw64(smem_u32(sm.p[0]));
                 bool ok = __all_sync(0xffffffffu,
                                      wait_bounded(&sm.q_full, 0, abort_flag, p.status, true, p.timeout_ns));
                 tc_fence_after();
-                if (ok && leader) {
+                if (ok && leader)
                     for (int i = 0; i < 2; ++i)
                         for (int ks = 0; ks < 2; ++ks)
                             tc_cp_sf(tmem + kColSfQ + 4 * (2 * i + ks),
                                      smem_desc_sf_atom(smem_u32(sm.qsf[i][ks])));
-                    // Scales of the ones row, once for the four V scale groups.
-                    for (int g = 0; g < 4; ++g)
-                        tc_cp_sf(tmem + kColSfV + 8 * g + 4, smem_desc_sf_atom(smem_u32(sm.ones_sf)));
-                }
                 __syncwarp();
-                auto ring_pos = [&](int j, int which) -> uint32_t {
-                    return 2u * (uint32_t)(j - ulo) + (uint32_t)which;
-                };
-                int k_ready = ulo - 1;  // last key block whose K slot was waited on
-                uint32_t n_qk = 0;      // Q K^T products issued (the shared S region's turns)
-                auto wait_k = [&](int j) {
-                    const uint32_t L = ring_pos(j, 0);
-                    if (ok)
-                        ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u,
-                                                                  abort_flag, p.status, true, p.timeout_ns));
+                uint32_t n_qk = 0;
+                for (int j = ulo; j <= uhi && ok; ++j) {
+                    const uint32_t Lk = 2u * (uint32_t)(j - ulo);
+                    const uint32_t kslot = Lk % NS;
+                    ATTN_TRACE_EVENT(2, j - ulo, 0);
+                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[kslot], (Lk / NS) & 1u,
+                                                              abort_flag, p.status, true, p.timeout_ns));
+                    if (!ok) break;
                     tc_fence_after();
-                    if (ok && leader) {
-                        const uint8_t *atoms = sm.kv[L % NS] + kFp4SfOff;
+                    if (leader)
                         for (int ks = 0; ks < 2; ++ks)
                             tc_cp_sf(tmem + kColSfK + 4 * (2 * (j & 1) + ks),
-                                     smem_desc_sf_atom(smem_u32(atoms + ks * kSfAtom)));
-                    }
+                                     smem_desc_sf_atom(smem_u32(sm.kv[kslot] + kFp4SfOff + ks * kSfAtom)));
                     __syncwarp();
-                    k_ready = j;
-                };
-                auto issue_s = [&](int i, int j) {
-                    if (k_ready < j) wait_k(j);
-                    if (!ok) return;
-                    if (n_qk > 0) {
-                        ok = __all_sync(0xffffffffu, wait_bounded(&sm.s_free, (n_qk - 1) & 1u, abort_flag,
-                                                                  p.status, true, p.timeout_ns));
-                        if (!ok) return;
-                        tc_fence_after();
-                    }
-                    const uint64_t a0 = q_desc + ((i * kFp4Tile) >> 4);
-                    const uint64_t b0 = kv_desc + (((ring_pos(j, 0) % NS) * kFp4Slot) >> 4);
-                    if (leader) {
+                    const uint64_t b0 = kv_desc + ((kslot * kFp4Slot) >> 4);
+                    for (int i = 0; i < 2 && ok; ++i) {
+                        const bool act = i == 0 ? (has0 && j >= lo0 && j <= hi0)
+                                                : (has1 && j >= lo1 && j <= hi1);
+                        if (!act) continue;
+                        if (n_qk > 0) {
+                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.s_free, (n_qk - 1) & 1u,
+                                                                      abort_flag, p.status, true,
+                                                                      p.timeout_ns));
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                        ATTN_TRACE_EVENT(2, j - ulo, 1 + i);
+                        const uint64_t a0 = q_desc + ((i * kFp4Tile) >> 4);
+                        if (leader) {
 #pragma unroll
-                        for (int ks = 0; ks < 2; ++ks)
-                            mma_nvf4(tmem + kColS, a0 + 2 * ks, b0 + 2 * ks, kIdescQK,
-                                     tmem + kColSfQ + 4 * (2 * i + ks),
-                                     tmem + kColSfK + 4 * (2 * (j & 1) + ks), ks > 0 ? 1u : 0u);
-                        tc_commit(&sm.s_full[i]);
+                            for (int ks = 0; ks < 2; ++ks)
+                                mma_nvf4(tmem + kColS, a0 + 2 * ks, b0 + 2 * ks, kIdescQK,
+                                         tmem + kColSfQ + 4 * (2 * i + ks),
+                                         tmem + kColSfK + 4 * (2 * (j & 1) + ks), ks > 0 ? 1u : 0u);
+                            tc_commit(&sm.s_full[i]);
+                        }
+                        __syncwarp();
+                        ++n_qk;
                     }
+                    if (!ok) break;
+                    if (leader) tc_commit(&sm.kv_empty[kslot]);
                     __syncwarp();
-                    ++n_qk;
-                };
-                auto active = [&](int i, int j) -> bool {
-                    return i == 0 ? (has0 && j >= lo0 && j <= hi0)
-                                  : (has1 && j >= lo1 && j <= hi1);
-                };
-
-                for (int i = 0; i < 2; ++i)
-                    if (active(i, ulo)) issue_s(i, ulo);
-                if (ok && k_ready < ulo) wait_k(ulo);
-                if (ok && leader) tc_commit(&sm.kv_empty[ring_pos(ulo, 0) % NS]);
+                }
+                if (!ok) {
+                    // Let every product and copy already issued finish before TMEM is freed.
+                    if (leader) tc_commit(&sm.drain);
+                    __syncwarp();
+                    wait_bounded(&sm.drain, 0, abort_flag, p.status, false, p.timeout_ns);
+                }
+            }
+            __syncwarp();
+        } else if (warp == 10) {
+            // ---------------------------------------------------- P V issuer
+            // P_i V(j) as soon as P_i of block j is in shared memory (keys
+            // [0, 64) first); pv_done[i] tells the softmax warps that P_i and
+            // O_i may be touched again.
+            if (n_blocks > 0) {
+                const bool leader = elect_one();
+                constexpr uint32_t kIdescPV = idesc_fp4_bs(kBlockM, kPvN, 1);  // UE8M0 scales
+                const uint64_t kv_desc = smem_desc_sw64(smem_u32(sm.kv[0]));
+                const uint64_t p_desc = smem_desc_sw64(smem_u32(sm.p[0]));
+                if (leader)  // scales of the ones row, once for the four V scale groups
+                    for (int g = 0; g < 4; ++g)
+                        tc_cp_sf(tmem + kColSfV + 8 * g + 4, smem_desc_sf_atom(smem_u32(sm.ones_sf)));
                 __syncwarp();
-
+                bool ok = true;
                 for (int j = ulo; j <= uhi && ok; ++j) {
-                    const uint32_t Lv = ring_pos(j, 1);
+                    const uint32_t Lv = 2u * (uint32_t)(j - ulo) + 1u;
                     const uint32_t vslot = Lv % NS;
                     ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[vslot], (Lv / NS) & 1u,
                                                               abort_flag, p.status, true, p.timeout_ns));
@@ -373,57 +390,51 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                     __syncwarp();
                     const uint64_t vb = kv_desc + ((vslot * kFp4Slot) >> 4);
                     for (int i = 0; i < 2 && ok; ++i) {
-                        if (active(i, j)) {
-                            const int lo_i = i == 0 ? lo0 : lo1;
-                            const int hi_i = i == 0 ? hi0 : hi1;
-                            const uint32_t par = (uint32_t)(j - lo_i) & 1u;
-                            const uint32_t o_tmem = tmem + kColO + i * kOStride;
-                            const uint64_t pa = p_desc + ((i * kFp4Tile) >> 4);
-                            // Keys [0, 64) as soon as their codes are in shared memory.
-                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_half[i], par, abort_flag,
-                                                                      p.status, true, p.timeout_ns));
+                        const int lo_i = i == 0 ? lo0 : lo1;
+                        const int hi_i = i == 0 ? hi0 : hi1;
+                        const bool act = i == 0 ? (has0 && j >= lo0 && j <= hi0)
+                                                : (has1 && j >= lo1 && j <= hi1);
+                        if (!act) continue;
+                        const uint32_t par = (uint32_t)(j - lo_i) & 1u;
+                        const uint32_t o_tmem = tmem + kColO + i * kOStride;
+                        const uint64_t pa = p_desc + ((i * kFp4Tile) >> 4);
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {
+                            ok = __all_sync(0xffffffffu, wait_bounded(ks == 0 ? &sm.p_half[i] : &sm.p_full[i],
+                                                                      par, abort_flag, p.status, true,
+                                                                      p.timeout_ns));
                             if (!ok) break;
                             tc_fence_after();
                             if (leader) {
-                                tc_cp_sf(tmem + kColSfP + 4 * (2 * i), smem_desc_sf_atom(smem_u32(sm.psf[i][0])));
-                                mma_mxf4(o_tmem, pa, vb, kIdescPV, tmem + kColSfP + 4 * (2 * i),
-                                         tmem + kColSfV + 8 * (2 * (j & 1)), j > lo_i ? 1u : 0u);
-                            }
-                            __syncwarp();
-                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_full[i], par, abort_flag,
-                                                                      p.status, true, p.timeout_ns));
-                            if (!ok) break;
-                            tc_fence_after();
-                            if (leader) {
-                                tc_cp_sf(tmem + kColSfP + 4 * (2 * i + 1),
-                                         smem_desc_sf_atom(smem_u32(sm.psf[i][1])));
-                                mma_mxf4(o_tmem, pa + 2, vb + 2, kIdescPV, tmem + kColSfP + 4 * (2 * i + 1),
-                                         tmem + kColSfV + 8 * (2 * (j & 1) + 1), 1u);
-                                if (j == hi_i) tc_commit(&sm.o_final[i]);
+                                tc_cp_sf(tmem + kColSfP + 4 * (2 * i + ks),
+                                         smem_desc_sf_atom(smem_u32(sm.psf[i][ks])));
+                                mma_mxf4(o_tmem, pa + 2 * ks, vb + 2 * ks, kIdescPV,
+                                         tmem + kColSfP + 4 * (2 * i + ks),
+                                         tmem + kColSfV + 8 * (2 * (j & 1) + ks),
+                                         (ks > 0 || j > lo_i) ? 1u : 0u);
                             }
                             __syncwarp();
                         }
-                        if (j + 1 <= uhi && active(i, j + 1)) issue_s(i, j + 1);
+                        if (!ok) break;
+                        if (leader) {
+                            tc_commit(&sm.pv_done[i]);
+                            if (j == hi_i) tc_commit(&sm.o_final[i]);
+                        }
+                        __syncwarp();
                     }
                     if (!ok) break;
-                    if (j + 1 <= uhi && k_ready < j + 1) wait_k(j + 1);
-                    if (!ok) break;
-                    if (leader) {
-                        tc_commit(&sm.kv_empty[vslot]);
-                        if (j + 1 <= uhi) tc_commit(&sm.kv_empty[ring_pos(j + 1, 0) % NS]);
-                    }
+                    if (leader) tc_commit(&sm.kv_empty[vslot]);
                     __syncwarp();
                 }
                 if (!ok) {
-                    // Let every product and copy already issued finish before TMEM is freed.
-                    if (leader) tc_commit(&sm.drain);
+                    if (leader) tc_commit(&sm.drain_pv);
                     __syncwarp();
-                    wait_bounded(&sm.drain, 0, abort_flag, p.status, false, p.timeout_ns);
+                    wait_bounded(&sm.drain_pv, 0, abort_flag, p.status, false, p.timeout_ns);
                 }
             }
             __syncwarp();
         }
-        // warps 10-11: idle
+        // warp 11: idle
     } else {
         // ------------------------------------- softmax / correction / epilogue
         setmaxnreg_inc<kSoftmaxRegs>();
@@ -452,10 +463,12 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
 
         for (int j = lo_b; j <= hi_b; ++j) {
             const int t = j - lo_b;
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 0);
             ok = wait_bounded(&sm.s_full[i], (uint32_t)t & 1u, abort_flag, p.status, true, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 1);
 
             uint32_t sr[kBlockN];
             tmem_ld32(s_tmem + 0, sr + 0);
@@ -470,6 +483,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
             // The S region is free for the other tile's next product.
             tc_fence_before();
             mbar_arrive(&sm.s_free);
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 2);
             float *s = reinterpret_cast<float *>(sr);
 
             const int key0 = j * kBlockN;
@@ -493,10 +507,21 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                 m_run = m_new;
             }
             const float neg_m = m_run == -INFINITY ? 0.0f : p.p_offset - m_run;
+            if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 3);
 
-            // Correction (of O and of its sum column): P_i V(j-1) is complete
-            // (S of this block was committed after it), P_i V(j) is not yet
-            // issued.
+            // Codes of keys [0, 64) in registers, then wait until P_i V(j-1)
+            // has completed: only then may O_i be rescaled (the correction,
+            // rare once the maximum settles; it covers the sum column too)
+            // and P_i and its scales be overwritten.
+            uint4 codes[2];
+            uint32_t sf2;
+            direct_p_codes<CLS>(s, bm, c, neg_m, codes, sf2);
+            if (t > 0) {
+                ok = __all_sync(0xffffffffu, wait_bounded(&sm.pv_done[i], (uint32_t)(t - 1) & 1u,
+                                                          abort_flag, p.status, true, p.timeout_ns));
+                if (!ok) break;
+                tc_fence_after();
+            }
             if (t > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #ifdef ATTN_COUNT_RESCALES
                 ++cnt_warp;
@@ -529,9 +554,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
             // memory, made visible to the tensor cores, then signalled.
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                uint4 codes[2];
-                uint32_t sf2;
-                direct_p_codes<CLS>(s + 64 * half, bm + 2 * half, c, neg_m, codes, sf2);
+                if (half == 1) direct_p_codes<CLS>(s + 64, bm + 2, c, neg_m, codes, sf2);
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
                     *reinterpret_cast<uint4 *>(p_row + (((2 * half + u) ^ swz) << 4)) = codes[u];
@@ -539,6 +562,7 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(half == 0 ? &sm.p_half[i] : &sm.p_full[i]);
+                if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, t, 4 + half);
             }
         }
 
