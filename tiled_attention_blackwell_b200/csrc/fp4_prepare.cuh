@@ -47,8 +47,19 @@ __device__ __forceinline__ uint32_t nvfp4_scale(uint32_t sb, const uint8_t *code
     return 0u;
 }
 
+// 4 x 4 byte transpose: out[q] byte p = x[p] byte q.
+__device__ __forceinline__ void byte_transpose4(const uint32_t *x, uint32_t *out) {
+    const uint32_t t0 = __byte_perm(x[0], x[1], 0x5140), t1 = __byte_perm(x[0], x[1], 0x7362);
+    const uint32_t t2 = __byte_perm(x[2], x[3], 0x5140), t3 = __byte_perm(x[2], x[3], 0x7362);
+    out[0] = __byte_perm(t0, t2, 0x5410);
+    out[1] = __byte_perm(t0, t2, 0x7632);
+    out[2] = __byte_perm(t1, t3, 0x5410);
+    out[3] = __byte_perm(t1, t3, 0x7632);
+}
+
 __global__ void __launch_bounds__(256) fp4_prepare_kernel(const __grid_constant__ Fp4PrepParams p) {
-    __shared__ __align__(16) uint8_t tile[128][64];
+    constexpr int kRow = 68;  // padded row of the key tile (bytes): 2-way bank conflicts at most
+    __shared__ __align__(16) uint8_t tile[128 * kRow];
     __shared__ uint32_t us[4][128];
     bool bad = false;
     const int t = threadIdx.x;
@@ -65,38 +76,45 @@ __global__ void __launch_bounds__(256) fp4_prepare_kernel(const __grid_constant_
             if (kg < p.Sk)
                 v = *reinterpret_cast<const uint4 *>(
                     p.v_codes + (((size_t)b * p.Sk + kg) * p.Hkv + h) * 64 + c * 16);
-            *reinterpret_cast<uint4 *>(&tile[key][c * 16]) = v;
+            uint32_t *row = reinterpret_cast<uint32_t *>(tile + key * kRow + c * 16);
+            row[0] = v.x;
+            row[1] = v.y;
+            row[2] = v.z;
+            row[3] = v.w;
             const int sb = idx >> 7, d = idx & 127;
             const int blk = kt * 4 + sb;
             us[sb][d] = blk < nb32 ? p.v_scales[(((size_t)b * nb32 + blk) * p.Hkv + h) * 128 + d]
                                    : 127u;
         }
         __syncthreads();
-        // Row d of V^T, keys [64 half, 64 half + 64): 32 bytes.
-        const int d = t >> 1, half = t & 1;
-        const int sh = 4 * (d & 1);
-        uint32_t w[8];
+        // Thread: keys [8 kq, 8 kq + 8) x dims [8 dq, 8 dq + 8).  Input word x:
+        // dims 8 dq .. 8 dq + 7 of key 8 kq + x; per key pair a 2 x 2 nibble
+        // swap gives the even-dim and odd-dim bytes, then a 4 x 4 byte
+        // transpose gives output row d = 8 dq + e (keys 8 kq .. 8 kq + 7).
+        const int w = t >> 5, l = t & 31;
+        const int kq = 8 * (w & 1) + (l >> 2), dq = 4 * (w >> 1) + (l & 3);
+        uint32_t ev[4], od[4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int sb = 2 * half + (q >> 2);
-            const bool in_range = us[sb][d] - 114u <= 26u;
-            uint32_t word = 0u;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int key = 64 * half + 8 * q + e;
-                uint32_t nib = (tile[key][d >> 1] >> sh) & 15u;
-                if (!in_range) {
-                    bad |= (nib & 7u) != 0u;
-                    nib = 0u;
-                }
-                word |= nib << (4 * e);
-            }
-            w[q] = word;
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t A = *reinterpret_cast<const uint32_t *>(tile + (8 * kq + 2 * q) * kRow + 4 * dq);
+            const uint32_t B = *reinterpret_cast<const uint32_t *>(tile + (8 * kq + 2 * q + 1) * kRow + 4 * dq);
+            ev[q] = (A & 0x0F0F0F0Fu) | ((B & 0x0F0F0F0Fu) << 4);
+            od[q] = ((A >> 4) & 0x0F0F0F0Fu) | (B & 0xF0F0F0F0u);
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(
-            p.vt + (((size_t)b * p.Hkv + h) * 128 + d) * ((size_t)p.nkt * 64) + kt * 64 + half * 32);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        uint32_t evt[4], odt[4];
+        byte_transpose4(ev, evt);
+        byte_transpose4(od, odt);
+        const int sb = kq >> 2;  // the 32-key block of these 8 keys
+        uint8_t *vrow = p.vt + (((size_t)b * p.Hkv + h) * 128 + 8 * dq) * ((size_t)p.nkt * 64) + kt * 64 + 4 * kq;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            uint32_t word = (e & 1) ? odt[e >> 1] : evt[e >> 1];
+            if (us[sb][8 * dq + e] - 114u > 26u) {  // scale out of range: the codes read as 0
+                bad |= (word & 0x77777777u) != 0u;
+                word = 0u;
+            }
+            *reinterpret_cast<uint32_t *>(vrow + (size_t)e * p.nkt * 64) = word;
+        }
         if (t < 128) {
             uint8_t *atom = p.sf_v + (((size_t)b * p.Hkv + h) * p.nkt + kt) * (2 * kSfAtom);
 #pragma unroll
