@@ -94,6 +94,12 @@ WORKLOADS = {
     # MXFP4 V), for the Direct-P forward.
     "causal_s8192_fp4": Workload("causal_s8192_fp4", 2, 16, 16, 8192, 128, True, seed=3,
                                  dtype="fp4"),
+    # The shape of the FP4 page's peak Direct-P figure ("Hardware-Aware FP4
+    # FlashAttention-4", "Rendimiento de Inferencia Forward": S32768/H24,
+    # D = 128, inference, so no mask), in FP4 and in bf16 for the ratio.
+    "full_s32768_h24_fp4": Workload("full_s32768_h24_fp4", 1, 24, 24, 32768, 128, False, seed=8,
+                                    dtype="fp4"),
+    "full_s32768_h24": Workload("full_s32768_h24", 1, 24, 24, 32768, 128, False, seed=8),
 }
 
 HEADLINE = "causal_s8192"
