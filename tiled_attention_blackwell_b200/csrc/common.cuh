@@ -71,14 +71,15 @@ __device__ __forceinline__ KeyRange tile_key_range(const Params &p, int r0, int 
 
 // Bounded wait.  Returns false when the CTA is aborting (own timeout or
 // another role's); `honor_abort` = false keeps waiting until the timeout only.
+template <bool kHint = false>
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
                                              volatile int *abort_flag, int *status,
                                              bool honor_abort = true,
                                              uint64_t timeout_ns = kWaitTimeoutNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<kHint>(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait<kHint>(bar, parity)) return true;
         if ((n & 15u) == 0u) {
             if (honor_abort && *abort_flag) return false;
             if (globaltimer_ns() - t0 > timeout_ns) {

@@ -177,7 +177,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
         const uint32_t slot = n & 1u;
         FwdItem it;
         it.lin = -2;
-        if (!__all_sync(0xffffffffu, wait_bounded(&sm.item_full[slot], (n >> 1) & 1u, abort_flag,
+        if (!__all_sync(0xffffffffu, wait_bounded<true>(&sm.item_full[slot], (n >> 1) & 1u, abort_flag,
                                                   p.status, true, p.timeout_ns)))
             return it;
         const volatile FwdItem &src = sm.item[slot];
@@ -238,7 +238,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                 const uint32_t slot = n & 1u;
                 if (n >= 2)
                     ok = __all_sync(0xffffffffu,
-                                    wait_bounded(&sm.item_empty[slot], ((n >> 1) - 1u) & 1u,
+                                    wait_bounded<true>(&sm.item_empty[slot], ((n >> 1) - 1u) & 1u,
                                                  abort_flag, p.status, true, p.timeout_ns));
                 if (!ok) return;
                 if (lane == 0) {
@@ -271,7 +271,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                     const int hkv = ic.hq / p.group;
                     if (lane == 0) {
                         if (q_loads > 0)
-                            ok = wait_bounded(&sm.q_free, (q_loads - 1u) & 1u, abort_flag, p.status,
+                            ok = wait_bounded<true>(&sm.q_free, (q_loads - 1u) & 1u, abort_flag, p.status,
                                               true, p.timeout_ns);
                         if (ok) {
                             mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
@@ -284,7 +284,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                             const int key0 = (ulo + t) * kBlockN;
                             for (int which = 0; which < 2 && ok; ++which, ++it) {
                                 const uint32_t kslot = it % NS;
-                                ok = wait_bounded(&sm.kv_empty[kslot], ((it / NS) & 1u) ^ 1u,
+                                ok = wait_bounded<true>(&sm.kv_empty[kslot], ((it / NS) & 1u) ^ 1u,
                                                   abort_flag, p.status, true, p.timeout_ns);
                                 if (!ok) break;
                                 // Testing only: the first CTA withholds its first K copy
@@ -309,11 +309,11 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
             // normal path they have been consumed already).
             if (lane == 0) {
                 if (q_loads > 0)
-                    wait_bounded(&sm.q_full, (q_loads - 1u) & 1u, abort_flag, p.status, false,
+                    wait_bounded<true>(&sm.q_full, (q_loads - 1u) & 1u, abort_flag, p.status, false,
                                  p.timeout_ns);
                 const uint32_t first = it > NS ? it - NS : 0;
                 for (uint32_t L = first; L < it; ++L)
-                    wait_bounded(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status, false,
+                    wait_bounded<true>(&sm.kv_full[L % NS], (L / NS) & 1u, abort_flag, p.status, false,
                                  p.timeout_ns);
             }
             __syncwarp();
@@ -356,7 +356,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                 if (!has0 && !has1) continue;
                 const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : lo1;
                 const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : hi1;
-                ok = __all_sync(0xffffffffu, wait_bounded(&sm.q_full, q_items & 1u, abort_flag,
+                ok = __all_sync(0xffffffffu, wait_bounded<true>(&sm.q_full, q_items & 1u, abort_flag,
                                                           p.status, true, p.timeout_ns));
                 if (!ok) break;
                 tc_fence_after();
@@ -367,7 +367,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                 auto wait_k = [&](int j) {
                     const uint32_t L = ring_pos(j, 0);
                     if (ok)
-                        ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[L % NS],
+                        ok = __all_sync(0xffffffffu, wait_bounded<true>(&sm.kv_full[L % NS],
                                                                   (L / NS) & 1u, abort_flag,
                                                                   p.status, true, p.timeout_ns));
                     tc_fence_after();
@@ -405,10 +405,10 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                 // tile's previous item must have read it.  (The first QK^T
                 // products above write S only, so they do not wait for this.)
                 if (ok && has0 && o_items0 > 0)
-                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.o_free[0], (o_items0 - 1u) & 1u,
+                    ok = __all_sync(0xffffffffu, wait_bounded<true>(&sm.o_free[0], (o_items0 - 1u) & 1u,
                                                               abort_flag, p.status, true, p.timeout_ns));
                 if (ok && has1 && o_items1 > 0)
-                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.o_free[1], (o_items1 - 1u) & 1u,
+                    ok = __all_sync(0xffffffffu, wait_bounded<true>(&sm.o_free[1], (o_items1 - 1u) & 1u,
                                                               abort_flag, p.status, true, p.timeout_ns));
                 tc_fence_after();
 
@@ -416,7 +416,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                     const uint32_t Lv = ring_pos(j, 1);
                     const uint32_t vslot = Lv % NS;
                     ATTN_TRACE_EVENT(2, blocks_done0 + (uint32_t)(j - ulo), 0);
-                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.kv_full[vslot], (Lv / NS) & 1u,
+                    ok = __all_sync(0xffffffffu, wait_bounded<true>(&sm.kv_full[vslot], (Lv / NS) & 1u,
                                                               abort_flag, p.status, true, p.timeout_ns));
                     ATTN_TRACE_EVENT(2, blocks_done0 + (uint32_t)(j - ulo), 1);
                     if (!ok) break;
@@ -435,7 +435,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                             // V chunk: key rows of 128 bytes, 8-row groups 1024 B apart
                             // (SBO), 64-column chunks kChunkBytes apart (LBO).
                             ATTN_TRACE_EVENT(2, blocks_done0 + (uint32_t)(j - ulo), 2 + 3 * i);
-                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_half[i], par,
+                            ok = __all_sync(0xffffffffu, wait_bounded<true>(&sm.p_half[i], par,
                                                                       abort_flag, p.status, true, p.timeout_ns));
                             if (!ok) break;
                             tc_fence_after();
@@ -447,7 +447,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                                                   ks > 0 ? 1u : first);
                             }
                             __syncwarp();
-                            ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_full[i], par,
+                            ok = __all_sync(0xffffffffu, wait_bounded<true>(&sm.p_full[i], par,
                                                                       abort_flag, p.status, true, p.timeout_ns));
                             ATTN_TRACE_EVENT(2, blocks_done0 + (uint32_t)(j - ulo), 3 + 3 * i);
                             if (!ok) break;
@@ -490,7 +490,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                 // Let every MMA already issued finish before TMEM is freed.
                 if (leader) tc_commit(&sm.drain);
                 __syncwarp();
-                wait_bounded(&sm.drain, 0, abort_flag, p.status, false, p.timeout_ns);
+                wait_bounded<true>(&sm.drain, 0, abort_flag, p.status, false, p.timeout_ns);
             }
             __syncwarp();
         }
@@ -531,7 +531,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
                 const int t = j - lo_b;
                 const uint32_t tg = blocks_done + (uint32_t)t;  // running block count of the tile
                 if ((warp & 3) == 0) ATTN_TRACE_EVENT(i, tg, 0);
-                ok = wait_bounded(&sm.s_full[i], tg & 1u, abort_flag, p.status, true, p.timeout_ns);
+                ok = wait_bounded<true>(&sm.s_full[i], tg & 1u, abort_flag, p.status, true, p.timeout_ns);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 tc_fence_after();
@@ -704,7 +704,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ FwdParams p) {
             const bool has_blocks = lo_b <= hi_b;
             if (has_blocks) {
                 // The last PV of this tile (and every MMA before it) is complete.
-                ok = wait_bounded(&sm.o_final[i], o_items & 1u, abort_flag, p.status, true,
+                ok = wait_bounded<true>(&sm.o_final[i], o_items & 1u, abort_flag, p.status, true,
                                   p.timeout_ns);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;

@@ -62,16 +62,30 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 
 // Test a phase; a waiting thread may be suspended (not spinning, so not
 // taking issue slots from the warps that work) until the phase completes or
-// the hinted time (ns) elapses.
+// a time limit elapses: the hardware's own limit, or with kHint 20 us.
+// Measured on B200: without the hint the forward, backward and FP4 kernels
+// run 0.4-1.9 % faster; the persistent kernel keeps the hint (1.2 % faster
+// with it).
+template <bool kHint = false>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
-        : "memory");
+    if constexpr (kHint) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+    }
     return ok != 0;
 }
 
