@@ -185,7 +185,6 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
 
     // ------------------------------------------------------------ prologue
     if (threadIdx.x == 0) {
-        mbar_init(&sm.q_full, 1);
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
@@ -216,6 +215,22 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
         reinterpret_cast<uint32_t *>(sm.ones_sf)[x] = 0x00007F7Fu;
     fence_proxy_async_smem();
     if (warp == 9) {
+        if (lane == 0) {
+            // The Q copy needs nothing computed below, so it starts first and
+            // its latency overlaps the rest of the prologue.
+            mbar_init(&sm.q_full, 1);
+            fence_mbar_init();
+            prefetch_tensormap(&p.tm_q);
+            prefetch_tensormap(&p.tm_k);
+            prefetch_tensormap(&p.tm_v);
+            mbar_arrive_expect_tx(&sm.q_full, 2 * kFp4Tile + 4 * kSfAtom);
+            for (int i = 0; i < 2; ++i)
+                tma_load_4d(sm.q[i], &p.tm_q, &sm.q_full, 0, q0 + i * kBlockM, hq, b);
+            // Both tiles' scale atoms (tiles 2 qb and 2 qb + 1) are adjacent.
+            bulk_load(sm.qsf, p.sf_q + (((size_t)b * p.Hq + hq) * p.nq_tiles + 2 * qb) * (2 * kSfAtom),
+                      4 * kSfAtom, &sm.q_full);
+        }
+        __syncwarp();
         for (int i = 0; i < 2; ++i) {
             const int r0 = q0 + i * kBlockM;
             KeyRange kr{1, 0};
@@ -253,15 +268,6 @@ attn_fwd_fp4bs_kernel(const __grid_constant__ FwdParams p) {
         if (warp == 9) {
             // ------------------------------------------------------ TMA producer
             if (lane == 0) {
-                prefetch_tensormap(&p.tm_q);
-                prefetch_tensormap(&p.tm_k);
-                prefetch_tensormap(&p.tm_v);
-                mbar_arrive_expect_tx(&sm.q_full, 2 * kFp4Tile + 4 * kSfAtom);
-                for (int i = 0; i < 2; ++i)
-                    tma_load_4d(sm.q[i], &p.tm_q, &sm.q_full, 0, q0 + i * kBlockM, hq, b);
-                // Both tiles' scale atoms (tiles 2 qb and 2 qb + 1) are adjacent.
-                bulk_load(sm.qsf, p.sf_q + (((size_t)b * p.Hq + hq) * p.nq_tiles + 2 * qb) * (2 * kSfAtom),
-                          4 * kSfAtom, &sm.q_full);
                 uint32_t it = 0;
                 bool ok = true;
                 for (int t = 0; t < n_blocks && ok; ++t) {

@@ -386,8 +386,8 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
     const int q0 = qb * 2 * kBlockM;
 
     // ------------------------------------------------------------ prologue
+    constexpr uint32_t kTileBytes = kBlockM * D * EB;
     if (threadIdx.x == 0) {
-        mbar_init(&sm.q_full, 1);
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
@@ -403,6 +403,21 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         fence_mbar_init();
     }
     if (warp == 9) {
+        if (lane == 0) {
+            // The Q copy needs nothing computed below, so it starts first and
+            // its latency overlaps the rest of the prologue.
+            mbar_init(&sm.q_full, 1);
+            fence_mbar_init();
+            prefetch_tensormap(&p.tm_q);
+            prefetch_tensormap(&p.tm_k);
+            prefetch_tensormap(&p.tm_v);
+            mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
+            for (int i = 0; i < 2; ++i)
+                for (int c = 0; c < Smem::kChunks; ++c)
+                    tma_load_4d(sm.q[i][c], &p.tm_q, &sm.q_full, c * Smem::kChunkElems,
+                                q0 + i * kBlockM, hq, b);
+        }
+        __syncwarp();
         // Key-block range of each query tile: union of its rows' key ranges.
         for (int i = 0; i < 2; ++i) {
             const int r0 = q0 + i * kBlockM;
@@ -435,7 +450,6 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
     const int ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : lo1;
     const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : hi1;
     const int n_blocks = (has0 || has1) ? (uhi - ulo + 1) : 0;
-    constexpr uint32_t kTileBytes = kBlockM * D * EB;
 
     // Registers: the softmax warpgroups hold a 128-column score row per
     // thread; the MMA / TMA warpgroup needs few.  384 x 168 at launch =
@@ -447,14 +461,6 @@ attn_fwd_kernel(const __grid_constant__ FwdParams p) {
         if (warp == 9) {
             // ------------------------------------------------------ TMA producer
             if (lane == 0) {
-                prefetch_tensormap(&p.tm_q);
-                prefetch_tensormap(&p.tm_k);
-                prefetch_tensormap(&p.tm_v);
-                mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
-                for (int i = 0; i < 2; ++i)
-                    for (int c = 0; c < Smem::kChunks; ++c)
-                        tma_load_4d(sm.q[i][c], &p.tm_q, &sm.q_full, c * Smem::kChunkElems,
-                                    q0 + i * kBlockM, hq, b);
                 uint32_t it = 0;
                 bool ok = true;
                 for (int t = 0; t < n_blocks && ok; ++t) {
